@@ -1,0 +1,280 @@
+"""Plain fp64 NumPy statement of what the fused norm+projection computes.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring): never called by the
+library, shares no code with the CUDA path.
+
+Sources.  The method is described on the FlashNorm talk summary ("RMS norm는
+연산량 1할인데 왜 33번 호출로 속도를 갉아먹나", news.juniverse.app): Proposal 1
+("웨이트리스 정규화", weightless normalisation) folds the norm gain into the
+following projection offline; Proposal 2 ("지연된 정규화", deferred
+normalisation) postpones the per-row 1/rms scalar until after the matmul;
+Proposal 3 ("이중 정규화 제거") removes a back-to-back norm by scale invariance.
+The SwiGLU epilogue (silu(gate) * up) is the activation of the fused FC1 on the
+FlashInfer PR #5521 analysis ("Segmented Chain" baseline and "Register-level
+SwiGLU" design item).  The pages print no formula; the readings used here are:
+
+    ms[m]  = (1/d) * sum_k x[m,k]^2              mean over the full row (divisor d)
+    r[m]   = 1 / sqrt(ms[m] + eps)               eps inside the square root
+    h[m,k] = x[m,k] * r[m] * g[k]                normalised row times the gain
+    y      = h @ W                               no bias
+    silu(z) = z / (1 + exp(-z))
+    swiglu  = silu(h @ W_gate) * (h @ W_up)
+
+The oracle computes these the *unfolded* way: normalise first, then multiply.
+All stored low-precision inputs are taken exactly as float64.
+
+The fold (Proposal 1) and the fp8 block quantisation are encodings, so the
+oracle spells out their rounding steps from the formats' definitions:
+
+    W'      = RN_bf16( fp32(g[k]) * fp32(W[k,n]) )        one fp32 product, one RN
+    fp8:    P = fp32(g[k]) * fp32(W[k,n]);  per 128x128 block b:
+            s_b = fp32( amax_b(|P|) / 448 )  (s_b = 1 when amax_b = 0)
+            q   = RN_e4m3_satfinite( fp32(P / s_b) )
+    SwiGLU storage: 128-column tiles of the gate and up halves alternate,
+            W'_cat[:, 256j : 256j+128]       = W'_gate[:, 128j : 128j+128]
+            W'_cat[:, 256j+128 : 256j+256]   = W'_up  [:, 128j : 128j+128]
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Tuple
+
+import numpy as np
+
+__all__ = [
+    "BF16", "E4M3", "round_to_format", "bf16_round", "bf16_bits", "bf16_from_bits",
+    "e4m3_round", "e4m3_encode", "e4m3_decode", "to_f64",
+    "rms_inv", "rmsnorm", "norm_proj", "silu", "norm_proj_swiglu",
+    "fold_bf16", "interleave128", "deinterleave128", "fold_fp8", "dequant_fp8",
+    "FP8_BLOCK", "E4M3_MAX",
+]
+
+FP8_BLOCK = 128
+E4M3_MAX = 448.0
+
+
+# ---------------------------------------------------------------------------
+# Number formats, from their definitions
+# ---------------------------------------------------------------------------
+class _Format:
+    """A binary floating-point format: stored mantissa bits, exponent bias,
+    largest finite value and what happens above it ("inf" or "sat")."""
+
+    def __init__(self, name, man_bits, exp_bits, bias, max_finite, overflow):
+        self.name = name
+        self.man_bits = man_bits
+        self.exp_bits = exp_bits
+        self.bias = bias
+        self.emin = 1 - bias                   # exponent of the smallest normal
+        self.max_finite = max_finite
+        self.overflow = overflow
+
+
+# bfloat16: 1 sign, 8 exponent (bias 127), 7 mantissa bits; IEEE-style inf.
+BF16 = _Format("bf16", 7, 8, 127, (2.0 - 2.0 ** -7) * 2.0 ** 127, "inf")
+# e4m3 ("fn" variant): 1 sign, 4 exponent (bias 7), 3 mantissa bits, no inf;
+# S.1111.111 is NaN, so the largest finite value is 1.75 * 2^8 = 448.
+# Conversions here saturate to +-448 (the "satfinite" rounding).
+E4M3 = _Format("e4m3", 3, 4, 7, 448.0, "sat")
+
+
+def round_to_format(v, fmt: _Format) -> np.ndarray:
+    """Round values to the nearest member of `fmt`, ties to even.
+
+    Works in float64, where every step below is exact: the quantum of the
+    binade holding |v| is a power of two, so |v| / quantum is exact and
+    np.rint rounds half to even.  Below the smallest normal the quantum is
+    fixed (subnormals).  Returns float64 values of the format.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))    # a = m * 2^ex, m in [0.5, 1)
+    e = np.maximum(ex.astype(np.int64) - 1, fmt.emin)   # floor(log2 a), clamped
+    quantum = np.ldexp(1.0, e - fmt.man_bits)
+    r = np.rint(a / quantum) * quantum
+    if fmt.overflow == "inf":
+        r = np.where(r > fmt.max_finite, np.inf, r)
+    else:
+        r = np.where(r > fmt.max_finite, fmt.max_finite, r)
+    r = np.where(np.isinf(a), np.inf if fmt.overflow == "inf" else fmt.max_finite, r)
+    out = np.copysign(r, v)
+    return np.where(np.isnan(v), np.nan, out)
+
+
+def bf16_round(v) -> np.ndarray:
+    return round_to_format(v, BF16)
+
+
+def bf16_bits(v) -> np.ndarray:
+    """uint16 bit patterns of RN_bf16(v).  A bf16 value is an fp32 value whose
+    low 16 bits are zero, so the pattern is the top half of its fp32 bits."""
+    r = bf16_round(v).astype(np.float32)
+    bits = (r.view(np.uint32) >> 16).astype(np.uint16)
+    return np.where(np.isnan(r), np.uint16(0x7FC0), bits).astype(np.uint16)
+
+
+def bf16_from_bits(bits) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def e4m3_round(v) -> np.ndarray:
+    return round_to_format(v, E4M3)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """uint8 codes of RN_e4m3_satfinite(v): sign | exponent field | mantissa."""
+    r = e4m3_round(v)
+    sign = (np.signbit(r)).astype(np.uint8) << 7
+    a = np.abs(r)
+    nan = np.isnan(a)
+    a = np.where(nan, 0.0, a)
+    min_normal = 2.0 ** E4M3.emin
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    e = ex.astype(np.int64) - 1
+    normal = a >= min_normal
+    exp_field = np.where(normal, e + E4M3.bias, 0)
+    mant = np.where(normal,
+                    np.ldexp(a, -e) - 1.0,                   # in [0, 1)
+                    a / min_normal)                          # subnormal: 0.mmm
+    mant_field = np.rint(mant * 8.0).astype(np.int64)
+    code = (exp_field.astype(np.int64) << 3) | mant_field
+    code = np.where(a == 0, 0, code).astype(np.uint8) | sign
+    return np.where(nan, np.uint8(0x7F), code).astype(np.uint8)
+
+
+def e4m3_decode(code) -> np.ndarray:
+    """float64 value of each uint8 e4m3 code (S.1111.111 decodes to NaN)."""
+    c = np.asarray(code, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    ef = (c >> 3) & 0xF
+    mf = c & 0x7
+    val = np.where(ef == 0,
+                   np.ldexp(mf / 8.0, E4M3.emin),
+                   np.ldexp(1.0 + mf / 8.0, ef - E4M3.bias))
+    val = np.where((ef == 0xF) & (mf == 0x7), np.nan, val)
+    return s * val
+
+
+def to_f64(a) -> np.ndarray:
+    """Stored values (NumPy array or a CPU torch tensor of any float dtype) as
+    float64, exactly."""
+    if hasattr(a, "detach"):
+        a = a.detach().cpu()
+        if str(a.dtype) in ("torch.bfloat16", "torch.float16"):
+            a = a.float()
+        a = a.double().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# The operation (FlashNorm talk: RMSNorm feeding its projection; unfolded form)
+# ---------------------------------------------------------------------------
+def rms_inv(x, eps: float) -> np.ndarray:
+    """r[m] = 1 / sqrt(mean_k x[m,k]^2 + eps); the per-row scalar that
+    Proposal 2 (deferred normalisation) postpones to after the matmul."""
+    x = to_f64(x)
+    ms = np.mean(x * x, axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return 1.0 / np.sqrt(ms + eps)
+
+
+def rmsnorm(x, g, eps: float) -> np.ndarray:
+    """h = (x * r) * g, the normalised activation an unfused chain writes."""
+    x = to_f64(x)
+    g = to_f64(g)
+    with np.errstate(invalid="ignore"):
+        return (x * rms_inv(x, eps)[:, None]) * g[None, :]
+
+
+def _matmul_chunked(h: np.ndarray, W, col_chunk: Optional[int]) -> np.ndarray:
+    W_is_np = isinstance(W, np.ndarray)
+    ncols = W.shape[1]
+    if col_chunk is None or col_chunk >= ncols:
+        return h @ to_f64(W)
+    out = np.empty((h.shape[0], ncols), dtype=np.float64)
+    for c0 in range(0, ncols, col_chunk):
+        c1 = min(ncols, c0 + col_chunk)
+        out[:, c0:c1] = h @ to_f64(W[:, c0:c1] if W_is_np else W[:, c0:c1])
+    return out
+
+
+def norm_proj(x, g, W, eps: float, col_chunk: Optional[int] = None) -> np.ndarray:
+    """y = RMSNorm(x; g, eps) @ W in float64, normalising first (unfolded)."""
+    h = rmsnorm(x, g, eps)
+    with np.errstate(invalid="ignore"):
+        return _matmul_chunked(h, W, col_chunk)
+
+
+def silu(z) -> np.ndarray:
+    """silu(z) = z / (1 + exp(-z)); exp overflow for z << 0 gives -0."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def norm_proj_swiglu(x, g, W_gate, W_up, eps: float,
+                     col_chunk: Optional[int] = None) -> np.ndarray:
+    """silu(h @ W_gate) * (h @ W_up) with h = RMSNorm(x; g, eps)."""
+    h = rmsnorm(x, g, eps)
+    with np.errstate(invalid="ignore"):
+        return silu(_matmul_chunked(h, W_gate, col_chunk)) * _matmul_chunked(h, W_up, col_chunk)
+
+
+# ---------------------------------------------------------------------------
+# The offline fold (Proposal 1) and the weight encodings
+# ---------------------------------------------------------------------------
+def _gain_product_f32(W, g) -> np.ndarray:
+    """fp32(g[k]) * fp32(W[k,n]) as an fp32 array (IEEE round-to-nearest)."""
+    Wf = to_f64(W).astype(np.float32)
+    gf = to_f64(g).astype(np.float32)
+    return gf[:, None] * Wf
+
+
+def fold_bf16(W, g) -> np.ndarray:
+    """bf16 bit patterns [d, N] of W' = RN_bf16(fp32(g) * fp32(W))."""
+    return bf16_bits(_gain_product_f32(W, g).astype(np.float64))
+
+
+def interleave128(A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """[d, 2N] with 128-column tiles alternating A, B, A, B, ..."""
+    d, N = A.shape
+    assert B.shape == (d, N) and N % 128 == 0
+    out = np.empty((d, 2 * N), dtype=A.dtype)
+    for j in range(N // 128):
+        out[:, 256 * j: 256 * j + 128] = A[:, 128 * j: 128 * j + 128]
+        out[:, 256 * j + 128: 256 * j + 256] = B[:, 128 * j: 128 * j + 128]
+    return out
+
+
+def deinterleave128(C: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    d, N2 = C.shape
+    N = N2 // 2
+    A = np.empty((d, N), dtype=C.dtype)
+    B = np.empty((d, N), dtype=C.dtype)
+    for j in range(N // 128):
+        A[:, 128 * j: 128 * j + 128] = C[:, 256 * j: 256 * j + 128]
+        B[:, 128 * j: 128 * j + 128] = C[:, 256 * j + 128: 256 * j + 256]
+    return A, B
+
+
+def fold_fp8(W, g) -> Tuple[np.ndarray, np.ndarray]:
+    """e4m3 codes [d, N] and fp32 block scales [d/128, N/128] of the folded
+    weight: s_b = fp32(amax_b / 448) (1 for an all-zero block) and
+    q = RN_e4m3_satfinite(fp32(P / s_b)), P = fp32(g) * fp32(W)."""
+    P = _gain_product_f32(W, g)
+    d, N = P.shape
+    assert d % FP8_BLOCK == 0 and N % FP8_BLOCK == 0
+    bd, bn = d // FP8_BLOCK, N // FP8_BLOCK
+    blocks = np.abs(P).reshape(bd, FP8_BLOCK, bn, FP8_BLOCK)
+    amax = blocks.max(axis=(1, 3)).astype(np.float32)
+    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    s_full = np.repeat(np.repeat(s, FP8_BLOCK, axis=0), FP8_BLOCK, axis=1)
+    quot = (P / s_full).astype(np.float32)          # fp32 IEEE division
+    return e4m3_encode(quot.astype(np.float64)), s
+
+
+def dequant_fp8(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """float64 W_deq[k,n] = e4m3(q[k,n]) * s[k/128, n/128] (exact in fp64)."""
+    s_full = np.repeat(np.repeat(to_f64(s), FP8_BLOCK, axis=0), FP8_BLOCK, axis=1)
+    return e4m3_decode(q) * s_full
