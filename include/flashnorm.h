@@ -1,0 +1,161 @@
+/*
+ * flashnorm.h — C ABI of the B200 (sm_100a) fused RMSNorm + linear projection
+ * in the FlashNorm form.
+ *
+ * The method (FlashNorm talk summary, "RMS norm는 연산량 1할인데 왜 33번 호출로
+ * 속도를 갉아먹나", news.juniverse.app):
+ *   Proposal 1 ("웨이트리스 정규화", weightless normalisation): fold the norm
+ *     gain into the projection offline, W' = diag(g) W.
+ *   Proposal 2 ("지연된 정규화", deferred normalisation): run the matmul on the
+ *     raw activations on the tensor cores, reduce each row's sum of squares on
+ *     the vector units at the same time, then post-scale by 1/rms(x).
+ *   Bug/cause/fix bullets: the post-scale must wait explicitly for both the
+ *     matmul and the reduction.
+ * SwiGLU epilogue: the fused FC1 + SwiGLU of the FlashInfer PR #5521 analysis
+ * ("Register-level SwiGLU" design item): out = silu(gate) * up.
+ *
+ * Definitions (the pages print no formula; these are the plain readings):
+ *   r[m]  = 1 / sqrt( (1/d) sum_k x[m,k]^2 + eps )
+ *   y     = r[m] * sum_k x[m,k] W'[k,n]              (= RMSNorm(x; g) @ W)
+ *   swiglu: out[m,n] = silu(r[m] * (x W'_gate)[m,n]) * (r[m] * (x W'_up)[m,n]),
+ *           silu(z) = z / (1 + e^-z)
+ * fp32 accumulation, one round-to-nearest-even to bf16 at the store.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, owned and allocated by the
+ *     caller; the library never allocates, frees or synchronises in the
+ *     compute calls.  Tensors are dense row-major.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Argument errors are returned synchronously, before any launch.
+ *     A failed launch returns FN_ERR_CUDA.  A device-side wait that ran out of
+ *     time is reported later by fn_query_device_status.
+ *   - Base pointers must be 16-byte aligned (TMA); FN_ERR_ALIGNMENT otherwise.
+ *   - No exception crosses the ABI; the functions are re-entrant.  Calls that
+ *     may overlap on the GPU need distinct workspaces.
+ */
+#ifndef FLASHNORM_H_
+#define FLASHNORM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without including the CUDA headers */
+typedef struct CUstream_st* fn_stream_t;
+
+typedef enum {
+  FN_OK = 0,
+  FN_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad eps or enum */
+  FN_ERR_UNSUPPORTED_SHAPE = 2,  /* d % 64, N % 128, fp8 d % 128, sizes over int32 */
+  FN_ERR_ALIGNMENT = 3,          /* a base pointer not 16-byte aligned */
+  FN_ERR_ALIAS = 4,              /* the output overlaps an input or the workspace */
+  FN_ERR_WORKSPACE = 5,          /* workspace missing or smaller than fn_workspace_size */
+  FN_ERR_CUDA = 6,               /* a CUDA runtime/driver call failed */
+  FN_ERR_TIMEOUT = 7,            /* a device-side wait exceeded its time budget */
+  FN_ERR_UNSUPPORTED_DEVICE = 8  /* not a compute capability 10.0 (B200-class) GPU */
+} fn_status;
+
+typedef enum {
+  FN_W_BF16 = 0,            /* W' stored as bf16 [d, ncols] */
+  FN_W_FP8_E4M3_B128 = 1    /* W' stored as e4m3 [d, ncols] + fp32 scales [d/128, ncols/128] */
+} fn_wtype;
+
+/*
+ * fn_fold_weights — offline fold (Proposal 1, weightless normalisation).
+ *   W0      bf16 [d, N]: the projection weight (the gate half for SwiGLU)
+ *   W1      bf16 [d, N]: the up half for SwiGLU, or NULL for a plain projection
+ *   g       fp32 [d]: the norm gain, as the effective multiplier (a (1+w) style
+ *           gain is the caller's conversion)
+ *   out_type FN_W_BF16: Wp = bf16 [d, ncols], Wp[k,n] = RN_bf16(fp32 g[k] * W[k,n])
+ *           FN_W_FP8_E4M3_B128: Wp = e4m3 bytes [d, ncols] and scales fp32
+ *           [d/128, ncols/128]: per 128x128 block s = amax|g*W| / 448 (1 if the
+ *           block is all zero), Wp = RN_e4m3_satfinite(fp32(g*W) / s); needs
+ *           d % 128 == 0.
+ *   ncols = N, or 2N with W1: then 128-column tiles alternate gate, up, gate,
+ *           up (stored columns [256j, 256j+128) = gate columns [128j, 128j+128),
+ *           [256j+128, 256j+256) = the same up columns).
+ *   Shapes: d >= 1, d % 64 == 0 (128 for fp8), N % 128 == 0.
+ *   Wp must not overlap W0, W1 or g (FN_ERR_ALIAS).
+ */
+fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_t d, int64_t N,
+                          fn_wtype out_type, void* Wp, float* scales, fn_stream_t stream);
+
+/*
+ * fn_workspace_size — bytes of workspace a call with these sizes needs.
+ * The workspace holds a 256-byte header (the device status word) and, for
+ * M <= 64, the stream-K partial sums and tile counters.  It must be
+ * zero-filled once before its first use; every call leaves it ready for the
+ * next one (after FN_ERR_TIMEOUT, zero it again).  Depends on the SM count of
+ * the current device (148 is assumed when no device is visible).
+ */
+size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swiglu);
+
+/*
+ * fn_norm_proj — y[M, N] = RMSNorm(x; g, eps) @ W, computed as
+ *   r[m] * (x @ W')[m, :] with W' from fn_fold_weights (Proposal 2).
+ *   x       bf16 [M, d] raw activations (never normalised in memory)
+ *   Wp      folded weight [d, N] of type wt (scales: fp32 [d/128, N/128] for fp8)
+ *   eps     >= 0 and finite, added to the mean inside the square root
+ *   y       bf16 [M, N] output; must not overlap x, Wp, scales or workspace
+ *   workspace, ws_bytes  >= fn_workspace_size(M, d, N, wt, 0), zeroed before first use
+ *   M == 0 is a no-op.  M <= 64 runs the split-K decode kernel, larger M the
+ *   tensor-core tile kernel; both are deterministic (repeated calls with the
+ *   same inputs give the same bits).
+ */
+fn_status fn_norm_proj(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
+                       int64_t N, float eps, void* y, void* workspace, size_t ws_bytes, fn_stream_t stream);
+
+/*
+ * fn_norm_proj_swiglu — out[M, N] = silu(h W_gate) * (h W_up), h = RMSNorm(x; g, eps),
+ * computed as silu(r * (x W'_gate)) * (r * (x W'_up)): r is applied to both halves
+ * before the nonlinearity.  Wp is the interleaved [d, 2N] fold of (W_gate, W_up);
+ * scales fp32 [d/128, 2N/128] for fp8.  Other arguments as fn_norm_proj, with
+ * workspace >= fn_workspace_size(M, d, N, wt, 1).
+ */
+fn_status fn_norm_proj_swiglu(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                              fn_wtype wt, int64_t N, float eps, void* out, void* workspace, size_t ws_bytes,
+                              fn_stream_t stream);
+
+/*
+ * fn_query_device_status — synchronises `stream`, reads and clears the status
+ * word in `workspace`.  Returns FN_OK or FN_ERR_TIMEOUT; *detail (if not NULL)
+ * receives the raw word (bits 8-15 name the wait site that gave up).
+ */
+fn_status fn_query_device_status(void* workspace, unsigned int* detail, fn_stream_t stream);
+
+/*
+ * Unfused-chain helpers, for baselines (FlashInfer PR #5521 analysis,
+ * "Segmented Chain" section: norm, then GEMM, then activation, each through HBM).
+ * fn_rmsnorm: h[M, d] = bf16((x * r) * g).  fn_dequant_fp8: W[d, ncols] =
+ * bf16(e4m3(q) * s).  Same conventions as above.
+ */
+fn_status fn_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, float eps, void* h,
+                     fn_stream_t stream);
+fn_status fn_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t ncols, void* W,
+                         fn_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* fn_status_string(fn_status s);
+
+/* ABI version of this library (increments on any signature change). */
+int fn_version(void);
+
+/*
+ * fn_set_debug — process-wide knobs for tests and diagnostics (not thread-safe;
+ * set them before issuing work):
+ *   FN_DEBUG_WAIT_BUDGET_NS   per-wait time limit inside the kernels (default 2e9)
+ *   FN_DEBUG_WITHHOLD_ARRIVE  1: the reducers withhold their first arrival, so the
+ *                             epilogue's wait must run out (exercises FN_ERR_TIMEOUT)
+ *   FN_DEBUG_FORCE_PATH       0 auto, 1 decode kernel (M <= 64 only), 2 tile kernel
+ */
+enum { FN_DEBUG_WAIT_BUDGET_NS = 1, FN_DEBUG_WITHHOLD_ARRIVE = 2, FN_DEBUG_FORCE_PATH = 3 };
+fn_status fn_set_debug(int key, int64_t value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHNORM_H_ */

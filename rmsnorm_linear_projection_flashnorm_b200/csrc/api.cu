@@ -1,0 +1,314 @@
+// C ABI layer: argument validation, dispatch, tensor-map encoding and the
+// device status word.  Declarations and contracts are in include/flashnorm.h.
+//
+// Dispatch ladder: M <= 64 runs the split-K decode kernel, larger M the
+// tensor-core tile kernel.  This mirrors the token-count ladder of the
+// FlashInfer PR #5668 analysis (K23_LADDER: run M on the smallest compiled
+// capacity that holds it, reject sizes out of range with an error, not an
+// exception); inside the decode kernel M is padded to 16, 32 or 64.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "flashnorm.h"
+#include "internal.h"
+
+namespace fn {
+
+namespace {
+std::atomic<long long> g_budget_ns{2000000000LL};
+std::atomic<int> g_withhold{0};
+std::atomic<int> g_force_path{0};
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];
+std::atomic<int> g_cc_major[kMaxDevices];
+
+bool device_info(int& dev, int& sms, int& cc_major) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return false;
+  }
+  sms = g_sms[dev].load(std::memory_order_relaxed);
+  cc_major = g_cc_major[dev].load(std::memory_order_relaxed);
+  if (sms <= 0) {
+    int s = 0, c = 0;
+    if (cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&c, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    g_sms[dev].store(s);
+    g_cc_major[dev].store(c);
+    sms = s;
+    cc_major = c;
+  }
+  return true;
+}
+
+int current_sms_or_default() {
+  int dev, sms, cc;
+  if (device_info(dev, sms, cc) && sms > 0) return sms;
+  return 148;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+bool eps_ok(float eps) { return std::isfinite(eps) && eps >= 0.0f; }
+
+constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
+}  // namespace
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows,
+                  uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  std::memset(map, 0, sizeof(*map));
+  const CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+fn_status check_device(int& sms) {
+  int dev, cc;
+  if (!device_info(dev, sms, cc)) return FN_ERR_CUDA;
+  if (cc != 10) return FN_ERR_UNSUPPORTED_DEVICE;
+  return FN_OK;
+}
+
+fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
+                           int64_t N, float eps, void* y, void* ws, size_t ws_bytes, fn_stream_t stream,
+                           bool swiglu) {
+  if (M < 0 || d <= 0 || N <= 0) return FN_ERR_INVALID_ARG;
+  if (wt != FN_W_BF16 && wt != FN_W_FP8_E4M3_B128) return FN_ERR_INVALID_ARG;
+  if (!eps_ok(eps)) return FN_ERR_INVALID_ARG;
+  if (d % 64 != 0 || N % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (wt == FN_W_FP8_E4M3_B128 && d % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
+  const int64_t ncols = swiglu ? 2 * N : N;
+  if (M > kMaxDim || d > kMaxDim || ncols > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return FN_OK;
+  if (!x || !Wp || !y) return FN_ERR_INVALID_ARG;
+  if (!ws) return FN_ERR_WORKSPACE;
+  if (wt == FN_W_FP8_E4M3_B128 && !scales) return FN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wp) || !aligned16(y) || !aligned16(ws)) return FN_ERR_ALIGNMENT;
+  if (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return FN_ERR_ALIGNMENT;
+
+  const size_t wbytes = static_cast<size_t>(d) * ncols * (wt == FN_W_BF16 ? 2 : 1);
+  const size_t xbytes = static_cast<size_t>(M) * d * 2;
+  const size_t ybytes = static_cast<size_t>(M) * N * 2;
+  const size_t sbytes = scales ? static_cast<size_t>(d / 128) * (ncols / 128) * 4 : 0;
+  if (overlaps(y, ybytes, x, xbytes) || overlaps(y, ybytes, Wp, wbytes) || overlaps(y, ybytes, scales, sbytes) ||
+      overlaps(y, ybytes, ws, ws_bytes) || overlaps(ws, ws_bytes, x, xbytes) || overlaps(ws, ws_bytes, Wp, wbytes))
+    return FN_ERR_ALIAS;
+
+  int force = g_force_path.load();
+  bool use_decode = M <= 64;
+  if (force == 1) {
+    if (M > 64) return FN_ERR_INVALID_ARG;
+    use_decode = true;
+  } else if (force == 2) {
+    use_decode = false;
+  }
+  if (wt == FN_W_FP8_E4M3_B128) return FN_ERR_UNSUPPORTED_SHAPE;  // fp8 kernels: not built yet
+
+  int sms = 0;
+  fn_status st = check_device(sms);
+  if (st != FN_OK) return st;
+  const size_t need = use_decode ? decode_workspace_bytes(M, d, ncols, swiglu, sms) : kWsHeaderBytes;
+  if (ws_bytes < need) return FN_ERR_WORKSPACE;
+
+  CallArgs a;
+  a.x = x;
+  a.M = M;
+  a.d = d;
+  a.Wp = Wp;
+  a.scales = scales;
+  a.wtype = static_cast<int>(wt);
+  a.N = N;
+  a.ncols = ncols;
+  a.swiglu = swiglu;
+  a.eps = eps;
+  a.y = y;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  a.num_sms = sms;
+  a.budget_ns = static_cast<uint64_t>(g_budget_ns.load());
+  a.withhold = g_withhold.load();
+  const cudaError_t e = use_decode ? launch_decode(a) : launch_tc(a);
+  return e == cudaSuccess ? FN_OK : FN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fn
+
+using namespace fn;
+
+extern "C" {
+
+fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, fn_wtype out_type,
+                          void* Wp, float* scales, fn_stream_t stream) {
+  if (d <= 0 || N <= 0) return FN_ERR_INVALID_ARG;
+  if (out_type != FN_W_BF16 && out_type != FN_W_FP8_E4M3_B128) return FN_ERR_INVALID_ARG;
+  if (!W0 || !g || !Wp) return FN_ERR_INVALID_ARG;
+  if (out_type == FN_W_FP8_E4M3_B128 && !scales) return FN_ERR_INVALID_ARG;
+  if (d % 64 != 0 || N % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (out_type == FN_W_FP8_E4M3_B128 && d % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
+  const int64_t ncols = W1 ? 2 * N : N;
+  if (d > kMaxDim || ncols > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W0) || (W1 && !aligned16(W1)) || !aligned16(Wp) || (reinterpret_cast<uintptr_t>(g) & 3u) ||
+      (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)))
+    return FN_ERR_ALIGNMENT;
+  const size_t in_bytes = static_cast<size_t>(d) * N * 2;
+  const size_t out_bytes = static_cast<size_t>(d) * ncols * (out_type == FN_W_BF16 ? 2 : 1);
+  const size_t s_bytes = scales ? static_cast<size_t>(d / 128) * (ncols / 128) * 4 : 0;
+  if (overlaps(Wp, out_bytes, W0, in_bytes) || overlaps(Wp, out_bytes, W1, in_bytes) ||
+      overlaps(Wp, out_bytes, g, static_cast<size_t>(d) * 4) || overlaps(scales, s_bytes, Wp, out_bytes) ||
+      overlaps(scales, s_bytes, W0, in_bytes) || overlaps(scales, s_bytes, W1, in_bytes))
+    return FN_ERR_ALIAS;
+  int sms = 0;
+  fn_status st = check_device(sms);
+  if (st != FN_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = out_type == FN_W_BF16 ? launch_fold_bf16(W0, W1, g, d, N, Wp, s)
+                                              : launch_fold_fp8(W0, W1, g, d, N, Wp, scales, s);
+  return e == cudaSuccess ? FN_OK : FN_ERR_CUDA;
+}
+
+size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swiglu) {
+  (void)wt;
+  if (M <= 0 || d <= 0 || N <= 0 || d % 64 != 0 || N % 128 != 0) return kWsHeaderBytes;
+  if (M > 64) return kWsHeaderBytes;
+  return decode_workspace_bytes(M, d, swiglu ? 2 * N : N, swiglu != 0, current_sms_or_default());
+}
+
+fn_status fn_norm_proj(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
+                       int64_t N, float eps, void* y, void* workspace, size_t ws_bytes, fn_stream_t stream) {
+  return norm_proj_common(x, M, d, Wp, scales, wt, N, eps, y, workspace, ws_bytes, stream, false);
+}
+
+fn_status fn_norm_proj_swiglu(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                              fn_wtype wt, int64_t N, float eps, void* out, void* workspace, size_t ws_bytes,
+                              fn_stream_t stream) {
+  return norm_proj_common(x, M, d, Wp, scales, wt, N, eps, out, workspace, ws_bytes, stream, true);
+}
+
+fn_status fn_query_device_status(void* workspace, unsigned int* detail, fn_stream_t stream) {
+  if (!workspace) return FN_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return FN_ERR_CUDA;
+  }
+  if (word != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+      cudaGetLastError();
+      return FN_ERR_CUDA;
+    }
+  }
+  if (detail) *detail = word;
+  if (word == 0) return FN_OK;
+  return (word & 0xFFu) == FN_ERR_TIMEOUT ? FN_ERR_TIMEOUT : FN_ERR_CUDA;
+}
+
+fn_status fn_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, float eps, void* h, fn_stream_t stream) {
+  if (M < 0 || d <= 0 || !eps_ok(eps)) return FN_ERR_INVALID_ARG;
+  if (d % 64 != 0 || M > kMaxDim || d > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return FN_OK;
+  if (!x || !g || !h) return FN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(h)) return FN_ERR_ALIGNMENT;
+  const size_t bytes = static_cast<size_t>(M) * d * 2;
+  if (overlaps(h, bytes, x, bytes) || overlaps(h, bytes, g, static_cast<size_t>(d) * 4)) return FN_ERR_ALIAS;
+  int sms = 0;
+  fn_status st = check_device(sms);
+  if (st != FN_OK) return st;
+  return launch_rmsnorm(x, M, d, g, eps, h, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FN_OK
+                                                                                                 : FN_ERR_CUDA;
+}
+
+fn_status fn_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t ncols, void* W, fn_stream_t stream) {
+  if (d <= 0 || ncols <= 0 || !q || !scales || !W) return FN_ERR_INVALID_ARG;
+  if (d % 128 != 0 || ncols % 128 != 0 || d > kMaxDim || ncols > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(W) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FN_ERR_ALIGNMENT;
+  const size_t out = static_cast<size_t>(d) * ncols * 2;
+  if (overlaps(W, out, q, static_cast<size_t>(d) * ncols) ||
+      overlaps(W, out, scales, static_cast<size_t>(d / 128) * (ncols / 128) * 4))
+    return FN_ERR_ALIAS;
+  int sms = 0;
+  fn_status st = check_device(sms);
+  if (st != FN_OK) return st;
+  return launch_dequant_fp8(q, scales, d, ncols, W, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FN_OK
+             : FN_ERR_CUDA;
+}
+
+const char* fn_status_string(fn_status s) {
+  switch (s) {
+    case FN_OK: return "FN_OK";
+    case FN_ERR_INVALID_ARG: return "FN_ERR_INVALID_ARG";
+    case FN_ERR_UNSUPPORTED_SHAPE: return "FN_ERR_UNSUPPORTED_SHAPE";
+    case FN_ERR_ALIGNMENT: return "FN_ERR_ALIGNMENT";
+    case FN_ERR_ALIAS: return "FN_ERR_ALIAS";
+    case FN_ERR_WORKSPACE: return "FN_ERR_WORKSPACE";
+    case FN_ERR_CUDA: return "FN_ERR_CUDA";
+    case FN_ERR_TIMEOUT: return "FN_ERR_TIMEOUT";
+    case FN_ERR_UNSUPPORTED_DEVICE: return "FN_ERR_UNSUPPORTED_DEVICE";
+  }
+  return "FN_ERR_UNKNOWN";
+}
+
+int fn_version(void) { return 1; }
+
+fn_status fn_set_debug(int key, int64_t value) {
+  switch (key) {
+    case FN_DEBUG_WAIT_BUDGET_NS:
+      if (value <= 0) return FN_ERR_INVALID_ARG;
+      g_budget_ns.store(value);
+      return FN_OK;
+    case FN_DEBUG_WITHHOLD_ARRIVE:
+      g_withhold.store(value ? 1 : 0);
+      return FN_OK;
+    case FN_DEBUG_FORCE_PATH:
+      if (value < 0 || value > 2) return FN_ERR_INVALID_ARG;
+      g_force_path.store(static_cast<int>(value));
+      return FN_OK;
+  }
+  return FN_ERR_INVALID_ARG;
+}
+
+}  // extern "C"

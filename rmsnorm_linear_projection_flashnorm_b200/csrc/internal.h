@@ -1,0 +1,63 @@
+// Host-side launcher interface shared by the C-ABI layer (api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fn {
+
+// Workspace header: the first 256 bytes hold the device status word.
+constexpr size_t kWsHeaderBytes = 256;
+
+// One fused norm+projection call, validated by the ABI layer.
+struct CallArgs {
+  const void* x;          // bf16 [M, d]
+  int64_t M, d;
+  const void* Wp;         // folded weight, bf16 or e4m3 [d, ncols]
+  const float* scales;    // fp8 block scales [d/128, ncols/128] or null
+  int wtype;              // 0 bf16, 1 e4m3 with 128x128 block scales
+  int64_t N;              // output columns
+  int64_t ncols;          // stored weight columns: N or 2N (SwiGLU)
+  bool swiglu;
+  float eps;
+  void* y;                // bf16 [M, N]
+  void* ws;               // workspace (status word + decode scratch)
+  size_t ws_bytes;
+  cudaStream_t stream;
+  int num_sms;
+  uint64_t budget_ns;     // per-wait time limit
+  int withhold;           // test knob: withhold one reducer arrival
+};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
+
+// 2D row-major tensor map with 128-byte swizzle: rows x cols elements of
+// `elem_bytes`, box of box_rows x box_cols (box_cols * elem_bytes <= 128).
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows,
+                  uint64_t cols, uint32_t box_rows, uint32_t box_cols);
+
+// Decode (M <= 64) path: stream-K split over all SMs with a deterministic
+// in-kernel fix-up through workspace partials.
+int decode_mpad(int64_t M);
+size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms);
+cudaError_t launch_decode(const CallArgs& a);
+
+// Tensor-core tile path (M > 64): persistent 128x256 tiles, tcgen05 + TMEM.
+cudaError_t launch_tc(const CallArgs& a);
+
+// Offline fold and the unfused-chain helper kernels.
+cudaError_t launch_fold_bf16(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wp,
+                             cudaStream_t s);
+cudaError_t launch_fold_fp8(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wq,
+                            float* scales, cudaStream_t s);
+cudaError_t launch_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, float eps, void* h,
+                           cudaStream_t s);
+cudaError_t launch_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t ncols, void* W,
+                               cudaStream_t s);
+
+}  // namespace fn

@@ -1,0 +1,344 @@
+// Fused RMSNorm + projection, tensor-core tile path (M > 64), sm_100a.
+//
+// What it computes is FlashNorm's deferred normalisation (FlashNorm talk
+// summary, Proposal 2 "지연된 정규화"): with the gain already folded into W'
+// (Proposal 1), y[m, n] = r[m] * sum_k x[m, k] W'[k, n], where
+// r[m] = 1/sqrt(sum_k x[m,k]^2 / d + eps).  The matmul runs on the raw
+// activations on the tensor cores while the per-row sum of squares is reduced
+// on the CUDA cores from the same staged x tiles, and the scalar is applied
+// afterwards.  The optional SwiGLU epilogue (FlashInfer PR #5521 analysis,
+// design item "Register-level SwiGLU") turns a 256-column tile holding
+// matching gate and up columns into silu(r * gate) * (r * up).
+//
+// The talk's bug ("실제 버그", "원인", "수정" bullets) was an implicit join:
+// the post-scale read a matmul result that was not finished.  Here every join
+// is an mbarrier: the epilogue waits on the MMA commit of *this* tile's
+// accumulator buffer and on the reducers' barrier for *this* tile's sums of
+// squares; a stage of x is refilled only after both the MMA and the reducers
+// released it; an accumulator buffer is reused only after the epilogue
+// drained it.
+//
+// Layout: one persistent CTA per SM, 10 warps.
+//   warp 0      TMA producer: x tile 128x64 (K-major) and W' tile 64x256
+//               (four 64-column boxes, N-major), 128-byte swizzle, 4 stages
+//   warp 1      TMEM owner and MMA issuer (tcgen05.mma M=128 N=256 K=16)
+//   warps 2-5   sum-of-squares reducers, one thread per tile row
+//   warps 6-9   epilogue: TMEM -> registers, post-scale (+SwiGLU), bf16 store
+// Accumulators are double-buffered in TMEM (2 x 256 columns) so the epilogue
+// of one tile overlaps the main loop of the next.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fn {
+namespace tc {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+constexpr int B_BOX_BYTES = 64 * BK * 2;        // 8 KB: 64 columns x 64 rows
+constexpr int B_BYTES = BN * BK * 2;            // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int NUM_THREADS = 320;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int GROUP_M = 16;                     // tile raster: bands of 16 row blocks
+
+// wait sites reported in the status word
+enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteRedFull, kSiteRedSsqEmpty,
+                  kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain };
+
+struct Params {
+  int M, d, ncols, nout;
+  int num_m, num_n, num_tiles, kblocks;
+  float eps, inv_d;
+  __nv_bfloat16* y;
+  unsigned int* status;
+  unsigned long long budget_ns;
+  int withhold;
+};
+
+struct alignas(8) Bars {
+  uint64_t full[STAGES], empty[STAGES];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t ssq_full[2], ssq_empty[2];
+  uint64_t drain;
+  float ssq[2][BM];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Bars);
+
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
+  const int per_group = GROUP_M * p.num_n;
+  const int group = t / per_group;
+  const int first_m = group * GROUP_M;
+  const int gm = min(p.num_m - first_m, GROUP_M);
+  const int r = t - group * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+// Bounded wait that ignores the abort flag: used only to drain this CTA's
+// own asynchronous work before teardown.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long budget) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > budget) return;
+  }
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+              const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars& bars = *reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
+  auto stage_a = [&](int s) { return smem + s * STAGE_BYTES; };
+  auto stage_b = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], 1 + 4);  // MMA commit + one arrival per reducer warp
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.acc_full[b], 1);
+      mbar_init(&bars.acc_empty[b], 128);
+      mbar_init(&bars.ssq_full[b], 128);
+      mbar_init(&bars.ssq_empty[b], 128);
+    }
+    mbar_init(&bars.drain, 1);
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_x);
+    tma_prefetch_desc(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bars.tmem_base;
+  const WaitCtl ctl{&bars.abort_flag, p.status, p.budget_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t issued = 0, last_ph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, p, mb, nb);
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(&bars.empty[s], ph ^ 1, ctl, kSiteProdEmpty)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars.full[s], STAGE_BYTES);
+          tma_load_2d(stage_a(s), &tmap_x, &bars.full[s], kb * BK, mb * BM);
+#pragma unroll
+          for (int bx = 0; bx < BN / 64; ++bx)
+            tma_load_2d(stage_b(s) + bx * B_BOX_BYTES, &tmap_w, &bars.full[s], nb * BN + bx * 64, kb * BK);
+          issued |= 1u << s;
+          last_ph = (last_ph & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      // no copy may still be landing in shared memory when the CTA exits
+      for (int i = 0; i < STAGES; ++i)
+        if (issued & (1u << i)) drain_wait(&bars.full[i], (last_ph >> i) & 1u, p.budget_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*a MN-major*/ false, /*b MN-major*/ true);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int i = 0;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++i) {
+        const int b = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        if (!mbar_wait(&bars.acc_empty[b], aph ^ 1, ctl, kSiteMmaAccEmpty)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * BN;
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(stage_a(s));
+          const uint32_t b0 = smem_u32(stage_b(s));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // A: x rows, K-major, 128-byte rows, 8-row groups 1024 B apart; a K=16
+            //    slice is 32 bytes further along the (swizzled) row.
+            const uint64_t adesc = sdesc_sw128(a0 + kk * 32, 16, 1024);
+            // B: W' rows k, N-major: 64-column groups 8 KB apart (LBO), 8-row
+            //    k groups 1024 B apart (SBO); a K=16 slice is 16 rows = 2048 B.
+            const uint64_t bdesc = sdesc_sw128(b0 + kk * 2048, B_BOX_BYTES, 1024);
+            umma_bf16(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0);
+          }
+          umma_commit(&bars.empty[s]);
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&bars.acc_full[b]);
+      }
+      umma_commit(&bars.drain);
+      drain_wait(&bars.drain, 0, p.budget_ns);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ sum-of-squares reducers
+    const int row = (warp - 2) * 32 + lane;
+    int s = 0;
+    uint32_t ph = 0;
+    int i = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++i) {
+      float acc = 0.f;
+      for (int kb = 0; kb < p.kblocks; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[s], ph, ctl, kSiteRedFull))) { ok = false; break; }
+        // the 128-byte row of this thread's tile row; the swizzle permutes its
+        // eight 16-byte chunks, which leaves their sum unchanged
+        const uint4* rp = reinterpret_cast<const uint4*>(stage_a(s) + row * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = rp[c];
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float a = bf16lo_to_f32(w[j]), bb = bf16hi_to_f32(w[j]);
+            acc = fmaf(a, a, acc);
+            acc = fmaf(bb, bb, acc);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.empty[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+      if (!ok) break;
+      const int b = i & 1;
+      const uint32_t aph = (i >> 1) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.ssq_empty[b], aph ^ 1, ctl, kSiteRedSsqEmpty))) break;
+      bars.ssq[b][row] = acc;
+      if (!(p.withhold && i == 0)) mbar_arrive(&bars.ssq_full[b]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;       // tile row == accumulator lane
+    int i = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      const int b = i & 1;
+      const uint32_t aph = (i >> 1) & 1;
+      // warp-uniform decision: tcgen05.ld below is .sync.aligned
+      bool ok = mbar_wait(&bars.acc_full[b], aph, ctl, kSiteEpiAccFull);
+      ok = ok && mbar_wait(&bars.ssq_full[b], aph, ctl, kSiteEpiSsqFull);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const float r = inv_rms(bars.ssq[b][row], p.inv_d, p.eps);
+      mbar_arrive(&bars.ssq_empty[b]);
+      const int grow = mb * BM + row;
+      const bool row_ok = grow < p.M;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+      if (SWIGLU) {
+        __nv_bfloat16* yrow = p.y + static_cast<int64_t>(grow) * p.nout + nb * (BN / 2);
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t gv[32], uv[32];
+          tmem_ld32(taddr + c, gv);
+          tmem_ld32(taddr + BN / 2 + c, uv);
+          tmem_ld_wait();
+          uint32_t o[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float g0 = __uint_as_float(gv[2 * j]) * r, g1 = __uint_as_float(gv[2 * j + 1]) * r;
+            const float u0 = __uint_as_float(uv[2 * j]) * r, u1 = __uint_as_float(uv[2 * j + 1]) * r;
+            o[j] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+          }
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(yrow + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+          }
+        }
+      } else {
+        __nv_bfloat16* yrow = p.y + static_cast<int64_t>(grow) * p.nout;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_ld_wait();
+          const int col = nb * BN + c;
+          if (row_ok && col < p.nout) {
+            uint32_t o[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              o[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * r, __uint_as_float(v[2 * j + 1]) * r);
+            uint4* dst = reinterpret_cast<uint4*>(yrow + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.acc_empty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <bool SWIGLU>
+cudaError_t launch_impl(const CallArgs& a) {
+  CUtensorMap tx, tw;
+  if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, BM, BK)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d, a.ncols, BK, 64))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.M = static_cast<int>(a.M);
+  p.d = static_cast<int>(a.d);
+  p.ncols = static_cast<int>(a.ncols);
+  p.nout = static_cast<int>(a.N);
+  p.num_m = static_cast<int>((a.M + BM - 1) / BM);
+  p.num_n = static_cast<int>((a.ncols + BN - 1) / BN);
+  p.num_tiles = p.num_m * p.num_n;
+  p.kblocks = static_cast<int>(a.d / BK);
+  p.eps = a.eps;
+  p.inv_d = 1.0f / static_cast<float>(a.d);
+  p.y = static_cast<__nv_bfloat16*>(a.y);
+  p.status = static_cast<unsigned int*>(a.ws);
+  p.budget_ns = a.budget_ns;
+  p.withhold = a.withhold;
+  cudaError_t e = cudaFuncSetAttribute(tc_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(SMEM_BYTES));
+  if (e != cudaSuccess) return e;
+  const int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
+  tc_kernel<SWIGLU><<<grid, NUM_THREADS, SMEM_BYTES, a.stream>>>(tx, tw, p);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_tc(const CallArgs& a) {
+  return a.swiglu ? tc::launch_impl<true>(a) : tc::launch_impl<false>(a);
+}
+
+}  // namespace fn

@@ -1,0 +1,60 @@
+"""torch-facing conveniences over the C ABI: allocate outputs and workspaces
+with torch (device memory is torch's job here) and call the library.  No
+arithmetic of the method happens in Python."""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import (FN_W_BF16, FN_W_FP8_E4M3_B128, check, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
+               fn_query_device_status, fn_workspace_size)
+
+
+def fold(W0: torch.Tensor, g: torch.Tensor, W1: Optional[torch.Tensor] = None, wtype: int = FN_W_BF16,
+         stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Fold g into W0 (and W1 for SwiGLU); returns (W', scales or None)."""
+    d, N = W0.shape
+    ncols = 2 * N if W1 is not None else N
+    dev = W0.device
+    if wtype == FN_W_BF16:
+        Wp = torch.empty((d, ncols), dtype=torch.bfloat16, device=dev)
+        scales = None
+    else:
+        Wp = torch.empty((d, ncols), dtype=torch.uint8, device=dev)
+        scales = torch.empty((d // 128, ncols // 128), dtype=torch.float32, device=dev)
+    check(fn_fold_weights(W0, W1, g, d, N, wtype, Wp, scales, stream), "fn_fold_weights")
+    return Wp, scales
+
+
+class Workspace:
+    """A zero-initialised device workspace that grows on demand."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.buf = torch.zeros(256, dtype=torch.uint8, device=device)
+
+    def get(self, M: int, d: int, N: int, wt: int, swiglu: bool) -> torch.Tensor:
+        need = fn_workspace_size(M, d, N, wt, int(swiglu))
+        if self.buf.numel() < need:
+            self.buf = torch.zeros(need, dtype=torch.uint8, device=self.device)
+        return self.buf
+
+    def status(self, stream=None):
+        return fn_query_device_status(self.buf, stream)
+
+
+def norm_proj(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float, swiglu: bool = False,
+              scales: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None,
+              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y = RMSNorm(x) @ W through the fused kernels (W' already folded)."""
+    M, d = x.shape
+    wt = FN_W_BF16 if Wp.dtype == torch.bfloat16 else FN_W_FP8_E4M3_B128
+    if ws is None:
+        ws = Workspace(x.device)
+    buf = ws.get(M, d, N, wt, swiglu)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    fn = fn_norm_proj_swiglu if swiglu else fn_norm_proj
+    check(fn(x, M, d, Wp, scales, wt, N, eps, out, buf, buf.numel(), stream), fn.__name__)
+    return out

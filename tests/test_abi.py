@@ -1,0 +1,133 @@
+"""The C-ABI library on the host: it loads without a GPU, exports every symbol
+the header declares, and rejects bad arguments with status codes before it
+touches the device.  No compute call runs here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rmsnorm_linear_projection_flashnorm_b200 as fnb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flashnorm.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    fnb.build()
+    return fnb.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fn_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fn_fold_weights", "fn_norm_proj", "fn_norm_proj_swiglu", "fn_workspace_size",
+                     "fn_query_device_status", "fn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert fnb.fn_version() == 1
+
+
+def test_status_strings(L):
+    for code in range(9):
+        assert fnb.status_string(code).startswith("FN_")
+
+
+# fake, never-dereferenced device addresses: validation must reject before use
+A = 1 << 20          # 16-byte aligned
+B = 1 << 30
+C = 1 << 34
+WS = 1 << 36
+
+
+def np_(x=A, M=4, d=256, Wp=B, scales=None, wt=0, N=512, eps=1e-6, y=C, ws=WS, ws_bytes=1 << 30, swiglu=False):
+    f = fnb.fn_norm_proj_swiglu if swiglu else fnb.fn_norm_proj
+    return f(x, M, d, Wp, scales, wt, N, eps, y, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(M=-1), fnb.FN_ERR_INVALID_ARG),
+    (dict(d=0), fnb.FN_ERR_INVALID_ARG),
+    (dict(N=0), fnb.FN_ERR_INVALID_ARG),
+    (dict(eps=-1e-6), fnb.FN_ERR_INVALID_ARG),
+    (dict(eps=float("nan")), fnb.FN_ERR_INVALID_ARG),
+    (dict(eps=float("inf")), fnb.FN_ERR_INVALID_ARG),
+    (dict(wt=7), fnb.FN_ERR_INVALID_ARG),
+    (dict(d=100), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(N=500), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(wt=1, d=192, scales=A + (1 << 18)), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(M=1 << 31), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(x=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(Wp=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(y=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(ws=None), fnb.FN_ERR_WORKSPACE),
+    (dict(wt=1, scales=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(x=A + 8), fnb.FN_ERR_ALIGNMENT),
+    (dict(y=C + 2), fnb.FN_ERR_ALIGNMENT),
+    (dict(Wp=B + 4), fnb.FN_ERR_ALIGNMENT),
+    (dict(ws=WS + 8), fnb.FN_ERR_ALIGNMENT),
+    (dict(y=A + 16), fnb.FN_ERR_ALIAS),          # y overlaps x
+    (dict(y=B + 1024), fnb.FN_ERR_ALIAS),        # y overlaps W'
+    (dict(ws=C + 256), fnb.FN_ERR_ALIAS),        # workspace overlaps y
+    (dict(swiglu=True, y=B + 307200), fnb.FN_ERR_ALIAS),  # W' is [d, 2N]: 512 KB
+])
+def test_norm_proj_rejects_bad_arguments(L, kw, code):
+    assert np_(**kw) == code
+
+
+def test_empty_batch_is_a_noop(L):
+    assert np_(M=0, x=None, y=None, ws=None) == fnb.FN_OK
+    assert np_(M=0, swiglu=True, x=None, y=None, ws=None) == fnb.FN_OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=0), fnb.FN_ERR_INVALID_ARG),
+    (dict(W0=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(g=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(out_type=3), fnb.FN_ERR_INVALID_ARG),
+    (dict(out_type=1, scales=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(N=100), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(out_type=1, d=192), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(W0=A + 2), fnb.FN_ERR_ALIGNMENT),
+    (dict(Wp=A + 64), fnb.FN_ERR_ALIAS),
+])
+def test_fold_rejects_bad_arguments(L, kw, code):
+    args = dict(W0=A, W1=None, g=B, d=256, N=512, out_type=0, Wp=C, scales=WS)
+    args.update(kw)
+    st = fnb.fn_fold_weights(args["W0"], args["W1"], args["g"], args["d"], args["N"], args["out_type"],
+                             args["Wp"], args["scales"], None)
+    assert st == code
+
+
+def test_workspace_size_is_monotone_in_m_bucket(L):
+    sizes = [fnb.fn_workspace_size(m, 4096, 6144, 0, 0) for m in (1, 16, 17, 32, 33, 64)]
+    assert sizes[0] == sizes[1] and sizes[2] == sizes[3] and sizes[4] == sizes[5]
+    assert sizes[0] < sizes[2] < sizes[4]
+    assert fnb.fn_workspace_size(65, 4096, 6144, 0, 0) == 256
+    assert fnb.fn_workspace_size(8, 4096, 14336, 0, 1) > fnb.fn_workspace_size(8, 4096, 14336, 0, 0)
+
+
+def test_set_debug_validates_keys(L):
+    assert fnb.fn_set_debug(99, 1) == fnb.FN_ERR_INVALID_ARG
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 0) == fnb.FN_ERR_INVALID_ARG
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 5) == fnb.FN_ERR_INVALID_ARG
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 2_000_000_000) == fnb.FN_OK
+
+
+def test_no_device_means_no_launch(L):
+    """Valid arguments without a GPU fail cleanly (no device), never crash."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = np_()
+    assert st in (fnb.FN_ERR_CUDA, fnb.FN_ERR_UNSUPPORTED_DEVICE)
