@@ -1,0 +1,567 @@
+"""Benchmark of the fused RMSNorm + projection (FlashNorm form) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--m M]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, as the reference arm
+
+Default workload: decode QKV projection, d = 4096, N = 6144; one step is one
+pass of the hot path over each batch size of the workload, M in {1, 8, 32, 64}
+(four calls).  Inputs are seeded synthetic data (the ``workloads`` recipe) with
+random-init weights; the folded weight is replicated into enough copies that
+the copies together exceed twice the 126 MB L2, and every call reads the next
+copy, so no call finds its weight in L2.
+
+Metric: achieved HBM GB/s at decode M (algorithmic bytes: x, W' and y, each
+read or written once, per call), or tensor TFLOP/s at prefill M (2 M d N_cols
+per call), with the dominant kernel's fraction of the measured roofline.
+
+Multi-GPU (torchrun): one process per GPU; every rank runs its own batch
+against its own weight replica (rows of a batch are independent, so the path
+shards by rows with no collective; weak scaling).  Timing is on the device
+with CUDA events, and the job time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import faulthandler
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as WL  # noqa: E402
+
+METRIC = "fused norm+proj HBM GB/s (decode) & TFLOP/s (prefill); % of roofline"
+L2_BYTES = 126 * 1024 * 1024
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# environment
+# ---------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(local_units: float, local_ms: float, world: int, device):
+    """Whole-job throughput inputs: units summed over ranks, time as the
+    maximum over ranks (the slowest rank finishes the job)."""
+    if world == 1:
+        return local_units, local_ms
+    import torch.distributed as dist
+    u = torch.tensor([local_units], dtype=torch.float64, device=device)
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(u.item()), float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# ---------------------------------------------------------------------------
+_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = None
+            props = torch.cuda.get_device_properties(device_index)
+            ids = [getattr(props, k, None) for k in ("pci_domain_id", "pci_bus_id", "pci_device_id")]
+            if all(isinstance(v, int) for v in ids):
+                # NVML wants the "domain:bus:device.function" string, never an integer
+                bus_id = f"{ids[0]:08x}:{ids[1]:02x}:{ids[2]:02x}.0"
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus_id)
+                except pynvml.NVMLError:
+                    handle = None
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nvml, self._h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that, never guess
+            self._nvml = None
+            self.error = str(e)
+        self.period = period_s
+
+    def _run(self):
+        nv, h = self._nvml, self._h
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except AttributeError:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                self.samples.append((sm, reasons))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "no NVML")}
+        mhz = [s for s, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        reasons = sorted(name for b, name in _REASONS.items() if bits & b and name != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# workload setup
+# ---------------------------------------------------------------------------
+def algorithmic(M: int, d: int, N: int, swiglu: bool, wbytes_per_elem: int = 2):
+    ncols = 2 * N if swiglu else N
+    by = M * d * 2 + d * ncols * wbytes_per_elem + M * N * 2
+    fl = 2.0 * M * d * ncols
+    return by, fl
+
+
+def kernel_source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "rmsnorm_linear_projection_flashnorm_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(profile_name: str, src_hash: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; None otherwise."""
+    path = os.path.join(ROOT, "profiles", profile_name)
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip().strip("-* ")] = v.strip().strip("`")
+        if kv.get("source_sha256") != src_hash:
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class Setup:
+    def __init__(self, wl: WL.Workload, Ms, device):
+        import rmsnorm_linear_projection_flashnorm_b200 as fnb
+        from rmsnorm_linear_projection_flashnorm_b200 import torch_api as T
+        self.fnb, self.T = fnb, T
+        self.wl, self.Ms, self.dev = wl, list(Ms), device
+        d, N, sw = wl.d, wl.N, wl.swiglu
+        self.wtype = fnb.FN_W_BF16 if wl.wtype == "bf16" else fnb.FN_W_FP8_E4M3_B128
+        g = WL.gain(d, wl.seed).to(device)
+        if sw:
+            W0, W1 = (w.to(device) for w in WL.weights(d, N, wl.seed, halves=2))
+        else:
+            W0, W1 = WL.weights(d, N, wl.seed).to(device), None
+        Wp, scales = T.fold(W0, g, W1, wtype=self.wtype)
+        wp_bytes = Wp.numel() * Wp.element_size()
+        self.copies = max(2, math.ceil(2 * L2_BYTES / wp_bytes) + 1)
+        self.Wp = [Wp] + [Wp.clone() for _ in range(self.copies - 1)]
+        self.scales = [scales] + ([scales.clone() for _ in range(self.copies - 1)] if scales is not None else
+                                  [None] * (self.copies - 1))
+        # unfused chain operands: original (unfolded) weights, same number of copies
+        self.g = g
+        Wcat = torch.cat([W0, W1], dim=1) if sw else W0
+        self.W_unf = [Wcat] + [Wcat.clone() for _ in range(self.copies - 1)]
+        del W0, W1
+        Mmax = max(self.Ms)
+        x_all = WL.activations(Mmax, d, wl.seed, wl.outliers)
+        self.x_host = {M: x_all[:M].contiguous().pin_memory() for M in self.Ms}
+        self.x = {M: self.x_host[M].to(device) for M in self.Ms}
+        self.y = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in self.Ms}
+        self.y_host = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in self.Ms}
+        self.ws = T.Workspace(device)
+        for M in self.Ms:
+            self.ws.get(M, d, N, self.wtype, sw)
+        self.fn = fnb.fn_norm_proj_swiglu if sw else fnb.fn_norm_proj
+        self.i = 0
+        torch.cuda.synchronize()
+
+    def call(self, M, x=None, y=None, stream=None):
+        wl, c = self.wl, self.i % self.copies
+        self.i += 1
+        x = self.x[M] if x is None else x
+        y = self.y[M] if y is None else y
+        st = self.fn(x, M, wl.d, self.Wp[c], self.scales[c], self.wtype, wl.N, WL.EPS, y, self.ws.buf,
+                     self.ws.buf.numel(), stream)
+        if st != 0:
+            raise RuntimeError(f"norm_proj failed: {self.fnb.status_string(st)}")
+
+    def chain(self, M, stream=None):
+        """Unfused chain: standalone RMSNorm kernel -> cuBLAS GEMM -> (silu * up)."""
+        wl, c = self.wl, self.i % self.copies
+        self.i += 1
+        h = torch.empty((M, wl.d), dtype=torch.bfloat16, device=self.dev)
+        st = self.fnb.fn_rmsnorm(self.x[M], M, wl.d, self.g, WL.EPS, h, stream)
+        if st != 0:
+            raise RuntimeError(self.fnb.status_string(st))
+        z = torch.matmul(h, self.W_unf[c])
+        if wl.swiglu:
+            return torch.nn.functional.silu(z[:, :wl.N]) * z[:, wl.N:]
+        return z
+
+
+def run_cpu_baseline(wl: WL.Workload, Ms, budget_s: float = 10.0):
+    """The fp64 oracle (unfolded: RMSNorm, then the matmul with the original W
+    and g) on this host's cores, on a bounded sample: whole passes over the
+    workload's batch sizes until `budget_s` of CPU time has been spent."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        threads = None
+    cores = len(os.sched_getaffinity(0))
+    d, N = wl.d, wl.N
+    g = WL.gain(d, wl.seed)
+    if wl.swiglu:
+        W0, W1 = WL.weights(d, N, wl.seed, halves=2)
+    else:
+        W0, W1 = WL.weights(d, N, wl.seed), None
+    x_all = WL.activations(max(Ms), d, wl.seed, wl.outliers)
+    nbytes = 0
+    passes = 0
+    t0 = time.perf_counter()
+    while True:
+        for M in Ms:
+            x = x_all[:M]
+            if wl.swiglu:
+                O.norm_proj_swiglu(x, g, W0, W1, WL.EPS)
+            else:
+                O.norm_proj(x, g, W0, WL.EPS)
+            nbytes += algorithmic(M, d, N, wl.swiglu)[0]
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or passes >= 1000:
+            break
+    return {"value": nbytes / el / 1e9, "unit": "GB/s", "cores": threads or cores, "host_cores": cores,
+            "kind": "oracle",
+            "sample": f"{passes} full pass(es) over M={list(Ms)} of {wl.name} (d={d}, N={N}), "
+                      f"fp64 NumPy, {el:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle as O
+    wl = WL.WORKLOADS[args.workload]
+    Ms = [args.m] if args.m else list(wl.Ms)
+    d, N = wl.d, wl.N
+    g = WL.gain(d, wl.seed)
+    if wl.swiglu:
+        W0, W1 = WL.weights(d, N, wl.seed, halves=2)
+    else:
+        W0, W1 = WL.weights(d, N, wl.seed), None
+    x_all = WL.activations(max(Ms), d, wl.seed, wl.outliers)
+
+    def step(j):
+        M = Ms[j % len(Ms)]
+        x = x_all[:M]
+        if wl.swiglu:
+            O.norm_proj_swiglu(x, g, W0, W1, WL.EPS)
+        else:
+            O.norm_proj(x, g, W0, WL.EPS)
+        return algorithmic(M, d, N, wl.swiglu)[0]
+
+    for j in range(args.warmup):
+        step(j)
+    nbytes = 0
+    t0 = time.perf_counter()
+    for j in range(args.steps):
+        nbytes += step(j)
+    el = time.perf_counter() - t0
+    value = nbytes / el / 1e9
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded workloads recipe; random-init weights)",
+        "config": {"workload": wl.name, "M": Ms, "d": d, "N": N, "swiglu": wl.swiglu,
+                   "step": "one oracle call per step, cycling through M"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} oracle calls cycling M={Ms}"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the fused path
+# ---------------------------------------------------------------------------
+def _stage(msg: str) -> None:
+    if os.environ.get("FN_BENCH_TRACE"):
+        print(f"[bench] {msg}", file=sys.stderr, flush=True)
+
+
+def main():
+    faulthandler.enable()
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="fused", choices=["fused", "reference"])
+    ap.add_argument("--workload", default="decode_qkv", choices=list(WL.WORKLOAD_ORDER))
+    ap.add_argument("--m", type=int, default=0, help="run a single batch size of the workload")
+    ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU oracle baseline")
+    ap.add_argument("--skip-chain", action="store_true", help="omit the unfused-chain baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import rmsnorm_linear_projection_flashnorm_b200 as fnb
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        fnb.build()
+    barrier(world)
+    fnb.lib()
+
+    wl = WL.WORKLOADS[args.workload]
+    Ms = [args.m] if args.m else list(wl.Ms)
+    _stage("setup")
+    S = Setup(wl, Ms, dev)
+    _stage("setup done")
+    stream = torch.cuda.current_stream()
+    peaks, peaks_kind = load_peaks()
+    wbyte = 2 if wl.wtype == "bf16" else 1
+    bytes_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte)[0] for M in Ms)
+    flops_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte)[1] for M in Ms)
+    hbm_bound = max(Ms) <= 64
+
+    # warm-up
+    for _ in range(args.warmup):
+        for M in Ms:
+            S.call(M)
+    torch.cuda.synchronize()
+    _stage("warm-up done")
+
+    # Timed region: K steps, each replaying a CUDA graph of one step (the way a
+    # decode loop issues work).  Graph p holds calls p*len(Ms) .. onward of the
+    # weight-copy rotation, so consecutive calls always read different copies;
+    # each graph also records an event pair around every launch, which gives
+    # the kernel's own duration on the launching stream.
+    K = args.steps
+    n_calls = len(Ms)
+    period = S.copies // math.gcd(n_calls, S.copies)
+    n_graphs = period * max(1, math.ceil(16 / period))
+    graphs = []
+    cap_stream = torch.cuda.Stream()
+    launches0 = fnb.fn_kernel_launches()
+    for gi in range(n_graphs):
+        S.i = (gi * n_calls) % S.copies
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n_calls)]
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=cap_stream):
+            for j, M in enumerate(Ms):
+                evs[2 * j].record()
+                S.call(M)
+                evs[2 * j + 1].record()
+        graphs.append((gr, evs))
+    kernels_per_step = (fnb.fn_kernel_launches() - launches0) // n_graphs
+    _stage(f"{n_graphs} graphs captured, {kernels_per_step} kernels per step")
+    for gi in range(max(args.warmup, n_graphs)):
+        graphs[gi % n_graphs][0].replay()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for k in range(K):
+            graphs[k % n_graphs][0].replay()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    _stage("timed region done")
+    elapsed_ms = t_start.elapsed_time(t_end)
+    job_units, job_ms = aggregate(float(bytes_per_step if hbm_bound else flops_per_step) * K, elapsed_ms,
+                                  world, dev)
+    gpu_launches = K * kernels_per_step
+    # per-launch durations: the last replay of each graph inside the timed region
+    kernel_ms, kernel_n = 0.0, 0
+    for gi in range(min(n_graphs, K)):
+        evs = graphs[gi][1]
+        for j in range(n_calls):
+            kernel_ms += evs[2 * j].elapsed_time(evs[2 * j + 1])
+            kernel_n += 1
+
+    value_bytes = job_units / (job_ms / 1e3) if hbm_bound else 0.0
+    value_flops = job_units / (job_ms / 1e3) if not hbm_bound else 0.0
+    kernel_avg_ms = kernel_ms / max(kernel_n, 1)
+    per_launch_bytes = bytes_per_step / len(Ms)
+    per_launch_flops = flops_per_step / len(Ms)
+    src_hash = kernel_source_hash(["decode.cu" if hbm_bound else "tc.cu", "ptx.cuh"])
+    prof_name = f"{'decode_kernel' if hbm_bound else 'tc_kernel'}_{wl.name}.md"
+    traffic = profile_traffic(prof_name, src_hash)
+    if hbm_bound:
+        peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+        achieved = per_launch_bytes / (kernel_avg_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": traffic, "kernel": "decode_kernel (+ decode_fixup_kernel): one fn_norm_proj call",
+                    "peak_source": f"hbm_gbs ({peaks_kind})",
+                    "bytes_per_launch": per_launch_bytes, "avg_launch_us": kernel_avg_ms * 1e3}
+        value, unit = value_bytes / 1e9, "GB/s"
+    else:
+        peak = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+        achieved = per_launch_flops / (kernel_avg_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": traffic, "kernel": "tc_kernel: one fn_norm_proj call",
+                    "peak_source": f"bf16_tflops_sustained ({peaks_kind})",
+                    "flops_per_launch": per_launch_flops, "avg_launch_us": kernel_avg_ms * 1e3}
+        value, unit = value_flops / 1e12, "TFLOP/s"
+
+    # end to end through the public API: pinned host x -> device -> call -> host y
+    e2e_steps = max(1, min(K, 2000))
+    h2d = sum(S.x_host[M].numel() * 2 for M in Ms)
+    d2h = sum(S.y_host[M].numel() * 2 for M in Ms)
+    xs = {M: torch.empty_like(S.x[M]) for M in Ms}
+    for _ in range(3):
+        for M in Ms:
+            xs[M].copy_(S.x_host[M], non_blocking=True)
+            S.call(M, x=xs[M])
+            S.y_host[M].copy_(S.y[M], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for M in Ms:
+            xs[M].copy_(S.x_host[M], non_blocking=True)
+            S.call(M, x=xs[M])
+            S.y_host[M].copy_(S.y[M], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_units, e2e_ms = aggregate(float(bytes_per_step if hbm_bound else flops_per_step) * e2e_steps,
+                                  e0.elapsed_time(e1), world, dev)
+    e2e_val = e2e_units / (e2e_ms / 1e3)
+    _stage("e2e done")
+    e2e = {"value": e2e_val / (1e9 if hbm_bound else 1e12), "unit": unit, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    # unfused chain (same rotation of weight copies): rmsnorm -> cuBLAS -> silu*up
+    chain = None
+    if not args.skip_chain:
+        for _ in range(3):
+            for M in Ms:
+                S.chain(M)
+        torch.cuda.synchronize()
+        c_steps = max(1, min(K, 2000))
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(c_steps):
+            for M in Ms:
+                S.chain(M)
+        c1.record(stream)
+        torch.cuda.synchronize()
+        chain_ms = c0.elapsed_time(c1) / c_steps
+        chain = {"ms_per_step": chain_ms, "fused_speedup": chain_ms / (elapsed_ms / K),
+                 "what": "fn_rmsnorm kernel -> torch.matmul (cuBLAS) with unfolded W"
+                         + (" -> silu(gate)*up" if wl.swiglu else "")}
+
+    _stage("chain done")
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        cpu = run_cpu_baseline(wl, Ms)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": job_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if wl.wtype == "bf16" else "bf16 (e4m3 weights)",
+            "data": "synthetic (seeded workloads recipe; random-init weights)",
+            "config": {"workload": wl.name, "M": Ms, "d": wl.d, "N": wl.N, "swiglu": wl.swiglu,
+                       "weights": wl.wtype, "parallelism": f"replicas x{world} (rows shard, no collective)",
+                       "l2": f"{S.copies} rotating W' copies ({S.copies * S.Wp[0].numel() * S.Wp[0].element_size() / 1e6:.0f} MB > L2)",
+                       "step": f"{len(Ms)} fused calls, one per M, replayed as one CUDA graph",
+                       "kernel_timing": f"event pairs around each call, last replay of {min(n_graphs, K)} graphs",
+                       "kernels_per_step": kernels_per_step},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks.summary(),
+            "gpu_launches": gpu_launches, "unfused_chain": chain,
+            "kernel_source_sha256": src_hash,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

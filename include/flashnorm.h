@@ -86,10 +86,11 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
 /*
  * fn_workspace_size — bytes of workspace a call with these sizes needs.
  * The workspace holds a 256-byte header (the device status word) and, for
- * M <= 64, the stream-K partial sums and tile counters.  It must be
- * zero-filled once before its first use; every call leaves it ready for the
- * next one (after FN_ERR_TIMEOUT, zero it again).  Depends on the SM count of
- * the current device (148 is assumed when no device is visible).
+ * M <= 64, the per-CTA partial sums of the split-K decode path.  Zero it once
+ * before its first use (the status word must start at zero); the calls keep
+ * the status word at zero unless a device-side wait times out.  Depends on
+ * the SM count of the current device (148 is assumed when no device is
+ * visible).
  */
 size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swiglu);
 
@@ -101,7 +102,8 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
  *   eps     >= 0 and finite, added to the mean inside the square root
  *   y       bf16 [M, N] output; must not overlap x, Wp, scales or workspace
  *   workspace, ws_bytes  >= fn_workspace_size(M, d, N, wt, 0), zeroed before first use
- *   M == 0 is a no-op.  M <= 64 runs the split-K decode kernel, larger M the
+ *   M == 0 is a no-op.  M <= 64 runs the split-K decode kernel (plus a small
+ *   fix-up kernel for the column tiles whose k range it split), larger M the
  *   tensor-core tile kernel; both are deterministic (repeated calls with the
  *   same inputs give the same bits).
  */
@@ -143,6 +145,10 @@ const char* fn_status_string(fn_status s);
 /* ABI version of this library (increments on any signature change). */
 int fn_version(void);
 
+/* Number of kernels this library has enqueued in this process (all devices,
+ * all streams); for accounting in benchmarks and tests. */
+uint64_t fn_kernel_launches(void);
+
 /*
  * fn_set_debug — process-wide knobs for tests and diagnostics (not thread-safe;
  * set them before issuing work):
@@ -150,8 +156,12 @@ int fn_version(void);
  *   FN_DEBUG_WITHHOLD_ARRIVE  1: the reducers withhold their first arrival, so the
  *                             epilogue's wait must run out (exercises FN_ERR_TIMEOUT)
  *   FN_DEBUG_FORCE_PATH       0 auto, 1 decode kernel (M <= 64 only), 2 tile kernel
+ *   FN_DEBUG_PREFETCH         decode path: weight prefetch into L2 before waiting on
+ *                             the previous kernel; value = mode | (k_blocks << 8),
+ *                             mode 0 off, 1 TMA prefetch, 2 per-thread prefetch
+ *                             (default: mode 2, 8 k-blocks)
  */
-enum { FN_DEBUG_WAIT_BUDGET_NS = 1, FN_DEBUG_WITHHOLD_ARRIVE = 2, FN_DEBUG_FORCE_PATH = 3 };
+enum { FN_DEBUG_WAIT_BUDGET_NS = 1, FN_DEBUG_WITHHOLD_ARRIVE = 2, FN_DEBUG_FORCE_PATH = 3, FN_DEBUG_PREFETCH = 4 };
 fn_status fn_set_debug(int key, int64_t value);
 
 #ifdef __cplusplus

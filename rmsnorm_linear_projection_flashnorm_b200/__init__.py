@@ -32,6 +32,7 @@ FN_W_FP8_E4M3_B128 = 1
 FN_DEBUG_WAIT_BUDGET_NS = 1
 FN_DEBUG_WITHHOLD_ARRIVE = 2
 FN_DEBUG_FORCE_PATH = 3
+FN_DEBUG_PREFETCH = 4
 
 _vp, _i64, _f32, _sz, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_int
 
@@ -45,6 +46,7 @@ _SIGNATURES = {
     "fn_dequant_fp8": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "fn_status_string": (ctypes.c_char_p, [_int]),
     "fn_version": (_int, []),
+    "fn_kernel_launches": (ctypes.c_uint64, []),
     "fn_set_debug": (_int, [_int, _i64]),
 }
 
@@ -104,6 +106,10 @@ def status_string(status: int) -> str:
 
 def fn_version() -> int:
     return lib().fn_version()
+
+
+def fn_kernel_launches() -> int:
+    return lib().fn_kernel_launches()
 
 
 def fn_set_debug(key: int, value: int) -> int:

@@ -24,6 +24,8 @@ namespace {
 std::atomic<long long> g_budget_ns{2000000000LL};
 std::atomic<int> g_withhold{0};
 std::atomic<int> g_force_path{0};
+std::atomic<int> g_prefetch_iters{8};
+std::atomic<int> g_prefetch_mode{2};
 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
@@ -68,7 +70,10 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 bool eps_ok(float eps) { return std::isfinite(eps) && eps >= 0.0f; }
 
 constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
+std::atomic<unsigned long long> g_launches{0};
 }  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -168,6 +173,8 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.num_sms = sms;
   a.budget_ns = static_cast<uint64_t>(g_budget_ns.load());
   a.withhold = g_withhold.load();
+  a.prefetch_iters = g_prefetch_iters.load();
+  a.prefetch_mode = g_prefetch_mode.load();
   const cudaError_t e = use_decode ? launch_decode(a) : launch_tc(a);
   return e == cudaSuccess ? FN_OK : FN_ERR_CUDA;
 }
@@ -294,6 +301,8 @@ const char* fn_status_string(fn_status s) {
 
 int fn_version(void) { return 1; }
 
+uint64_t fn_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
 fn_status fn_set_debug(int key, int64_t value) {
   switch (key) {
     case FN_DEBUG_WAIT_BUDGET_NS:
@@ -306,6 +315,11 @@ fn_status fn_set_debug(int key, int64_t value) {
     case FN_DEBUG_FORCE_PATH:
       if (value < 0 || value > 2) return FN_ERR_INVALID_ARG;
       g_force_path.store(static_cast<int>(value));
+      return FN_OK;
+    case FN_DEBUG_PREFETCH:
+      if (value < 0 || (value & 0xFF) > 2) return FN_ERR_INVALID_ARG;
+      g_prefetch_mode.store(static_cast<int>(value & 0xFF));
+      g_prefetch_iters.store(static_cast<int>(value >> 8));
       return FN_OK;
   }
   return FN_ERR_INVALID_ARG;

@@ -14,18 +14,22 @@
 //
 // The weight is split over every SM with a stream-K partition of the
 // (column tile, 64-deep k block) iterations, so every SM streams the same
-// number of weight bytes whatever the tile count.  A tile whose k range is
-// split between CTAs is finished in the same kernel: each CTA writes its fp32
-// partial accumulators and partial sums of squares to the workspace, and the
-// CTA that arrives last on the tile's counter adds the partials in ascending
-// k order (a fixed order, so repeated calls are bit-identical), applies the
-// post-scale (and SwiGLU) and stores the result.  No floating-point atomics.
+// number of weight bytes whatever the tile count.  A tile whose k range falls
+// to one CTA is finished by that CTA.  A tile whose k range is split between
+// CTAs is finished by a second, small kernel (decode_fixup_kernel): each
+// contributing CTA writes its fp32 partial accumulators and partial sums of
+// squares to the workspace, and the fix-up kernel, launched programmatically
+// so it is resident before the first kernel ends, adds the partials in
+// ascending k order (a fixed order, so repeated calls are bit-identical),
+// applies the post-scale (and SwiGLU) and stores the result.  No atomics, no
+// cross-CTA waits, no counters to reset.
 //
 // Layout: 8 warps.
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
 //   warps 2-3   sum-of-squares reducers (one thread per activation row)
 //   warps 4-7   epilogue / fix-up (one thread per weight column of the tile)
+#include <cstddef>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -38,7 +42,7 @@ namespace dec {
 constexpr int BK = 64;
 constexpr int NUM_THREADS = 256;
 constexpr int W_BOX_BYTES = 64 * BK * 2;   // 64 columns x 64 k rows, bf16
-constexpr int SMEM_BUDGET = 200 * 1024;
+constexpr int SMEM_BUDGET = 200 * 1024;   // pipeline stages; barriers and staging come on top
 
 enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteRedFull, kSiteRedSsqEmpty,
                   kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain };
@@ -63,23 +67,25 @@ struct Params {
   float eps, inv_d;
   __nv_bfloat16* y;
   float* part;               // [grid][2][SLOT_FLOATS]
-  unsigned int* counters;    // [tiles]
   unsigned int* status;
   unsigned long long budget_ns;
   int withhold;
+  const uint8_t* wp;         // folded weight base (L2 prefetch addresses)
+  int prefetch_iters;        // k-blocks per CTA prefetched into L2 before the dependency wait
+  int prefetch_mode;         // 0 none, 1 TMA prefetch, 2 per-thread prefetch from idle warps
 };
 
 template <int MPAD, int HALVES, int STAGES>
-struct alignas(8) Bars {
+struct alignas(16) Bars {
   uint64_t full[STAGES], empty[STAGES];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t ssq_full[2], ssq_empty[2];
   uint64_t drain;
   float ssq[2][MPAD];
+  alignas(16) __nv_bfloat16 ybuf[MPAD * 128];   // one tile's output rows, staged for 16-byte stores
   uint32_t tmem_base;
   int abort_flag;
   int epi_ok[2];
-  int last_flag[2];
 };
 
 __device__ __forceinline__ long long it_begin(int c, const Params& p) {
@@ -94,6 +100,22 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > budget) return;
+  }
+}
+
+// Copy the staged output rows of one 128-column tile to y with 16-byte
+// stores: 16 consecutive threads write one 256-byte row segment.  The next
+// write to the staging buffer happens only after the epilogue group's next
+// named barrier, which every thread reaches after finishing this copy.
+__device__ __forceinline__ void store_tile_rows(const __nv_bfloat16* ybuf, const Params& p, int tile, int et) {
+  const int col0 = tile * 128;
+  const int chunks = p.M * 16;
+  for (int i = et; i < chunks; i += 128) {
+    const int m = i >> 4, c16 = i & 15;
+    if (col0 + c16 * 8 < p.nout) {
+      const uint4 v = *reinterpret_cast<const uint4*>(ybuf + m * 128 + c16 * 8);
+      *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m) * p.nout + col0 + c16 * 8) = v;
+    }
   }
 }
 
@@ -162,6 +184,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Everything above overlaps the previous kernel in the stream.  So does an
+  // L2 prefetch of the first part of this CTA's weight range (the weight does
+  // not depend on the previous kernel's output, and an L2 prefetch cannot
+  // return stale data).  Nothing below may read or write global memory
+  // through shared memory or registers before the previous kernel completed.
+  if (p.prefetch_mode == 1 && warp == 0 && lane == 0) {
+    int n_pf = 0;
+    for (long long it = it0; it < it1 && n_pf < p.prefetch_iters; ++it, ++n_pf) {
+      const int tile = static_cast<int>(it / p.kblocks);
+      const int kb = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
+#pragma unroll
+      for (int bx = 0; bx < 2 * HALVES; ++bx) tma_prefetch_l2_2d(&tmap_w, tile * 128 * HALVES + bx * 64, kb * BK);
+    }
+  } else if (p.prefetch_mode == 2 && warp >= 2) {
+    // one 128-byte line per thread and step: (k row, 128-byte column chunk)
+    const int lines_per_row = HALVES * 2;              // 256 or 512 bytes of a k row per tile
+    const long long n_it = min(static_cast<long long>(p.prefetch_iters), it1 - it0);
+    const int total = static_cast<int>(n_it) * BK * lines_per_row;
+    for (int i = threadIdx.x - 64; i < total; i += NUM_THREADS - 64) {
+      const int chunk = i % lines_per_row;
+      const int r = (i / lines_per_row) % BK;
+      const long long it = it0 + i / (lines_per_row * BK);
+      const int tile = static_cast<int>(it / p.kblocks);
+      const int kb = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
+      const uint8_t* a = p.wp + (static_cast<int64_t>(kb) * BK + r) * p.ncols * 2 +
+                         static_cast<int64_t>(tile) * 256 * HALVES + chunk * 128;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+    }
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
   const uint32_t tmem_base = bars.tmem_base;
   const WaitCtl ctl{&bars.abort_flag, p.status, p.budget_ns};
 
@@ -253,20 +306,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float acc = 0.f;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[s], ph, ctl, kSiteRedFull))) { ok = false; break; }
-        if (row < MPAD) {
-          const uint4* rp = reinterpret_cast<const uint4*>(stage_x(s) + row * 128);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = rp[c];
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float a = bf16lo_to_f32(w[j]), bb = bf16hi_to_f32(w[j]);
-              acc = fmaf(a, a, acc);
-              acc = fmaf(bb, bb, acc);
-            }
-          }
-        }
+        if (row < MPAD && row < p.M) acc += row_sumsq_sw128(stage_x(s), row);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.empty[s]);
         if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -308,7 +348,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld_cols<MPAD>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (b * HALVES + h) * MPAD, acc[h]);
       tc_fence_before();
       mbar_arrive(&bars.acc_empty[b]);
-      const int col = tile * 128 + n;            // output column
       const bool whole = (kb0 == 0 && kb1 == p.kblocks);
       if (whole) {
 #pragma unroll
@@ -318,54 +357,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           float v;
           if (HALVES == 2) v = silu_f32(acc[0][m] * r) * (acc[1][m] * r);
           else v = acc[0][m] * r;
-          if (col < p.nout) p.y[static_cast<int64_t>(m) * p.nout + col] = __float2bfloat16_rn(v);
+          bars.ybuf[m * 128 + n] = __float2bfloat16_rn(v);
         }
         mbar_arrive(&bars.ssq_empty[b]);
+        named_bar_sync(1, 128);
+        store_tile_rows(bars.ybuf, p, tile, et);
         continue;
       }
-      // split tile: publish this CTA's partial, then the last arrival finishes it
+      // Split tile: publish this CTA's partial for the fix-up kernel.  A slot
+      // holds float4 groups [half][row / 4][column] (a warp's 16-byte accesses
+      // are contiguous), only for the rows < M, then the MPAD partial sums of
+      // squares.
+      const int Q = (p.M + 3) >> 2;
       const int slot = cta * 2 + (seg == 0 ? 0 : 1);
-      float* part = p.part + static_cast<int64_t>(slot) * C::SLOT_FLOATS;
+      float4* part4 = reinterpret_cast<float4*>(p.part + static_cast<int64_t>(slot) * C::SLOT_FLOATS);
 #pragma unroll
       for (int h = 0; h < HALVES; ++h)
 #pragma unroll
-        for (int m = 0; m < MPAD; ++m)
-          if (m < p.M) __stcg(part + (h * MPAD + m) * 128 + n, acc[h][m]);
+        for (int q4 = 0; q4 < MPAD / 4; ++q4)
+          if (q4 < Q)
+            __stcg(part4 + (h * (MPAD / 4) + q4) * 128 + n,
+                   make_float4(acc[h][4 * q4], acc[h][4 * q4 + 1], acc[h][4 * q4 + 2], acc[h][4 * q4 + 3]));
+      float* part = p.part + static_cast<int64_t>(slot) * C::SLOT_FLOATS;
       if (et < MPAD) __stcg(part + HALVES * MPAD * 128 + et, bars.ssq[b][et]);
       mbar_arrive(&bars.ssq_empty[b]);
-      __threadfence();
-      named_bar_sync(1, 128);
-      const int c_first = owner_of(static_cast<long long>(tile) * p.kblocks, p);
-      const int c_last = owner_of(static_cast<long long>(tile + 1) * p.kblocks - 1, p);
-      if (et == 0) {
-        const unsigned prev = atomicAdd(&p.counters[tile], 1u);
-        bars.last_flag[seg & 1] = (prev == static_cast<unsigned>(c_last - c_first)) ? 1 : 0;
-      }
-      named_bar_sync(1, 128);
-      if (!bars.last_flag[seg & 1]) continue;
-      __threadfence();
-#pragma unroll 1
-      for (int m = 0; m < p.M && m < MPAD; ++m) {
-        float tot[HALVES];
-        float ssq = 0.f;
-#pragma unroll
-        for (int h = 0; h < HALVES; ++h) tot[h] = 0.f;
-#pragma unroll 1
-        for (int c = c_first; c <= c_last; ++c) {
-          const long long cb = it_begin(c, p);
-          const int cslot = c * 2 + (cb >= static_cast<long long>(tile) * p.kblocks ? 0 : 1);
-          const float* cp = p.part + static_cast<int64_t>(cslot) * C::SLOT_FLOATS;
-#pragma unroll
-          for (int h = 0; h < HALVES; ++h) tot[h] += __ldcg(cp + (h * MPAD + m) * 128 + n);
-          ssq += __ldcg(cp + HALVES * MPAD * 128 + m);
-        }
-        const float r = inv_rms(ssq, p.inv_d, p.eps);
-        float v;
-        if (HALVES == 2) v = silu_f32(tot[0] * r) * (tot[1] * r);
-        else v = tot[0] * r;
-        if (col < p.nout) p.y[static_cast<int64_t>(m) * p.nout + col] = __float2bfloat16_rn(v);
-      }
-      if (et == 0) p.counters[tile] = 0u;   // ready for the next call
     }
   }
 
@@ -377,6 +392,83 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// Fix-up of the tiles whose k range was split between CTAs.  One thread per
+// (tile, row group of 4, column): it loads the float4 partials of every
+// contributing CTA (up to four in flight at once), adds them in ascending k
+// order together with the partial sums of squares of its four rows, applies
+// 1/rms (and SwiGLU) and stores four bf16 outputs.
+constexpr int FIX_THREADS = 128;
+
+template <int MPAD, int HALVES>
+__global__ void __launch_bounds__(FIX_THREADS) decode_fixup_kernel(const Params p) {
+  using C = Cfg<MPAD, HALVES>;
+  // Let the next kernel in the stream launch now: its CTAs take SMs as the
+  // stream-K CTAs leave and prefetch their weights into L2 meanwhile.  All
+  // CTAs of the stream-K grid are resident by now (each triggered this
+  // launch after its own start), so no generation can starve another.
+  grid_launch_dependents();
+  grid_dependency_wait();        // the partials of the stream-K kernel are complete and visible
+  const int Q = (p.M + 3) >> 2;
+  const long long gid = static_cast<long long>(blockIdx.x) * FIX_THREADS + threadIdx.x;
+  const int n = static_cast<int>(gid & 127);
+  const long long rest = gid >> 7;
+  const int q = static_cast<int>(rest % Q);
+  const int tile = static_cast<int>(rest / Q);
+  if (tile >= p.tiles) return;
+  const long long t_it0 = static_cast<long long>(tile) * p.kblocks;
+  const int c_first = owner_of(t_it0, p);
+  const int c_last = owner_of(t_it0 + p.kblocks - 1, p);
+  if (c_first == c_last) return;   // finished by the stream-K kernel itself
+  float4 acc[HALVES];
+#pragma unroll
+  for (int h = 0; h < HALVES; ++h) acc[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 ss = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto add = [](float4& t, const float4& v) { t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w; };
+  constexpr int CB = 4;
+  for (int c0 = c_first; c0 <= c_last; c0 += CB) {
+    float4 v[CB][HALVES], s4[CB];
+#pragma unroll
+    for (int j = 0; j < CB; ++j) {
+      const int c = c0 + j;
+      if (c <= c_last) {
+        const int slot = c * 2 + (it_begin(c, p) >= t_it0 ? 0 : 1);
+        const float4* base = reinterpret_cast<const float4*>(p.part + static_cast<int64_t>(slot) * C::SLOT_FLOATS);
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h) v[j][h] = __ldcg(base + (h * (MPAD / 4) + q) * 128 + n);
+        s4[j] = __ldcg(base + HALVES * (MPAD / 4) * 128 + q);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < CB; ++j) {
+      if (c0 + j <= c_last) {
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h) add(acc[h], v[j][h]);
+        add(ss, s4[j]);
+      }
+    }
+  }
+  const float a0[4] = {acc[0].x, acc[0].y, acc[0].z, acc[0].w};
+  const float a1[4] = {acc[HALVES - 1].x, acc[HALVES - 1].y, acc[HALVES - 1].z, acc[HALVES - 1].w};
+  const float sq[4] = {ss.x, ss.y, ss.z, ss.w};
+  const int col = tile * 128 + n;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = 4 * q + i;
+    if (m >= p.M) break;
+    const float r = inv_rms(sq[i], p.inv_d, p.eps);
+    float v = a0[i] * r;
+    if (HALVES == 2) v = silu_f32(v) * (a1[i] * r);
+    if (col < p.nout) p.y[static_cast<int64_t>(m) * p.nout + col] = __float2bfloat16_rn(v);
+  }
+}
+
+// The staging buffer is read as 16-byte vectors; the barrier block itself is
+// placed at a 1024-byte multiple.
+using BarsSmall = Bars<16, 1, 8>;
+using BarsLarge = Bars<64, 2, 5>;
+static_assert(offsetof(BarsSmall, ybuf) % 16 == 0 && offsetof(BarsLarge, ybuf) % 16 == 0,
+              "ybuf must be 16-byte aligned");
+
 template <int MPAD, int HALVES>
 constexpr size_t smem_bytes() {
   using C = Cfg<MPAD, HALVES>;
@@ -386,7 +478,7 @@ constexpr size_t smem_bytes() {
 struct Layout {
   int tiles, kblocks, grid;
   long long total;
-  size_t counters_off, part_off, bytes;
+  size_t part_off, bytes;
 };
 
 template <int MPAD, int HALVES>
@@ -396,8 +488,7 @@ Layout layout_for(int64_t d, int64_t ncols, int num_sms) {
   L.kblocks = static_cast<int>(d / BK);
   L.total = static_cast<long long>(L.tiles) * L.kblocks;
   L.grid = static_cast<int>(L.total < num_sms ? L.total : num_sms);
-  L.counters_off = kWsHeaderBytes;
-  L.part_off = L.counters_off + (static_cast<size_t>(L.tiles) * 4 + 255) / 256 * 256;
+  L.part_off = kWsHeaderBytes;
   L.bytes = L.part_off + static_cast<size_t>(L.grid) * 2 * Cfg<MPAD, HALVES>::SLOT_FLOATS * 4;
   return L;
 }
@@ -424,16 +515,31 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.y = static_cast<__nv_bfloat16*>(a.y);
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
   p.status = reinterpret_cast<unsigned int*>(ws);
-  p.counters = reinterpret_cast<unsigned int*>(ws + L.counters_off);
   p.part = reinterpret_cast<float*>(ws + L.part_off);
   p.budget_ns = a.budget_ns;
   p.withhold = a.withhold;
+  p.wp = static_cast<const uint8_t*>(a.Wp);
+  p.prefetch_iters = a.prefetch_iters;
+  p.prefetch_mode = a.prefetch_mode;
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<MPAD, HALVES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(SMEM));
+  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
-  decode_kernel<MPAD, HALVES><<<L.grid, NUM_THREADS, SMEM, a.stream>>>(tx, tw, p);
-  return cudaGetLastError();
+  e = launch_pdl(decode_kernel<MPAD, HALVES>, L.grid, NUM_THREADS, SMEM, a.stream, tx, tw, p);
+  if (e != cudaSuccess) return e;
+  if (L.grid <= L.tiles) {
+    // every CTA's range covers whole tiles only when the grid is at most the
+    // tile count and divides the iterations evenly; otherwise some tile is split
+    bool split = false;
+    for (int c = 0; c < L.grid && !split; ++c) {
+      const long long b0 = static_cast<long long>(c) * L.total / L.grid;
+      const long long b1 = static_cast<long long>(c + 1) * L.total / L.grid;
+      split = (b0 % L.kblocks) != 0 || (b1 % L.kblocks) != 0;
+    }
+    if (!split) return cudaSuccess;
+  }
+  const long long threads = static_cast<long long>(L.tiles) * 128 * ((a.M + 3) / 4);
+  const unsigned fgrid = static_cast<unsigned>((threads + FIX_THREADS - 1) / FIX_THREADS);
+  return launch_pdl(decode_fixup_kernel<MPAD, HALVES>, fgrid, FIX_THREADS, 0, a.stream, p);
 }
 
 template <int MPAD>

@@ -217,7 +217,9 @@ cudaError_t launch_fold_bf16(const void* W0, const void* W1, const float* g, int
   fold_bf16_kernel<<<grid_for(d * ncols / 8, kFoldThreads), kFoldThreads, 0, s>>>(
       static_cast<const __nv_bfloat16*>(W0), static_cast<const __nv_bfloat16*>(W1), g, d, N,
       static_cast<__nv_bfloat16*>(Wp));
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launch();
+  return e;
 }
 
 cudaError_t launch_fold_fp8(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wq,
@@ -227,7 +229,9 @@ cudaError_t launch_fold_fp8(const void* W0, const void* W1, const float* g, int6
   fold_fp8_kernel<<<grid, kFoldThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(W0),
                                                 static_cast<const __nv_bfloat16*>(W1), g, d, N,
                                                 static_cast<uint8_t*>(Wq), scales);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launch();
+  return e;
 }
 
 cudaError_t launch_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, float eps, void* h,
@@ -235,14 +239,18 @@ cudaError_t launch_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, 
   const int grid = static_cast<int>(M < 148 * 16 ? M : 148 * 16);
   rmsnorm_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), M, d, g, eps,
                                       static_cast<__nv_bfloat16*>(h));
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launch();
+  return e;
 }
 
 cudaError_t launch_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t ncols, void* W,
                                cudaStream_t s) {
   dequant_fp8_kernel<<<grid_for(d * ncols / 8, 256), 256, 0, s>>>(static_cast<const uint8_t*>(q), scales, d,
                                                                   ncols, static_cast<__nv_bfloat16*>(W));
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launch();
+  return e;
 }
 
 }  // namespace fn

@@ -1,8 +1,10 @@
 // Host-side launcher interface shared by the C-ABI layer (api.cu) and the
 // kernel translation units.  Not part of the public ABI.
 #pragma once
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -29,6 +31,8 @@ struct CallArgs {
   int num_sms;
   uint64_t budget_ns;     // per-wait time limit
   int withhold;           // test knob: withhold one reducer arrival
+  int prefetch_iters;     // decode: weight k-blocks per CTA prefetched into L2 early
+  int prefetch_mode;      // decode: 0 none, 1 TMA prefetch, 2 per-thread prefetch
 };
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -59,5 +63,45 @@ cudaError_t launch_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, 
                            cudaStream_t s);
 cudaError_t launch_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t ncols, void* W,
                                cudaStream_t s);
+
+// Raise a kernel's dynamic shared-memory limit once per device (a host-only
+// call, done on the first launch so later launches can be graph-captured).
+// One flag set per kernel: the kernel itself is the template argument.
+template <auto Kernel>
+cudaError_t ensure_smem_limit(int bytes) {
+  static std::atomic<unsigned long long> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+// Process-wide count of kernels enqueued by the library.
+void count_launch();
+
+// Launch with programmatic stream serialization: the kernel may start (and
+// run its prologue) while the preceding kernel in the stream finishes; it
+// calls griddepcontrol.wait before touching global memory.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) count_launch();
+  return e;
+}
 
 }  // namespace fn

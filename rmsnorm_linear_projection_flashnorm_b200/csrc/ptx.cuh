@@ -31,6 +31,15 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Programmatic dependent launch: wait until the preceding grid in the stream
+// has completed and its writes are visible; allow the next grid to launch.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // abort / status plumbing shared by all roles of one CTA
 // ---------------------------------------------------------------------------
@@ -121,6 +130,16 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, ui
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)),
         "r"(c0), "r"(c1), "l"(policy)
       : "memory");
+}
+
+// Bring a 2D tile of a tensor into L2 only (no shared memory, no barrier).
+// L2 is the coherence point for global memory, so a prefetch can never leave
+// a stale copy behind: it is safe to issue before griddepcontrol.wait, even if
+// the preceding kernel is still writing the same tensor.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1)
+               : "memory");
 }
 
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
@@ -247,6 +266,29 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_fl
 // silu(z) = z / (1 + e^-z), written with CUDA's exp; for z << 0 the
 // denominator overflows to inf and the result is -0.
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + __expf(-z)); }
+
+// Sum of squares of one 64-element bf16 row of a tile that TMA stored with
+// the 128-byte swizzle (row r's 16-byte chunk c sits at chunk c ^ (r & 7)).
+// Reading chunk c ^ (r & 7) on step c makes the eight rows of a bank group
+// hit eight different 16-byte bank slots, so a warp's loads are
+// conflict-free; four partial sums shorten the FMA dependency chain.  The
+// order of the additions is fixed.
+__device__ __forceinline__ float row_sumsq_sw128(const uint8_t* tile, int row) {
+  const uint8_t* base = tile + row * 128;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(base + ((c ^ (row & 7)) << 4));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = bf16lo_to_f32(w[j]), hi = bf16hi_to_f32(w[j]);
+      a[j] = fmaf(lo, lo, a[j]);
+      a[j] = fmaf(hi, hi, a[j]);
+    }
+  }
+  return (a[0] + a[1]) + (a[2] + a[3]);
+}
 
 // 1 / sqrt(mean + eps) for a row, from its sum of squares over d columns.
 __device__ __forceinline__ float inv_rms(float ssq, float inv_d, float eps) {

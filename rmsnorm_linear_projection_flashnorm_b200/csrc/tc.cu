@@ -128,6 +128,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Everything above overlaps the previous kernel in the stream; nothing
+  // below may touch global memory before that kernel has completed.
+  grid_dependency_wait();
+  grid_launch_dependents();
   const uint32_t tmem_base = bars.tmem_base;
   const WaitCtl ctl{&bars.abort_flag, p.status, p.budget_ns};
 
@@ -208,20 +212,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float acc = 0.f;
       for (int kb = 0; kb < p.kblocks; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[s], ph, ctl, kSiteRedFull))) { ok = false; break; }
-        // the 128-byte row of this thread's tile row; the swizzle permutes its
-        // eight 16-byte chunks, which leaves their sum unchanged
-        const uint4* rp = reinterpret_cast<const uint4*>(stage_a(s) + row * 128);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = rp[c];
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float a = bf16lo_to_f32(w[j]), bb = bf16hi_to_f32(w[j]);
-            acc = fmaf(a, a, acc);
-            acc = fmaf(bb, bb, acc);
-          }
-        }
+        acc += row_sumsq_sw128(stage_a(s), row);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.empty[s]);
         if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -327,12 +318,10 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.status = static_cast<unsigned int*>(a.ws);
   p.budget_ns = a.budget_ns;
   p.withhold = a.withhold;
-  cudaError_t e = cudaFuncSetAttribute(tc_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(SMEM_BYTES));
+  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU>>(static_cast<int>(SMEM_BYTES));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
-  tc_kernel<SWIGLU><<<grid, NUM_THREADS, SMEM_BYTES, a.stream>>>(tx, tw, p);
-  return cudaGetLastError();
+  return launch_pdl(tc_kernel<SWIGLU>, grid, NUM_THREADS, SMEM_BYTES, a.stream, tx, tw, p);
 }
 
 }  // namespace tc
