@@ -122,6 +122,30 @@ fn_status fn_norm_proj_swiglu(const void* x, int64_t M, int64_t d, const void* W
                               fn_stream_t stream);
 
 /*
+ * fn_norm_proj_static — fn_norm_proj for callers that cannot allocate device
+ * memory, so cannot pass a workspace: code recording work under a CUDA stream
+ * capture (where cudaMalloc is not permitted), plug-ins whose host application
+ * owns every device allocation, and loops that must never call cudaMalloc
+ * because it can synchronise the device.  The pages have no counterpart of
+ * this entry point; it only moves the scratch memory.
+ *   Arguments, layout and results as fn_norm_proj, minus the workspace.  The
+ *   call's scratch (status word and split-K partials) lives in a fixed
+ *   8 MiB array inside the library that every GPU loading the library holds
+ *   until the process exits.  Sizes whose scratch exceeds it (as computed by
+ *   fn_workspace_size) are rejected with FN_ERR_WORKSPACE before any launch:
+ *   on a 148-SM B200 every shape with M <= 32 or M > 64 fits, and M in 33..64
+ *   fits only while the split-K partials stay under 8 MiB.
+ *   The first call on a device fetches the array's device address and zeroes
+ *   its status word (a synchronous set-up step): make that first call before
+ *   any stream capture.  All calls on a device share the array and it keeps
+ *   the last call's contents; calls that may overlap on the GPU race on it.
+ *   Device-side wait timeouts are recorded in the array, not reported.  The
+ *   call allocates nothing.
+ */
+fn_status fn_norm_proj_static(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                              fn_wtype wt, int64_t N, float eps, void* y, fn_stream_t stream);
+
+/*
  * fn_query_device_status — synchronises `stream`, reads and clears the status
  * word in `workspace`.  Returns FN_OK or FN_ERR_TIMEOUT; *detail (if not NULL)
  * receives the raw word (bits 8-15 name the wait site that gave up).
