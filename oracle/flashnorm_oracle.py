@@ -45,7 +45,7 @@ __all__ = [
     "BF16", "E4M3", "round_to_format", "bf16_round", "bf16_bits", "bf16_from_bits",
     "e4m3_round", "e4m3_encode", "e4m3_decode", "to_f64",
     "rms_inv", "rmsnorm", "norm_proj", "silu", "norm_proj_swiglu",
-    "fold_bf16", "interleave128", "deinterleave128", "fold_fp8", "dequant_fp8",
+    "fold_bf16", "interleave128", "deinterleave128", "fold_fp8", "dequant_fp8", "dequant_fp8_bf16_bits",
     "FP8_BLOCK", "E4M3_MAX",
 ]
 
@@ -278,3 +278,12 @@ def dequant_fp8(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     """float64 W_deq[k,n] = e4m3(q[k,n]) * s[k/128, n/128] (exact in fp64)."""
     s_full = np.repeat(np.repeat(to_f64(s), FP8_BLOCK, axis=0), FP8_BLOCK, axis=1)
     return e4m3_decode(q) * s_full
+
+
+def dequant_fp8_bf16_bits(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of the on-chip dequantisation step: the e4m3 value
+    (exact in fp32) times the fp32 block scale, rounded to fp32, then rounded
+    once more to bf16 (the bf16 operand the tensor cores multiply)."""
+    s_full = np.repeat(np.repeat(np.asarray(s, dtype=np.float32), FP8_BLOCK, axis=0), FP8_BLOCK, axis=1)
+    prod = e4m3_decode(q).astype(np.float32) * s_full        # fp32 IEEE product
+    return bf16_bits(prod.astype(np.float64))

@@ -91,7 +91,7 @@ EncodeTiledFn encode_fn() {
 }
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows,
-                  uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+                  uint64_t cols, uint32_t box_rows, uint32_t box_cols, bool swizzle128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cols, rows};
@@ -100,7 +100,8 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, in
   const cuuint32_t estr[2] = {1, 1};
   std::memset(map, 0, sizeof(*map));
   const CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -147,7 +148,6 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   } else if (force == 2) {
     use_decode = false;
   }
-  if (wt == FN_W_FP8_E4M3_B128) return FN_ERR_UNSUPPORTED_SHAPE;  // fp8 kernels: not built yet
 
   int sms = 0;
   fn_status st = check_device(sms);

@@ -40,18 +40,21 @@ namespace fn {
 namespace dec {
 
 constexpr int BK = 64;
-constexpr int NUM_THREADS = 256;
+// 8 warps: producer, MMA, 2 reducers, 4 epilogue; fp8 weights add 2 converter warps
+template <bool FP8>
+__host__ __device__ constexpr int num_threads() { return FP8 ? 320 : 256; }
 constexpr int W_BOX_BYTES = 64 * BK * 2;   // 64 columns x 64 k rows, bf16
 constexpr int SMEM_BUDGET = 200 * 1024;   // pipeline stages; barriers and staging come on top
 
 enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteRedFull, kSiteRedSsqEmpty,
-                  kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain };
+                  kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain, kSiteMmaConv, kSiteConvFull };
 
-template <int MPAD, int HALVES>
+template <int MPAD, int HALVES, bool FP8 = false>
 struct Cfg {
-  static constexpr int W_BYTES = HALVES * 2 * W_BOX_BYTES;          // 16 or 32 KB
+  static constexpr int W_BYTES = HALVES * 2 * W_BOX_BYTES;          // bf16 operand: 16 or 32 KB
   static constexpr int X_BYTES = MPAD * BK * 2;                     // 2, 4 or 8 KB
-  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;             // multiple of 1024
+  static constexpr int E4_BYTES = FP8 ? HALVES * 128 * BK : 0;      // e4m3 staging: 8 or 16 KB
+  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + E4_BYTES;  // multiple of 1024
   static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int ACC_COLS = HALVES * MPAD;                    // one accumulator buffer
@@ -73,11 +76,13 @@ struct Params {
   const uint8_t* wp;         // folded weight base (L2 prefetch addresses)
   int prefetch_iters;        // k-blocks per CTA prefetched into L2 before the dependency wait
   int prefetch_mode;         // 0 none, 1 TMA prefetch, 2 per-thread prefetch from idle warps
+  const float* scales;       // fp8: block scales [d/128][ncols/128]
 };
 
 template <int MPAD, int HALVES, int STAGES>
 struct alignas(16) Bars {
   uint64_t full[STAGES], empty[STAGES];
+  uint64_t conv[STAGES];     // fp8: the stage's weight tile has been converted to bf16
   uint64_t acc_full[2], acc_empty[2];
   uint64_t ssq_full[2], ssq_empty[2];
   uint64_t drain;
@@ -139,11 +144,12 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[MPAD]) {
   }
 }
 
-template <int MPAD, int HALVES>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int MPAD, int HALVES, bool FP8>
+__global__ void __launch_bounds__(num_threads<FP8>(), 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   const Params p) {
-  using C = Cfg<MPAD, HALVES>;
+  using C = Cfg<MPAD, HALVES, FP8>;
+  constexpr int NUM_THREADS = num_threads<FP8>();
   constexpr int STAGES = C::STAGES;
   using B = Bars<MPAD, HALVES, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -151,6 +157,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   B& bars = *reinterpret_cast<B*>(smem + STAGES * C::STAGE_BYTES);
   auto stage_w = [&](int s) { return smem + s * C::STAGE_BYTES; };
   auto stage_x = [&](int s) { return smem + s * C::STAGE_BYTES + C::W_BYTES; };
+  auto stage_e4 = [&](int s) { return smem + s * C::STAGE_BYTES + C::W_BYTES + C::X_BYTES; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -162,6 +169,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1 + 2);   // MMA commit + two reducer warps
+      mbar_init(&bars.conv[s], 64);       // fp8: every converter thread
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
@@ -195,11 +203,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int tile = static_cast<int>(it / p.kblocks);
       const int kb = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
 #pragma unroll
-      for (int bx = 0; bx < 2 * HALVES; ++bx) tma_prefetch_l2_2d(&tmap_w, tile * 128 * HALVES + bx * 64, kb * BK);
+      if (FP8) tma_prefetch_l2_2d(&tmap_w, tile * 128 * HALVES, kb * BK);
+      else
+        for (int bx = 0; bx < 2 * HALVES; ++bx) tma_prefetch_l2_2d(&tmap_w, tile * 128 * HALVES + bx * 64, kb * BK);
     }
   } else if (p.prefetch_mode == 2 && warp >= 2) {
     // one 128-byte line per thread and step: (k row, 128-byte column chunk)
-    const int lines_per_row = HALVES * 2;              // 256 or 512 bytes of a k row per tile
+    constexpr int WB = FP8 ? 1 : 2;                    // weight bytes per element
+    const int lines_per_row = HALVES * WB;             // 128 * HALVES * WB bytes of a k row per tile
     const long long n_it = min(static_cast<long long>(p.prefetch_iters), it1 - it0);
     const int total = static_cast<int>(n_it) * BK * lines_per_row;
     for (int i = threadIdx.x - 64; i < total; i += NUM_THREADS - 64) {
@@ -208,8 +219,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const long long it = it0 + i / (lines_per_row * BK);
       const int tile = static_cast<int>(it / p.kblocks);
       const int kb = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
-      const uint8_t* a = p.wp + (static_cast<int64_t>(kb) * BK + r) * p.ncols * 2 +
-                         static_cast<int64_t>(tile) * 256 * HALVES + chunk * 128;
+      const uint8_t* a = p.wp + (static_cast<int64_t>(kb) * BK + r) * p.ncols * WB +
+                         static_cast<int64_t>(tile) * 128 * HALVES * WB + chunk * 128;
       asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
     }
   }
@@ -231,12 +242,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int kb1 = static_cast<int>(min(static_cast<long long>(p.kblocks), kb0 + (it1 - it)));
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&bars.empty[s], ph ^ 1, ctl, kSiteProdEmpty)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars.full[s], C::STAGE_BYTES);
+          // TMA fills x and either the bf16 weight boxes or the e4m3 staging tile
+          mbar_arrive_expect_tx(&bars.full[s], C::X_BYTES + (FP8 ? C::E4_BYTES : C::W_BYTES));
           tma_load_2d(stage_x(s), &tmap_x, &bars.full[s], kb * BK, 0);
+          if (FP8) {
+            // one unswizzled box of 128 * HALVES e4m3 columns x 64 k rows
+            tma_load_2d_hint(stage_e4(s), &tmap_w, &bars.full[s], tile * 128 * HALVES, kb * BK, w_policy);
+          } else {
 #pragma unroll
-          for (int bx = 0; bx < 2 * HALVES; ++bx)
-            tma_load_2d_hint(stage_w(s) + bx * W_BOX_BYTES, &tmap_w, &bars.full[s], tile * 128 * HALVES + bx * 64,
-                             kb * BK, w_policy);
+            for (int bx = 0; bx < 2 * HALVES; ++bx)
+              tma_load_2d_hint(stage_w(s) + bx * W_BOX_BYTES, &tmap_w, &bars.full[s],
+                               tile * 128 * HALVES + bx * 64, kb * BK, w_policy);
+          }
           issued |= 1u << s;
           last_ph = (last_ph & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -265,6 +282,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
+          if (FP8 && !mbar_wait(&bars.conv[s], ph, ctl, kSiteMmaConv)) { ok = false; break; }
           tc_fence_after();
           const uint32_t w0 = smem_u32(stage_w(s));
           const uint32_t x0 = smem_u32(stage_x(s));
@@ -318,6 +336,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (row < MPAD) bars.ssq[b][row] = acc;
       if (!(p.withhold && seg == 0)) mbar_arrive(&bars.ssq_full[b]);
       it += kb1 - kb0;
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ fp8 converters
+    // e4m3 tile (64 k rows x 128*HALVES bytes, unswizzled) -> bf16 operand tile
+    // with the 128x128 block scale folded in: bf16(fp32(q) * s), one rounding.
+    if (FP8) {
+      const int ct = threadIdx.x - 256;                 // 0..63
+      constexpr int UNITS_PER_ROW = 8 * HALVES;         // 16-byte e4m3 chunks per k row
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (long long it = it0; it < it1 && ok;) {
+        const int tile = static_cast<int>(it / p.kblocks);
+        const int kb0 = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
+        const int kb1 = static_cast<int>(min(static_cast<long long>(p.kblocks), kb0 + (it1 - it)));
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const int scale_row = (kb * BK) >> 7;
+          float sc[HALVES];
+#pragma unroll
+          for (int h = 0; h < HALVES; ++h) sc[h] = __ldg(p.scales + static_cast<int64_t>(scale_row) * (p.ncols >> 7) +
+                                                         tile * HALVES + h);
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[s], ph, ctl, kSiteConvFull))) { ok = false; break; }
+          const uint8_t* e4 = stage_e4(s);
+          uint8_t* wt = stage_w(s);
+#pragma unroll
+          for (int i = 0; i < BK * UNITS_PER_ROW / 64; ++i) {
+            const int u = ct + 64 * i;
+            const int k = u / UNITS_PER_ROW;
+            const int n0 = (u % UNITS_PER_ROW) * 16;
+            const float scale = (HALVES == 2 && n0 >= 128) ? sc[HALVES - 1] : sc[0];
+            e4m3x16_scale_to_bf16_sw128(e4 + k * (128 * HALVES) + n0, scale, wt, k, n0);
+          }
+          fence_proxy_async_smem();   // generic-proxy writes -> visible to tcgen05.mma
+          mbar_arrive(&bars.conv[s]);
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+        it += kb1 - kb0;
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue / fix-up
@@ -468,10 +524,11 @@ using BarsSmall = Bars<16, 1, 8>;
 using BarsLarge = Bars<64, 2, 5>;
 static_assert(offsetof(BarsSmall, ybuf) % 16 == 0 && offsetof(BarsLarge, ybuf) % 16 == 0,
               "ybuf must be 16-byte aligned");
+static_assert(Cfg<64, 2, true>::STAGES >= 2 && Cfg<64, 2, false>::STAGES >= 2, "pipeline needs two stages");
 
-template <int MPAD, int HALVES>
+template <int MPAD, int HALVES, bool FP8>
 constexpr size_t smem_bytes() {
-  using C = Cfg<MPAD, HALVES>;
+  using C = Cfg<MPAD, HALVES, FP8>;
   return 1024 + C::STAGES * C::STAGE_BYTES + sizeof(Bars<MPAD, HALVES, C::STAGES>);
 }
 
@@ -493,14 +550,19 @@ Layout layout_for(int64_t d, int64_t ncols, int num_sms) {
   return L;
 }
 
-template <int MPAD, int HALVES>
+template <int MPAD, int HALVES, bool FP8>
 cudaError_t launch_impl(const CallArgs& a) {
   const Layout L = layout_for<MPAD, HALVES>(a.d, a.ncols, a.num_sms);
   if (a.ws_bytes < L.bytes) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, MPAD, BK)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d, a.ncols, BK, 64))
+  if (FP8) {
+    // e4m3 bytes, one unswizzled box of 128 * HALVES columns x 64 k rows per stage
+    if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.d, a.ncols, BK, 128 * HALVES, false))
+      return cudaErrorInvalidValue;
+  } else if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d, a.ncols, BK, 64)) {
     return cudaErrorInvalidValue;
+  }
   Params p;
   p.M = static_cast<int>(a.M);
   p.d = static_cast<int>(a.d);
@@ -521,10 +583,11 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.wp = static_cast<const uint8_t*>(a.Wp);
   p.prefetch_iters = a.prefetch_iters;
   p.prefetch_mode = a.prefetch_mode;
-  constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
-  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES>>(static_cast<int>(SMEM));
+  p.scales = a.scales;
+  constexpr size_t SMEM = smem_bytes<MPAD, HALVES, FP8>();
+  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES, FP8>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
-  e = launch_pdl(decode_kernel<MPAD, HALVES>, L.grid, NUM_THREADS, SMEM, a.stream, tx, tw, p);
+  e = launch_pdl(decode_kernel<MPAD, HALVES, FP8>, L.grid, num_threads<FP8>(), SMEM, a.stream, tx, tw, p);
   if (e != cudaSuccess) return e;
   if (L.grid <= L.tiles) {
     // every CTA's range covers whole tiles only when the grid is at most the
@@ -544,7 +607,8 @@ cudaError_t launch_impl(const CallArgs& a) {
 
 template <int MPAD>
 cudaError_t launch_halves(const CallArgs& a) {
-  return a.swiglu ? launch_impl<MPAD, 2>(a) : launch_impl<MPAD, 1>(a);
+  if (a.wtype == 1) return a.swiglu ? launch_impl<MPAD, 2, true>(a) : launch_impl<MPAD, 1, true>(a);
+  return a.swiglu ? launch_impl<MPAD, 2, false>(a) : launch_impl<MPAD, 1, false>(a);
 }
 
 }  // namespace dec

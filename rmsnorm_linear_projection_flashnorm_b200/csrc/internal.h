@@ -43,7 +43,7 @@ EncodeTiledFn encode_fn();
 // 2D row-major tensor map with 128-byte swizzle: rows x cols elements of
 // `elem_bytes`, box of box_rows x box_cols (box_cols * elem_bytes <= 128).
 bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows,
-                  uint64_t cols, uint32_t box_rows, uint32_t box_cols);
+                  uint64_t cols, uint32_t box_rows, uint32_t box_cols, bool swizzle128 = true);
 
 // Decode (M <= 64) path: stream-K split over all SMs with a deterministic
 // in-kernel fix-up through workspace partials.

@@ -290,6 +290,32 @@ __device__ __forceinline__ float row_sumsq_sw128(const uint8_t* tile, int row) {
   return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
+// Sixteen e4m3 weights (one k row, tile columns n0 .. n0+15) times the fp32
+// block scale s, each product rounded once to bf16, stored into the N-major
+// 128-byte-swizzled operand tile that tcgen05.mma reads: 64-column boxes of
+// 64 k rows, 8 KB apart; row k of a box is 128 bytes whose 16-byte chunk j
+// sits at chunk j ^ (k & 7).  n0 is a multiple of 16.
+__device__ __forceinline__ void e4m3x16_scale_to_bf16_sw128(const uint8_t* src16, float s, uint8_t* wtile,
+                                                            int k, int n0) {
+  const uint4 v = *reinterpret_cast<const uint4*>(src16);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __half2_raw hr =
+          __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>((w[j] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+      o[2 * j + h] = pack_bf16x2(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
+    }
+  }
+  const int j0 = (n0 & 63) >> 3;
+  uint8_t* row = wtile + (n0 >> 6) * 8192 + k * 128;
+  *reinterpret_cast<uint4*>(row + ((j0 ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+  *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
 // 1 / sqrt(mean + eps) for a row, from its sum of squares over d columns.
 __device__ __forceinline__ float inv_rms(float ssq, float inv_d, float eps) {
   return rsqrtf(fmaf(ssq, inv_d, eps));

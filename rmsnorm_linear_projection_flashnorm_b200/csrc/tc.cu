@@ -18,7 +18,8 @@
 // released it; an accumulator buffer is reused only after the epilogue
 // drained it.
 //
-// Layout: one persistent CTA per SM, 10 warps.
+// Layout: one persistent CTA per SM, 10 warps (14 with fp8 weights: warps
+// 10-13 convert each staged e4m3 weight tile to the bf16 operand tile).
 //   warp 0      TMA producer: x tile 128x64 (K-major) and W' tile 64x256
 //               (four 64-column boxes, N-major), 128-byte swizzle, 4 stages
 //   warp 1      TMEM owner and MMA issuer (tcgen05.mma M=128 N=256 K=16)
@@ -35,18 +36,25 @@
 namespace fn {
 namespace tc {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BOX_BYTES = 64 * BK * 2;        // 8 KB: 64 columns x 64 rows
 constexpr int B_BYTES = BN * BK * 2;            // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
-constexpr int NUM_THREADS = 320;
+constexpr int E4_BYTES = BN * BK;               // fp8 weights: 16 KB e4m3 staging per stage
 constexpr int TMEM_COLS = 2 * BN;
+
+// bf16 weights: 4 stages of 48 KB, 10 warps.  fp8 weights: 3 stages of 64 KB
+// (x, bf16 operand, e4m3 staging) and 4 more warps converting e4m3 to bf16.
+template <bool FP8> struct Cfg {
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + (FP8 ? E4_BYTES : 0);
+  static constexpr int STAGES = FP8 ? 3 : 4;
+  static constexpr int NUM_THREADS = FP8 ? 448 : 320;
+};
 constexpr int GROUP_M = 16;                     // tile raster: bands of 16 row blocks
 
 // wait sites reported in the status word
 enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteRedFull, kSiteRedSsqEmpty,
-                  kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain };
+                  kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain, kSiteMmaConv, kSiteConvFull };
 
 struct Params {
   int M, d, ncols, nout;
@@ -56,10 +64,13 @@ struct Params {
   unsigned int* status;
   unsigned long long budget_ns;
   int withhold;
+  const float* scales;   // fp8: block scales [d/128][ncols/128]
 };
 
+template <int STAGES>
 struct alignas(8) Bars {
   uint64_t full[STAGES], empty[STAGES];
+  uint64_t conv[STAGES];   // fp8: the stage's weight tile has been converted to bf16
   uint64_t acc_full[2], acc_empty[2];
   uint64_t ssq_full[2], ssq_empty[2];
   uint64_t drain;
@@ -68,7 +79,11 @@ struct alignas(8) Bars {
   int abort_flag;
 };
 
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Bars);
+template <bool FP8>
+constexpr size_t smem_bytes() {
+  return 1024 + Cfg<FP8>::STAGES * Cfg<FP8>::STAGE_BYTES + sizeof(Bars<Cfg<FP8>::STAGES>);
+}
+static_assert(smem_bytes<true>() <= 232448 && smem_bytes<false>() <= 232448, "shared memory budget");
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
   const int per_group = GROUP_M * p.num_n;
@@ -89,15 +104,18 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
   }
 }
 
-template <bool SWIGLU>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <bool SWIGLU, bool FP8>
+__global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
               const Params p) {
+  constexpr int STAGES = Cfg<FP8>::STAGES;
+  constexpr int STAGE_BYTES = Cfg<FP8>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars& bars = *reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
+  Bars<STAGES>& bars = *reinterpret_cast<Bars<STAGES>*>(smem + STAGES * STAGE_BYTES);
   auto stage_a = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stage_b = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
+  auto stage_e4 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B_BYTES; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -106,6 +124,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1 + 4);  // MMA commit + one arrival per reducer warp
+      mbar_init(&bars.conv[s], 128);     // fp8: every converter thread
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
@@ -147,11 +166,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tile_coords(t, p, mb, nb);
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(&bars.empty[s], ph ^ 1, ctl, kSiteProdEmpty)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars.full[s], STAGE_BYTES);
+          mbar_arrive_expect_tx(&bars.full[s], FP8 ? A_BYTES + E4_BYTES : A_BYTES + B_BYTES);
           tma_load_2d(stage_a(s), &tmap_x, &bars.full[s], kb * BK, mb * BM);
+          if (FP8) {
+            // one unswizzled box of 256 e4m3 columns x 64 k rows
+            tma_load_2d(stage_e4(s), &tmap_w, &bars.full[s], nb * BN, kb * BK);
+          } else {
 #pragma unroll
-          for (int bx = 0; bx < BN / 64; ++bx)
-            tma_load_2d(stage_b(s) + bx * B_BOX_BYTES, &tmap_w, &bars.full[s], nb * BN + bx * 64, kb * BK);
+            for (int bx = 0; bx < BN / 64; ++bx)
+              tma_load_2d(stage_b(s) + bx * B_BOX_BYTES, &tmap_w, &bars.full[s], nb * BN + bx * 64, kb * BK);
+          }
           issued |= 1u << s;
           last_ph = (last_ph & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -178,6 +202,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d_tmem = tmem_base + b * BN;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
+          if (FP8 && !mbar_wait(&bars.conv[s], ph, ctl, kSiteMmaConv)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(stage_a(s));
           const uint32_t b0 = smem_u32(stage_b(s));
@@ -201,6 +226,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_wait(&bars.drain, 0, p.budget_ns);
     }
     __syncwarp();
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------ fp8 converters
+    // e4m3 tile (64 k rows x 256 bytes, unswizzled) -> bf16 operand tile with
+    // the 128x128 block scales folded in: bf16(fp32(q) * s), one rounding.
+    if (FP8) {
+      const int ct = threadIdx.x - 320;   // 0..127
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      const int sld = p.ncols >> 7;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, p, mb, nb);
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          const float* srow = p.scales + static_cast<int64_t>((kb * BK) >> 7) * sld + nb * 2;
+          // a plain projection with an odd number of 128-column blocks has a last
+          // tile whose second half lies past the weight (TMA fills it with zeros)
+          const float s0 = __ldg(srow), s1 = (nb * 2 + 1 < sld) ? __ldg(srow + 1) : 0.f;
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[s], ph, ctl, kSiteConvFull))) { ok = false; break; }
+          const uint8_t* e4 = stage_e4(s);
+          uint8_t* wt = stage_b(s);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int u = ct + 128 * i;          // 64 rows x 16 chunks of 16 bytes
+            const int k = u >> 4;
+            const int n0 = (u & 15) * 16;
+            e4m3x16_scale_to_bf16_sw128(e4 + k * BN + n0, n0 < 128 ? s0 : s1, wt, k, n0);
+          }
+          fence_proxy_async_smem();   // generic-proxy writes -> visible to tcgen05.mma
+          mbar_arrive(&bars.conv[s]);
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+    }
   } else if (warp < 6) {
     // ------------------------------------------------------------ sum-of-squares reducers
     const int row = (warp - 2) * 32 + lane;
@@ -297,12 +356,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool FP8>
 cudaError_t launch_impl(const CallArgs& a) {
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, BM, BK)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d, a.ncols, BK, 64))
+  if (FP8) {
+    if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.d, a.ncols, BK, BN, false))
+      return cudaErrorInvalidValue;
+  } else if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d, a.ncols, BK, 64)) {
     return cudaErrorInvalidValue;
+  }
   Params p;
   p.M = static_cast<int>(a.M);
   p.d = static_cast<int>(a.d);
@@ -318,16 +381,19 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.status = static_cast<unsigned int*>(a.ws);
   p.budget_ns = a.budget_ns;
   p.withhold = a.withhold;
-  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU>>(static_cast<int>(SMEM_BYTES));
+  p.scales = a.scales;
+  constexpr size_t SMEM_BYTES = smem_bytes<FP8>();
+  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU, FP8>>(static_cast<int>(SMEM_BYTES));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
-  return launch_pdl(tc_kernel<SWIGLU>, grid, NUM_THREADS, SMEM_BYTES, a.stream, tx, tw, p);
+  return launch_pdl(tc_kernel<SWIGLU, FP8>, grid, Cfg<FP8>::NUM_THREADS, SMEM_BYTES, a.stream, tx, tw, p);
 }
 
 }  // namespace tc
 
 cudaError_t launch_tc(const CallArgs& a) {
-  return a.swiglu ? tc::launch_impl<true>(a) : tc::launch_impl<false>(a);
+  if (a.wtype == 1) return a.swiglu ? tc::launch_impl<true, true>(a) : tc::launch_impl<false, true>(a);
+  return a.swiglu ? tc::launch_impl<true, false>(a) : tc::launch_impl<false, false>(a);
 }
 
 }  // namespace fn

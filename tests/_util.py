@@ -53,3 +53,24 @@ def sample_cols(N: int, seed: int, per_tile: int = 8, tile: int = 128) -> np.nda
     for t0 in range(0, N, tile):
         cols.extend(rng.choice(np.arange(t0, min(N, t0 + tile)), size=min(per_tile, tile), replace=False))
     return np.unique(np.asarray(cols, dtype=np.int64))
+
+
+def fold_fp8_ref(W0, g, W1=None, col_chunk: int = 1024):
+    """The oracle's fp8 fold (codes, fp32 block scales), computed in column
+    chunks of whole 128-column blocks; with W1 the gate/up tiles are
+    interleaved per 128 columns like the stored layout."""
+    def one(W):
+        d, N = W.shape
+        q = np.empty((d, N), dtype=np.uint8)
+        s = np.empty((d // 128, N // 128), dtype=np.float32)
+        for c0 in range(0, N, col_chunk):
+            c1 = min(N, c0 + col_chunk)
+            q[:, c0:c1], s[:, c0 // 128:c1 // 128] = O.fold_fp8(W[:, c0:c1], g)
+        return q, s
+    if W1 is None:
+        return one(W0)
+    qg, sg = one(W0)
+    qu, su = one(W1)
+    s = np.empty((sg.shape[0], 2 * sg.shape[1]), dtype=np.float32)
+    s[:, 0::2], s[:, 1::2] = sg, su
+    return O.interleave128(qg, qu), s

@@ -293,6 +293,19 @@ def test_fold_fp8_properties():
     assert np.array_equal(q, want)
 
 
+def test_dequant_bf16_rounding_matches_torch_route():
+    """bf16(fp32(e4m3(q)) * s): torch computes the same product and cast."""
+    rng = np.random.default_rng(13)
+    q = rng.integers(0, 256, size=(256, 384), dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0                                  # no NaN codes
+    s = (10.0 ** rng.uniform(-4, 1, size=(2, 3))).astype(np.float32)
+    got = O.dequant_fp8_bf16_bits(q, s)
+    qt = torch.from_numpy(q).view(torch.float8_e4m3fn).float()
+    st = torch.from_numpy(np.repeat(np.repeat(s, 128, 0), 128, 1))
+    want = (qt * st).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+
+
 def test_dequant_exact():
     q = np.array([[0x38, 0x7E], [0x01, 0xC0]], dtype=np.uint8)
     q = np.tile(q, (64, 64))
