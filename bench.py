@@ -416,53 +416,84 @@ def main():
     _stage("warm-up done")
 
     # Timed region: K steps, each replaying a CUDA graph of one step (the way a
-    # decode loop issues work).  Graph p holds calls p*len(Ms) .. onward of the
-    # weight-copy rotation, so consecutive calls always read different copies;
-    # each graph also records an event pair around every launch, which gives
-    # the kernel's own duration on the launching stream.
+    # decode loop issues work).  Graph p holds calls p*len(Ms) .. of the
+    # weight-copy rotation, so consecutive calls always read different copies.
+    # Event records between kernels would break the programmatic launch
+    # overlap between consecutive calls, so the graphs that carry the per-call
+    # event pairs are separate copies, replayed in every 8th step of the timed
+    # region; they give the calls' own durations on the launching stream.
     K = args.steps
     n_calls = len(Ms)
-    period = S.copies // math.gcd(n_calls, S.copies)
-    n_graphs = period * max(1, math.ceil(16 / period))
-    graphs = []
+    # G steps per graph (at least 16 calls, as a decode loop captures many
+    # layers per graph); a tail of K mod G steps uses one-step graphs.
+    G = max(1, min(K, math.ceil(16 / n_calls)))
+    per_graph = G * n_calls
+    n_graphs = S.copies // math.gcd(per_graph, S.copies)
+    n_graphs = n_graphs * max(1, math.ceil(8 / n_graphs))
     cap_stream = torch.cuda.Stream()
-    launches0 = fnb.fn_kernel_launches()
-    for gi in range(n_graphs):
-        S.i = (gi * n_calls) % S.copies
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n_calls)]
+
+    def capture(start_call, steps, with_events):
+        S.i = start_call % S.copies
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * steps * n_calls)] \
+            if with_events else []
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=cap_stream):
-            for j, M in enumerate(Ms):
-                evs[2 * j].record()
-                S.call(M)
-                evs[2 * j + 1].record()
-        graphs.append((gr, evs))
-    kernels_per_step = (fnb.fn_kernel_launches() - launches0) // n_graphs
-    _stage(f"{n_graphs} graphs captured, {kernels_per_step} kernels per step")
+            for st in range(steps):
+                for j, M in enumerate(Ms):
+                    if with_events:
+                        evs[2 * (st * n_calls + j)].record()
+                    S.call(M)
+                    if with_events:
+                        evs[2 * (st * n_calls + j) + 1].record()
+        return gr, evs
+
+    launches0 = fnb.fn_kernel_launches()
+    clean = [capture(gi * per_graph, G, False)[0] for gi in range(n_graphs)]
+    kernels_per_step = (fnb.fn_kernel_launches() - launches0) // (n_graphs * G)
+    timed = [capture(gi * per_graph, G, True) for gi in range(n_graphs)]
+    tail = [capture(j * n_calls, 1, False)[0] for j in range(K % G)]
+    _stage(f"{2 * n_graphs} graphs of {G} steps captured, {kernels_per_step} kernels per step")
     for gi in range(max(args.warmup, n_graphs)):
-        graphs[gi % n_graphs][0].replay()
+        clean[gi % n_graphs].replay()
+        timed[gi % n_graphs][0].replay()
+    for gr in tail:
+        gr.replay()
     torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
+    instrumented = set()
+    n_full = K // G
     with ClockSampler(local) as clocks:
         t_start.record(stream)
-        for k in range(K):
-            graphs[k % n_graphs][0].replay()
+        for k in range(n_full):
+            gi = k % n_graphs
+            if k % 8 == 7:
+                timed[gi][0].replay()
+                instrumented.add(gi)
+            else:
+                clean[gi].replay()
+        for gr in tail:
+            gr.replay()
         t_end.record(stream)
         torch.cuda.synchronize()
-    barrier(world)
     _stage("timed region done")
+    barrier(world)
     elapsed_ms = t_start.elapsed_time(t_end)
     job_units, job_ms = aggregate(float(bytes_per_step if hbm_bound else flops_per_step) * K, elapsed_ms,
                                   world, dev)
     gpu_launches = K * kernels_per_step
-    # per-launch durations: the last replay of each graph inside the timed region
+    # per-call durations: the last replay of each instrumented graph in the timed region
     kernel_ms, kernel_n = 0.0, 0
-    for gi in range(min(n_graphs, K)):
-        evs = graphs[gi][1]
-        for j in range(n_calls):
-            kernel_ms += evs[2 * j].elapsed_time(evs[2 * j + 1])
+    if not instrumented:   # too few steps for an instrumented replay inside the timed region
+        for gi in range(n_graphs):
+            timed[gi][0].replay()
+            instrumented.add(gi)
+        torch.cuda.synchronize()
+    for gi in sorted(instrumented):
+        evs = timed[gi][1]
+        for c in range(G * n_calls):
+            kernel_ms += evs[2 * c].elapsed_time(evs[2 * c + 1])
             kernel_n += 1
 
     value_bytes = job_units / (job_ms / 1e3) if hbm_bound else 0.0
@@ -479,7 +510,8 @@ def main():
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "traffic": traffic, "kernel": "decode_kernel (+ decode_fixup_kernel): one fn_norm_proj call",
                     "peak_source": f"hbm_gbs ({peaks_kind})",
-                    "bytes_per_launch": per_launch_bytes, "avg_launch_us": kernel_avg_ms * 1e3}
+                    "bytes_per_launch": per_launch_bytes, "avg_launch_us": kernel_avg_ms * 1e3,
+                    "stream_us_per_call": job_ms / K / n_calls * 1e3}
         value, unit = value_bytes / 1e9, "GB/s"
     else:
         # burst peak for a kernel that ran at full clock, sustained when the
@@ -495,7 +527,8 @@ def main():
                     "frac": achieved / peak, "traffic": traffic, "kernel": "tc_kernel: one fn_norm_proj call",
                     "peak_source": f"bf16_tflops{'_sustained' if capped else ''} ({peaks_kind})",
                     "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
-                    "flops_per_launch": per_launch_flops, "avg_launch_us": kernel_avg_ms * 1e3}
+                    "flops_per_launch": per_launch_flops, "avg_launch_us": kernel_avg_ms * 1e3,
+                    "stream_us_per_call": job_ms / K / n_calls * 1e3}
         value, unit = value_flops / 1e12, "TFLOP/s"
 
     # end to end through the public API: pinned host x -> device -> call -> host y
@@ -560,8 +593,9 @@ def main():
             "config": {"workload": wl.name, "M": Ms, "d": wl.d, "N": wl.N, "swiglu": wl.swiglu,
                        "weights": wl.wtype, "parallelism": f"replicas x{world} (rows shard, no collective)",
                        "l2": f"{S.copies} rotating W' copies ({S.copies * S.Wp[0].numel() * S.Wp[0].element_size() / 1e6:.0f} MB > L2)",
-                       "step": f"{len(Ms)} fused calls, one per M, replayed as one CUDA graph",
-                       "kernel_timing": f"event pairs around each call, last replay of {min(n_graphs, K)} graphs",
+                       "step": f"{len(Ms)} fused calls, one per M; CUDA graphs of {G} steps",
+                       "kernel_timing": "event pairs around each call in the instrumented graphs "
+                                        "(every 8th step of the timed region)",
                        "kernels_per_step": kernels_per_step},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks.summary(),
             "gpu_launches": gpu_launches, "unfused_chain": chain,

@@ -86,7 +86,11 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
 /*
  * fn_workspace_size — bytes of workspace a call with these sizes needs.
  * The workspace holds a 256-byte header (the device status word) and, for
- * M <= 64, the per-CTA partial sums of the split-K decode path.  Zero it once
+ * M <= 64, the per-CTA partial sums of the split-K decode path; with fp8
+ * weights and M >= 1024 it also holds one bf16 copy of the weight, converted
+ * once per call with the same rounding the on-chip conversion uses
+ * (bf16(fp32(q) * s)), because converting each weight tile once per 128-row
+ * tile would repeat that work M/128 times.  Zero it once
  * before its first use (the status word must start at zero); the calls keep
  * the status word at zero unless a device-side wait times out.  Depends on
  * the SM count of the current device (148 is assumed when no device is
@@ -184,8 +188,13 @@ uint64_t fn_kernel_launches(void);
  *                             the previous kernel; value = mode | (k_blocks << 8),
  *                             mode 0 off, 1 TMA prefetch, 2 per-thread prefetch
  *                             (default: mode 2, 8 k-blocks)
+ *   FN_DEBUG_CLUSTER          decode path: 1 (default) split K inside thread-block
+ *                             clusters when the column tiles fill at most half the SMs,
+ *                             with the largest cluster size whose clusters all fit at
+ *                             once; 2..8 start from that size; 0 always stream-K + fix-up
  */
-enum { FN_DEBUG_WAIT_BUDGET_NS = 1, FN_DEBUG_WITHHOLD_ARRIVE = 2, FN_DEBUG_FORCE_PATH = 3, FN_DEBUG_PREFETCH = 4 };
+enum { FN_DEBUG_WAIT_BUDGET_NS = 1, FN_DEBUG_WITHHOLD_ARRIVE = 2, FN_DEBUG_FORCE_PATH = 3, FN_DEBUG_PREFETCH = 4,
+       FN_DEBUG_CLUSTER = 5 };
 fn_status fn_set_debug(int key, int64_t value);
 
 #ifdef __cplusplus

@@ -26,6 +26,7 @@ std::atomic<int> g_withhold{0};
 std::atomic<int> g_force_path{0};
 std::atomic<int> g_prefetch_iters{8};
 std::atomic<int> g_prefetch_mode{2};
+std::atomic<int> g_cluster_mode{1};
 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
@@ -152,7 +153,10 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   int sms = 0;
   fn_status st = check_device(sms);
   if (st != FN_OK) return st;
-  const size_t need = use_decode ? decode_workspace_bytes(M, d, ncols, swiglu, sms) : kWsHeaderBytes;
+  const bool dequant_once = wt == FN_W_FP8_E4M3_B128 && !use_decode && M >= kFp8DequantOnceM;
+  const size_t need = use_decode     ? decode_workspace_bytes(M, d, ncols, swiglu, sms)
+                      : dequant_once ? kWsHeaderBytes + wbytes * 2
+                                     : kWsHeaderBytes;
   if (ws_bytes < need) return FN_ERR_WORKSPACE;
 
   CallArgs a;
@@ -175,6 +179,15 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.withhold = g_withhold.load();
   a.prefetch_iters = g_prefetch_iters.load();
   a.prefetch_mode = g_prefetch_mode.load();
+  a.cluster_mode = g_cluster_mode.load();
+  if (dequant_once) {
+    // the bf16 weight bf16(fp32(q) * s), the rounding the on-chip conversion uses
+    void* wbf = static_cast<uint8_t*>(ws) + kWsHeaderBytes;
+    if (launch_dequant_fp8(Wp, scales, d, ncols, wbf, a.stream) != cudaSuccess) return FN_ERR_CUDA;
+    a.Wp = wbf;
+    a.wtype = FN_W_BF16;
+    a.scales = nullptr;
+  }
   const cudaError_t e = use_decode ? launch_decode(a) : launch_tc(a);
   return e == cudaSuccess ? FN_OK : FN_ERR_CUDA;
 }
@@ -216,10 +229,14 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
 }
 
 size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swiglu) {
-  (void)wt;
   if (M <= 0 || d <= 0 || N <= 0 || d % 64 != 0 || N % 128 != 0) return kWsHeaderBytes;
-  if (M > 64) return kWsHeaderBytes;
-  return decode_workspace_bytes(M, d, swiglu ? 2 * N : N, swiglu != 0, current_sms_or_default());
+  const int64_t ncols = swiglu ? 2 * N : N;
+  if (M > 64) {
+    if (wt == FN_W_FP8_E4M3_B128 && M >= kFp8DequantOnceM)
+      return kWsHeaderBytes + static_cast<size_t>(d) * static_cast<size_t>(ncols) * 2;
+    return kWsHeaderBytes;
+  }
+  return decode_workspace_bytes(M, d, ncols, swiglu != 0, current_sms_or_default());
 }
 
 fn_status fn_norm_proj(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
@@ -315,6 +332,10 @@ fn_status fn_set_debug(int key, int64_t value) {
     case FN_DEBUG_FORCE_PATH:
       if (value < 0 || value > 2) return FN_ERR_INVALID_ARG;
       g_force_path.store(static_cast<int>(value));
+      return FN_OK;
+    case FN_DEBUG_CLUSTER:
+      if (value < 0 || value > 8) return FN_ERR_INVALID_ARG;
+      g_cluster_mode.store(static_cast<int>(value));
       return FN_OK;
     case FN_DEBUG_PREFETCH:
       if (value < 0 || (value & 0xFF) > 2) return FN_ERR_INVALID_ARG;

@@ -28,7 +28,9 @@
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
 //   warps 2-3   sum-of-squares reducers (one thread per activation row)
+//   warps 8-11  fp8 weights only: e4m3 -> bf16 operand conversion
 //   warps 4-7   epilogue / fix-up (one thread per weight column of the tile)
+#include <atomic>
 #include <cstddef>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -40,23 +42,29 @@ namespace fn {
 namespace dec {
 
 constexpr int BK = 64;
-// 8 warps: producer, MMA, 2 reducers, 4 epilogue; fp8 weights add 2 converter warps
+// 8 warps: producer, MMA, 2 reducers, 4 epilogue; fp8 weights add 4 converter warps
 template <bool FP8>
-__host__ __device__ constexpr int num_threads() { return FP8 ? 320 : 256; }
+__host__ __device__ constexpr int num_threads() { return FP8 ? 384 : 256; }
 constexpr int W_BOX_BYTES = 64 * BK * 2;   // 64 columns x 64 k rows, bf16
 constexpr int SMEM_BUDGET = 200 * 1024;   // pipeline stages; barriers and staging come on top
 
 enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteRedFull, kSiteRedSsqEmpty,
                   kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain, kSiteMmaConv, kSiteConvFull };
 
+// bf16 weights: one TMA ring whose stages hold the weight tile and the x tile.
+// fp8 weights: a deeper TMA ring of (x tile, e4m3 tile) stages and two bf16
+// operand buffers that the converters fill and the MMA releases, so that many
+// e4m3 tiles are in flight while only two bf16 tiles take shared memory.
 template <int MPAD, int HALVES, bool FP8 = false>
 struct Cfg {
   static constexpr int W_BYTES = HALVES * 2 * W_BOX_BYTES;          // bf16 operand: 16 or 32 KB
   static constexpr int X_BYTES = MPAD * BK * 2;                     // 2, 4 or 8 KB
   static constexpr int E4_BYTES = FP8 ? HALVES * 128 * BK : 0;      // e4m3 staging: 8 or 16 KB
-  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + E4_BYTES;  // multiple of 1024
-  static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int NB = FP8 ? 2 : 0;                            // bf16 operand buffers (fp8)
+  static constexpr int STAGE_BYTES = (FP8 ? 0 : W_BYTES) + X_BYTES + E4_BYTES;  // multiple of 1024
+  static constexpr int STAGES_RAW = (SMEM_BUDGET - NB * W_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_MAX = FP8 ? 12 : 8;
+  static constexpr int STAGES = STAGES_RAW > STAGES_MAX ? STAGES_MAX : STAGES_RAW;
   static constexpr int ACC_COLS = HALVES * MPAD;                    // one accumulator buffer
   static constexpr int TMEM_COLS = 2 * ACC_COLS;                    // double buffered: 32..256
   static constexpr int SLOT_FLOATS = ((HALVES * MPAD * 128 + MPAD) + 31) / 32 * 32;
@@ -77,12 +85,13 @@ struct Params {
   int prefetch_iters;        // k-blocks per CTA prefetched into L2 before the dependency wait
   int prefetch_mode;         // 0 none, 1 TMA prefetch, 2 per-thread prefetch from idle warps
   const float* scales;       // fp8: block scales [d/128][ncols/128]
+  int cluster;               // > 1: split-K inside clusters of this many CTAs, one tile each
 };
 
 template <int MPAD, int HALVES, int STAGES>
 struct alignas(16) Bars {
   uint64_t full[STAGES], empty[STAGES];
-  uint64_t conv[STAGES];     // fp8: the stage's weight tile has been converted to bf16
+  uint64_t conv_full[2], conv_empty[2];   // fp8: bf16 operand buffer converted / released
   uint64_t acc_full[2], acc_empty[2];
   uint64_t ssq_full[2], ssq_empty[2];
   uint64_t drain;
@@ -91,6 +100,7 @@ struct alignas(16) Bars {
   uint32_t tmem_base;
   int abort_flag;
   int epi_ok[2];
+  float rfix[MPAD];          // cluster mode: 1/rms of each row
 };
 
 __device__ __forceinline__ long long it_begin(int c, const Params& p) {
@@ -154,22 +164,37 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
   using B = Bars<MPAD, HALVES, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  B& bars = *reinterpret_cast<B*>(smem + STAGES * C::STAGE_BYTES);
+  B& bars = *reinterpret_cast<B*>(smem + STAGES * C::STAGE_BYTES + C::NB * C::W_BYTES);
+  // bf16 stage: [weight tile][x tile]; fp8 stage: [x tile][e4m3 tile]; fp8 bf16
+  // operand buffers follow the ring.  Every region starts on a 1024-byte multiple.
   auto stage_w = [&](int s) { return smem + s * C::STAGE_BYTES; };
-  auto stage_x = [&](int s) { return smem + s * C::STAGE_BYTES + C::W_BYTES; };
-  auto stage_e4 = [&](int s) { return smem + s * C::STAGE_BYTES + C::W_BYTES + C::X_BYTES; };
+  auto stage_x = [&](int s) { return smem + s * C::STAGE_BYTES + (FP8 ? 0 : C::W_BYTES); };
+  auto stage_e4 = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES; };
+  auto bufb = [&](int bb) { return smem + STAGES * C::STAGE_BYTES + bb * C::W_BYTES; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  const long long it0 = it_begin(cta, p);
-  const long long it1 = it_begin(cta + 1, p);
+  // stream-K: an even share of all (tile, k block) iterations; cluster mode:
+  // cluster c owns tile c and its CTAs split the tile's k blocks by rank
+  long long it0, it1;
+  if (p.cluster > 1) {
+    const int tile = cta / p.cluster, rank = cta % p.cluster;
+    it0 = static_cast<long long>(tile) * p.kblocks + static_cast<long long>(rank) * p.kblocks / p.cluster;
+    it1 = static_cast<long long>(tile) * p.kblocks + static_cast<long long>(rank + 1) * p.kblocks / p.cluster;
+  } else {
+    it0 = it_begin(cta, p);
+    it1 = it_begin(cta + 1, p);
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1 + 2);   // MMA commit + two reducer warps
-      mbar_init(&bars.conv[s], 64);       // fp8: every converter thread
+    }
+    for (int bb = 0; bb < 2; ++bb) {
+      mbar_init(&bars.conv_full[bb], 128);  // fp8: every converter thread
+      mbar_init(&bars.conv_empty[bb], 1);   // fp8: MMA commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
@@ -272,6 +297,7 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
       uint32_t ph = 0;
       bool ok = true;
       int seg = 0;
+      int gi = 0;   // running iteration count (fp8 operand buffer rotation)
       for (long long it = it0; it < it1 && ok; ++seg) {
         const int tile = static_cast<int>(it / p.kblocks);
         const int kb0 = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
@@ -280,11 +306,12 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
         const uint32_t aph = (seg >> 1) & 1;
         if (!mbar_wait(&bars.acc_empty[b], aph ^ 1, ctl, kSiteMmaAccEmpty)) break;
         tc_fence_after();
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb, ++gi) {
+          const int bb = gi & 1;
           if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
-          if (FP8 && !mbar_wait(&bars.conv[s], ph, ctl, kSiteMmaConv)) { ok = false; break; }
+          if (FP8 && !mbar_wait(&bars.conv_full[bb], (gi >> 1) & 1, ctl, kSiteMmaConv)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t w0 = smem_u32(stage_w(s));
+          const uint32_t w0 = smem_u32(FP8 ? bufb(bb) : stage_w(s));
           const uint32_t x0 = smem_u32(stage_x(s));
 #pragma unroll
           for (int h = 0; h < HALVES; ++h) {
@@ -300,6 +327,7 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
             }
           }
           umma_commit(&bars.empty[s]);
+          if (FP8) umma_commit(&bars.conv_empty[bb]);
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
         if (!ok) break;
@@ -342,34 +370,38 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
     // e4m3 tile (64 k rows x 128*HALVES bytes, unswizzled) -> bf16 operand tile
     // with the 128x128 block scale folded in: bf16(fp32(q) * s), one rounding.
     if (FP8) {
-      const int ct = threadIdx.x - 256;                 // 0..63
+      const int ct = threadIdx.x - 256;                 // 0..127
       constexpr int UNITS_PER_ROW = 8 * HALVES;         // 16-byte e4m3 chunks per k row
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      int gi = 0;
       for (long long it = it0; it < it1 && ok;) {
         const int tile = static_cast<int>(it / p.kblocks);
         const int kb0 = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
         const int kb1 = static_cast<int>(min(static_cast<long long>(p.kblocks), kb0 + (it1 - it)));
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb, ++gi) {
+          const int bb = gi & 1;
           const int scale_row = (kb * BK) >> 7;
           float sc[HALVES];
 #pragma unroll
           for (int h = 0; h < HALVES; ++h) sc[h] = __ldg(p.scales + static_cast<int64_t>(scale_row) * (p.ncols >> 7) +
                                                          tile * HALVES + h);
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[s], ph, ctl, kSiteConvFull))) { ok = false; break; }
+          bool ready = mbar_wait(&bars.full[s], ph, ctl, kSiteConvFull);
+          ready = ready && mbar_wait(&bars.conv_empty[bb], ((gi >> 1) & 1) ^ 1, ctl, kSiteConvFull);
+          if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
           const uint8_t* e4 = stage_e4(s);
-          uint8_t* wt = stage_w(s);
+          uint8_t* wt = bufb(bb);
 #pragma unroll
-          for (int i = 0; i < BK * UNITS_PER_ROW / 64; ++i) {
-            const int u = ct + 64 * i;
+          for (int i = 0; i < BK * UNITS_PER_ROW / 128; ++i) {
+            const int u = ct + 128 * i;
             const int k = u / UNITS_PER_ROW;
             const int n0 = (u % UNITS_PER_ROW) * 16;
             const float scale = (HALVES == 2 && n0 >= 128) ? sc[HALVES - 1] : sc[0];
             e4m3x16_scale_to_bf16_sw128(e4 + k * (128 * HALVES) + n0, scale, wt, k, n0);
           }
           fence_proxy_async_smem();   // generic-proxy writes -> visible to tcgen05.mma
-          mbar_arrive(&bars.conv[s]);
+          mbar_arrive(&bars.conv_full[bb]);
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
         it += kb1 - kb0;
@@ -420,6 +452,20 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
         store_tile_rows(bars.ybuf, p, tile, et);
         continue;
       }
+      if (p.cluster > 1) {
+        // Cluster mode: this CTA's only segment.  Its pipeline stages are idle
+        // now (every MMA and every reducer read has completed), so the partial
+        // accumulators [half][row][column] and sums of squares go there for the
+        // peers to read over distributed shared memory after the cluster barrier.
+        float* red = reinterpret_cast<float*>(smem);
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h)
+#pragma unroll
+          for (int m = 0; m < MPAD; ++m) red[(h * MPAD + m) * 128 + n] = acc[h][m];
+        if (et < MPAD) red[HALVES * MPAD * 128 + et] = bars.ssq[b][et];
+        mbar_arrive(&bars.ssq_empty[b]);
+        continue;
+      }
       // Split tile: publish this CTA's partial for the fix-up kernel.  A slot
       // holds float4 groups [half][row / 4][column] (a warp's 16-byte accesses
       // are contiguous), only for the rows < M, then the MPAD partial sums of
@@ -438,6 +484,52 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
       if (et < MPAD) __stcg(part + HALVES * MPAD * 128 + et, bars.ssq[b][et]);
       mbar_arrive(&bars.ssq_empty[b]);
     }
+  }
+
+  if (p.cluster > 1) {
+    // every CTA of the cluster has its partial in shared memory
+    cluster_sync_all();
+    if (warp >= 4 && warp < 8) {
+      const int et = threadIdx.x - 128;
+      const uint32_t S = static_cast<uint32_t>(p.cluster);
+      const uint32_t rank = cluster_ctarank();
+      const int tile = cta / p.cluster;
+      const float* red = reinterpret_cast<const float*>(smem);
+      uint32_t base[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) base[q] = q < static_cast<int>(S) ? dsmem_addr(red, q) : 0u;
+      if (et < p.M && et < MPAD) {
+        float ss = 0.f;                      // partial sums of squares in rank (= k) order
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < static_cast<int>(S)) ss += dsmem_ld_f32(base[q] + 4u * (HALVES * MPAD * 128 + et));
+        bars.rfix[et] = inv_rms(ss, p.inv_d, p.eps);
+      }
+      named_bar_sync(1, 128);
+      // this rank finishes a contiguous share of the tile's (row, column) outputs
+      const int E = p.M * 128;
+      const int lo = static_cast<int>(static_cast<long long>(rank) * E / S);
+      const int hi = static_cast<int>(static_cast<long long>(rank + 1) * E / S);
+#pragma unroll 2
+      for (int e = lo + et; e < hi; e += 128) {
+        const int m = e >> 7, nn = e & 127;
+        float g = 0.f, u = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q < static_cast<int>(S)) {
+            g += dsmem_ld_f32(base[q] + 4u * (m * 128 + nn));
+            if (HALVES == 2) u += dsmem_ld_f32(base[q] + 4u * ((MPAD + m) * 128 + nn));
+          }
+        }
+        const float r = bars.rfix[m];
+        float v = g * r;
+        if (HALVES == 2) v = silu_f32(v) * (u * r);
+        const int col = tile * 128 + nn;
+        if (col < p.nout) p.y[static_cast<int64_t>(m) * p.nout + col] = __float2bfloat16_rn(v);
+      }
+    }
+    // no CTA may leave while a peer still reads its shared memory
+    cluster_sync_all();
   }
 
   tc_fence_before();
@@ -525,11 +617,57 @@ using BarsLarge = Bars<64, 2, 5>;
 static_assert(offsetof(BarsSmall, ybuf) % 16 == 0 && offsetof(BarsLarge, ybuf) % 16 == 0,
               "ybuf must be 16-byte aligned");
 static_assert(Cfg<64, 2, true>::STAGES >= 2 && Cfg<64, 2, false>::STAGES >= 2, "pipeline needs two stages");
+// cluster mode reuses the ring for its partials: HALVES x MPAD x 128 floats + MPAD
+static_assert(Cfg<64, 2, true>::STAGES * Cfg<64, 2, true>::STAGE_BYTES >= (2 * 64 * 128 + 64) * 4 &&
+                  Cfg<64, 2, false>::STAGES * Cfg<64, 2, false>::STAGE_BYTES >= (2 * 64 * 128 + 64) * 4,
+              "cluster partials must fit the ring");
 
 template <int MPAD, int HALVES, bool FP8>
 constexpr size_t smem_bytes() {
   using C = Cfg<MPAD, HALVES, FP8>;
-  return 1024 + C::STAGES * C::STAGE_BYTES + sizeof(Bars<MPAD, HALVES, C::STAGES>);
+  return 1024 + C::STAGES * C::STAGE_BYTES + C::NB * C::W_BYTES + sizeof(Bars<MPAD, HALVES, C::STAGES>);
+}
+
+// Cluster size for split-K with a distributed-shared-memory reduction: as
+// many CTAs per column tile as the SMs allow (at most 8, at most one per k
+// block); 1 when the tiles alone already occupy half the SMs or more.
+inline int cluster_split(int tiles, int kblocks, int num_sms) {
+  if (tiles * 2 > num_sms) return 1;
+  int S = num_sms / tiles;
+  if (S > 8) S = 8;
+  if (S > kblocks) S = kblocks;
+  return S;
+}
+
+// Whether `tiles` clusters of S CTAs can all be resident at once (cached per
+// device and cluster size).
+template <auto Kernel>
+bool clusters_fit(int S, int tiles, int threads, size_t smem) {
+  static std::atomic<int> cache[64][9];   // 0 unknown, else max active clusters + 1
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64 || S > 8) return false;
+  int v = cache[dev][S].load(std::memory_order_relaxed);
+  if (v == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles * S));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, Kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    v = n + 1;
+    cache[dev][S].store(v, std::memory_order_relaxed);
+  }
+  return v - 1 >= tiles;
 }
 
 struct Layout {
@@ -584,9 +722,27 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.prefetch_iters = a.prefetch_iters;
   p.prefetch_mode = a.prefetch_mode;
   p.scales = a.scales;
+  p.cluster = 1;
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES, FP8>();
   cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES, FP8>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
+  // Split K inside clusters when the tiles fill the GPU at least twice over
+  // and every cluster can be resident at once; otherwise stream-K.
+  // The largest cluster size whose clusters can all be resident (GPC sizes
+  // decide that, not just the SM count), or the size forced by the caller.
+  int S = a.cluster_mode >= 2 ? a.cluster_mode : cluster_split(L.tiles, L.kblocks, a.num_sms);
+  if (S > L.kblocks) S = L.kblocks;
+  if (S > 8) S = 8;
+  while (S >= 2 && !clusters_fit<decode_kernel<MPAD, HALVES, FP8>>(S, L.tiles, num_threads<FP8>(), SMEM)) --S;
+  // Clusters only pay off when they occupy about as many SMs as stream-K
+  // would: fewer SMs cannot pull the full HBM bandwidth.
+  const long long sk_ctas = L.total < a.num_sms ? L.total : a.num_sms;
+  if (S >= 2 && a.cluster_mode != 0 && (a.cluster_mode >= 2 || 10LL * L.tiles * S >= 9LL * sk_ctas)) {
+    p.cluster = S;
+    p.grid = L.tiles * S;
+    return launch_pdl_cluster(decode_kernel<MPAD, HALVES, FP8>, static_cast<unsigned>(p.grid), S,
+                              num_threads<FP8>(), SMEM, a.stream, tx, tw, p);
+  }
   e = launch_pdl(decode_kernel<MPAD, HALVES, FP8>, L.grid, num_threads<FP8>(), SMEM, a.stream, tx, tw, p);
   if (e != cudaSuccess) return e;
   if (L.grid <= L.tiles) {

@@ -13,6 +13,10 @@ namespace fn {
 // Workspace header: the first 256 bytes hold the device status word.
 constexpr size_t kWsHeaderBytes = 256;
 
+// fp8 weights at M >= this: dequantise the weight once per call into the
+// workspace (bf16) instead of converting every weight tile once per row tile.
+constexpr int64_t kFp8DequantOnceM = 1024;
+
 // One fused norm+projection call, validated by the ABI layer.
 struct CallArgs {
   const void* x;          // bf16 [M, d]
@@ -33,6 +37,7 @@ struct CallArgs {
   int withhold;           // test knob: withhold one reducer arrival
   int prefetch_iters;     // decode: weight k-blocks per CTA prefetched into L2 early
   int prefetch_mode;      // decode: 0 none, 1 TMA prefetch, 2 per-thread prefetch
+  int cluster_mode;       // decode: 1 allow split-K inside clusters, 0 stream-K only
 };
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -99,6 +104,29 @@ cudaError_t launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) count_launch();
+  return e;
+}
+
+// Same, with thread-block clusters of `cluster` CTAs along x.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kernel)(Params...), unsigned grid, int cluster, unsigned block, size_t smem,
+                               cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   if (e == cudaSuccess) count_launch();
   return e;

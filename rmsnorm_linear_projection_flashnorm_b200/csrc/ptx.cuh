@@ -31,6 +31,28 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Thread-block clusters: rank of this CTA, a barrier over every thread of the
+// cluster (release/acquire orders shared-memory writes before peers' reads),
+// and loads from a peer CTA's shared memory (distributed shared memory).
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // Programmatic dependent launch: wait until the preceding grid in the stream
 // has completed and its writes are visible; allow the next grid to launch.
 __device__ __forceinline__ void grid_dependency_wait() {
@@ -300,14 +322,21 @@ __device__ __forceinline__ void e4m3x16_scale_to_bf16_sw128(const uint8_t* src16
   const uint4 v = *reinterpret_cast<const uint4*>(src16);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[8];
+  // (s, s) as a packed f32 pair for the sm_100a paired multiply
+  const uint64_t s2 = (static_cast<uint64_t>(__float_as_uint(s)) << 32) | __float_as_uint(s);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const __half2_raw hr =
-          __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>((w[j] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-      o[2 * j + h] = pack_bf16x2(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
+      uint32_t h2;   // two e4m3 -> two f16 (exact)
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(w[j] >> (16 * h))));
+      float lo, hi;  // f16 -> f32 (exact)
+      asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(static_cast<uint16_t>(h2 & 0xFFFFu)));
+      asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(static_cast<uint16_t>(h2 >> 16)));
+      uint64_t p2 = (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+      asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(p2) : "l"(s2));   // fp32 products, IEEE rounding
+      o[2 * j + h] = pack_bf16x2(__uint_as_float(static_cast<uint32_t>(p2)),
+                                 __uint_as_float(static_cast<uint32_t>(p2 >> 32)));
     }
   }
   const int j0 = (n0 & 63) >> 3;

@@ -18,8 +18,8 @@
 // released it; an accumulator buffer is reused only after the epilogue
 // drained it.
 //
-// Layout: one persistent CTA per SM, 10 warps (14 with fp8 weights: warps
-// 10-13 convert each staged e4m3 weight tile to the bf16 operand tile).
+// Layout: one persistent CTA per SM, 10 warps (18 with fp8 weights: warps
+// 10-17 convert each staged e4m3 weight tile to the bf16 operand tile).
 //   warp 0      TMA producer: x tile 128x64 (K-major) and W' tile 64x256
 //               (four 64-column boxes, N-major), 128-byte swizzle, 4 stages
 //   warp 1      TMEM owner and MMA issuer (tcgen05.mma M=128 N=256 K=16)
@@ -44,11 +44,11 @@ constexpr int E4_BYTES = BN * BK;               // fp8 weights: 16 KB e4m3 stagi
 constexpr int TMEM_COLS = 2 * BN;
 
 // bf16 weights: 4 stages of 48 KB, 10 warps.  fp8 weights: 3 stages of 64 KB
-// (x, bf16 operand, e4m3 staging) and 4 more warps converting e4m3 to bf16.
+// (x, bf16 operand, e4m3 staging) and 8 more warps converting e4m3 to bf16.
 template <bool FP8> struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + (FP8 ? E4_BYTES : 0);
   static constexpr int STAGES = FP8 ? 3 : 4;
-  static constexpr int NUM_THREADS = FP8 ? 448 : 320;
+  static constexpr int NUM_THREADS = FP8 ? 576 : 320;
 };
 constexpr int GROUP_M = 16;                     // tile raster: bands of 16 row blocks
 
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1 + 4);  // MMA commit + one arrival per reducer warp
-      mbar_init(&bars.conv[s], 128);     // fp8: every converter thread
+      mbar_init(&bars.conv[s], 256);     // fp8: every converter thread
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
     // e4m3 tile (64 k rows x 256 bytes, unswizzled) -> bf16 operand tile with
     // the 128x128 block scales folded in: bf16(fp32(q) * s), one rounding.
     if (FP8) {
-      const int ct = threadIdx.x - 320;   // 0..127
+      const int ct = threadIdx.x - 320;   // 0..255
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
           const uint8_t* e4 = stage_e4(s);
           uint8_t* wt = stage_b(s);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int u = ct + 128 * i;          // 64 rows x 16 chunks of 16 bytes
+          for (int i = 0; i < 4; ++i) {
+            const int u = ct + 256 * i;          // 64 rows x 16 chunks of 16 bytes
             const int k = u >> 4;
             const int n0 = (u & 15) * 16;
             e4m3x16_scale_to_bf16_sw128(e4 + k * BN + n0, n0 < 128 ? s0 : s1, wt, k, n0);

@@ -221,3 +221,21 @@ def test_repeated_calls_bit_identical():
     for _ in range(50):
         assert torch.equal(run(x, Wp, 768, 1e-6, ws=ws), first)
     assert ws.status()[0] == fnb.FN_OK
+
+
+@pytest.mark.parametrize("cluster", [0, 1])
+@pytest.mark.parametrize("M,d,N,swiglu", [(1, 4096, 6144, False), (40, 4096, 6144, False), (8, 1024, 1024, True),
+                                          (64, 640, 1280, True), (17, 2048, 256, False)])
+def test_decode_cluster_and_stream_k_agree_with_oracle(cluster, M, d, N, swiglu):
+    """The decode path either splits K inside thread-block clusters (reduced over
+    distributed shared memory) or uses stream-K with the fix-up kernel; both
+    must match the oracle."""
+    fnb.fn_set_debug(fnb.FN_DEBUG_CLUSTER, cluster)
+    try:
+        if swiglu:
+            y, ref, _ = _swiglu_case(M, d, N, seed=97)
+        else:
+            y, ref, _ = _plain_case(M, d, N, seed=97)
+        assert rel_err(y, ref) <= BF16_TOL
+    finally:
+        fnb.fn_set_debug(fnb.FN_DEBUG_CLUSTER, 1)

@@ -63,6 +63,8 @@ def _case(M, d, N, swiglu, seed):
     (300, 512, 384, True),     # tile SwiGLU, ragged M
     (64, 128, 128, False),     # single k block, single tile
     (129, 640, 640, True),
+    (1100, 256, 256, True),    # M >= 1024: the weight is dequantised once into the workspace
+    (1024, 384, 384, False),
 ])
 def test_fp8_small(M, d, N, swiglu):
     y, ref = _case(M, d, N, swiglu, seed=131)
