@@ -28,70 +28,40 @@
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
 //   warps 2-3   sum-of-squares reducers (one thread per activation row)
-//   warps 8-11  fp8 weights only: e4m3 -> bf16 operand conversion
 //   warps 4-7   epilogue / fix-up (one thread per weight column of the tile)
+//
+// This file holds the bf16-weight kernel; fp8 weights have their own kernel
+// (decode_fp8.cu) that feeds the e4m3 tiles to the tensor cores unconverted.
 #include <atomic>
 #include <cstddef>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include "internal.h"
-#include "ptx.cuh"
+#include "decode_common.cuh"
 
 namespace fn {
 namespace dec {
 
-constexpr int BK = 64;
-// 8 warps: producer, MMA, 2 reducers, 4 epilogue; fp8 weights add 4 converter warps
-template <bool FP8>
-__host__ __device__ constexpr int num_threads() { return FP8 ? 384 : 256; }
+constexpr int NUM_THREADS = 256;   // producer, MMA, 2 reducers, 4 epilogue warps
 constexpr int W_BOX_BYTES = 64 * BK * 2;   // 64 columns x 64 k rows, bf16
 constexpr int SMEM_BUDGET = 200 * 1024;   // pipeline stages; barriers and staging come on top
 
-enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteRedFull, kSiteRedSsqEmpty,
-                  kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain, kSiteMmaConv, kSiteConvFull };
-
-// bf16 weights: one TMA ring whose stages hold the weight tile and the x tile.
-// fp8 weights: a deeper TMA ring of (x tile, e4m3 tile) stages and two bf16
-// operand buffers that the converters fill and the MMA releases, so that many
-// e4m3 tiles are in flight while only two bf16 tiles take shared memory.
-template <int MPAD, int HALVES, bool FP8 = false>
+// One TMA ring whose stages hold the weight tile and the x tile.
+template <int MPAD, int HALVES>
 struct Cfg {
   static constexpr int W_BYTES = HALVES * 2 * W_BOX_BYTES;          // bf16 operand: 16 or 32 KB
   static constexpr int X_BYTES = MPAD * BK * 2;                     // 2, 4 or 8 KB
-  static constexpr int E4_BYTES = FP8 ? HALVES * 128 * BK : 0;      // e4m3 staging: 8 or 16 KB
-  static constexpr int NB = FP8 ? 2 : 0;                            // bf16 operand buffers (fp8)
-  static constexpr int STAGE_BYTES = (FP8 ? 0 : W_BYTES) + X_BYTES + E4_BYTES;  // multiple of 1024
-  static constexpr int STAGES_RAW = (SMEM_BUDGET - NB * W_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES_MAX = FP8 ? 12 : 8;
-  static constexpr int STAGES = STAGES_RAW > STAGES_MAX ? STAGES_MAX : STAGES_RAW;
+  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;             // multiple of 1024
+  static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int ACC_COLS = HALVES * MPAD;                    // one accumulator buffer
   static constexpr int TMEM_COLS = 2 * ACC_COLS;                    // double buffered: 32..256
-  static constexpr int SLOT_FLOATS = ((HALVES * MPAD * 128 + MPAD) + 31) / 32 * 32;
-};
-
-struct Params {
-  int M, d, ncols, nout;
-  int kblocks, tiles;
-  long long total;   // tiles * kblocks
-  int grid;
-  float eps, inv_d;
-  __nv_bfloat16* y;
-  float* part;               // [grid][2][SLOT_FLOATS]
-  unsigned int* status;
-  unsigned long long budget_ns;
-  int withhold;
-  const uint8_t* wp;         // folded weight base (L2 prefetch addresses)
-  int prefetch_iters;        // k-blocks per CTA prefetched into L2 before the dependency wait
-  int prefetch_mode;         // 0 none, 1 TMA prefetch, 2 per-thread prefetch from idle warps
-  const float* scales;       // fp8: block scales [d/128][ncols/128]
-  int cluster;               // > 1: split-K inside clusters of this many CTAs, one tile each
+  static constexpr int SLOT_FLOATS = slot_floats<MPAD, HALVES>();
 };
 
 template <int MPAD, int HALVES, int STAGES>
 struct alignas(16) Bars {
   uint64_t full[STAGES], empty[STAGES];
-  uint64_t conv_full[2], conv_empty[2];   // fp8: bf16 operand buffer converted / released
   uint64_t acc_full[2], acc_empty[2];
   uint64_t ssq_full[2], ssq_empty[2];
   uint64_t drain;
@@ -103,74 +73,19 @@ struct alignas(16) Bars {
   float rfix[MPAD];          // cluster mode: 1/rms of each row
 };
 
-__device__ __forceinline__ long long it_begin(int c, const Params& p) {
-  return static_cast<long long>(c) * p.total / p.grid;
-}
-// CTA whose iteration range holds iteration `it`
-__device__ __forceinline__ int owner_of(long long it, const Params& p) {
-  return static_cast<int>(((it + 1) * p.grid - 1) / p.total);
-}
-
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long budget) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > budget) return;
-  }
-}
-
-// Copy the staged output rows of one 128-column tile to y with 16-byte
-// stores: 16 consecutive threads write one 256-byte row segment.  The next
-// write to the staging buffer happens only after the epilogue group's next
-// named barrier, which every thread reaches after finishing this copy.
-__device__ __forceinline__ void store_tile_rows(const __nv_bfloat16* ybuf, const Params& p, int tile, int et) {
-  const int col0 = tile * 128;
-  const int chunks = p.M * 16;
-  for (int i = et; i < chunks; i += 128) {
-    const int m = i >> 4, c16 = i & 15;
-    if (col0 + c16 * 8 < p.nout) {
-      const uint4 v = *reinterpret_cast<const uint4*>(ybuf + m * 128 + c16 * 8);
-      *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m) * p.nout + col0 + c16 * 8) = v;
-    }
-  }
-}
-
-template <int MPAD>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[MPAD]) {
-  if constexpr (MPAD == 16) {
-    uint32_t r[16];
-    tmem_ld16(taddr, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-  } else {
-#pragma unroll
-    for (int c = 0; c < MPAD; c += 32) {
-      uint32_t r[32];
-      tmem_ld32(taddr + c, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[c + j] = __uint_as_float(r[j]);
-    }
-  }
-}
-
-template <int MPAD, int HALVES, bool FP8>
-__global__ void __launch_bounds__(num_threads<FP8>(), 1)
+template <int MPAD, int HALVES>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   const Params p) {
-  using C = Cfg<MPAD, HALVES, FP8>;
-  constexpr int NUM_THREADS = num_threads<FP8>();
+  using C = Cfg<MPAD, HALVES>;
   constexpr int STAGES = C::STAGES;
   using B = Bars<MPAD, HALVES, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  B& bars = *reinterpret_cast<B*>(smem + STAGES * C::STAGE_BYTES + C::NB * C::W_BYTES);
-  // bf16 stage: [weight tile][x tile]; fp8 stage: [x tile][e4m3 tile]; fp8 bf16
-  // operand buffers follow the ring.  Every region starts on a 1024-byte multiple.
+  B& bars = *reinterpret_cast<B*>(smem + STAGES * C::STAGE_BYTES);
+  // stage: [weight tile][x tile], each on a 1024-byte multiple
   auto stage_w = [&](int s) { return smem + s * C::STAGE_BYTES; };
-  auto stage_x = [&](int s) { return smem + s * C::STAGE_BYTES + (FP8 ? 0 : C::W_BYTES); };
-  auto stage_e4 = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES; };
-  auto bufb = [&](int bb) { return smem + STAGES * C::STAGE_BYTES + bb * C::W_BYTES; };
+  auto stage_x = [&](int s) { return smem + s * C::STAGE_BYTES + C::W_BYTES; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -191,10 +106,6 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1 + 2);   // MMA commit + two reducer warps
-    }
-    for (int bb = 0; bb < 2; ++bb) {
-      mbar_init(&bars.conv_full[bb], 128);  // fp8: every converter thread
-      mbar_init(&bars.conv_empty[bb], 1);   // fp8: MMA commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
@@ -227,14 +138,11 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
     for (long long it = it0; it < it1 && n_pf < p.prefetch_iters; ++it, ++n_pf) {
       const int tile = static_cast<int>(it / p.kblocks);
       const int kb = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
-#pragma unroll
-      if (FP8) tma_prefetch_l2_2d(&tmap_w, tile * 128 * HALVES, kb * BK);
-      else
-        for (int bx = 0; bx < 2 * HALVES; ++bx) tma_prefetch_l2_2d(&tmap_w, tile * 128 * HALVES + bx * 64, kb * BK);
+      for (int bx = 0; bx < 2 * HALVES; ++bx) tma_prefetch_l2_2d(&tmap_w, tile * 128 * HALVES + bx * 64, kb * BK);
     }
   } else if (p.prefetch_mode == 2 && warp >= 2) {
     // one 128-byte line per thread and step: (k row, 128-byte column chunk)
-    constexpr int WB = FP8 ? 1 : 2;                    // weight bytes per element
+    constexpr int WB = 2;                              // weight bytes per element
     const int lines_per_row = HALVES * WB;             // 128 * HALVES * WB bytes of a k row per tile
     const long long n_it = min(static_cast<long long>(p.prefetch_iters), it1 - it0);
     const int total = static_cast<int>(n_it) * BK * lines_per_row;
@@ -267,18 +175,12 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
         const int kb1 = static_cast<int>(min(static_cast<long long>(p.kblocks), kb0 + (it1 - it)));
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&bars.empty[s], ph ^ 1, ctl, kSiteProdEmpty)) { ok = false; break; }
-          // TMA fills x and either the bf16 weight boxes or the e4m3 staging tile
-          mbar_arrive_expect_tx(&bars.full[s], C::X_BYTES + (FP8 ? C::E4_BYTES : C::W_BYTES));
+          mbar_arrive_expect_tx(&bars.full[s], C::X_BYTES + C::W_BYTES);
           tma_load_2d(stage_x(s), &tmap_x, &bars.full[s], kb * BK, 0);
-          if (FP8) {
-            // one unswizzled box of 128 * HALVES e4m3 columns x 64 k rows
-            tma_load_2d_hint(stage_e4(s), &tmap_w, &bars.full[s], tile * 128 * HALVES, kb * BK, w_policy);
-          } else {
 #pragma unroll
-            for (int bx = 0; bx < 2 * HALVES; ++bx)
-              tma_load_2d_hint(stage_w(s) + bx * W_BOX_BYTES, &tmap_w, &bars.full[s],
-                               tile * 128 * HALVES + bx * 64, kb * BK, w_policy);
-          }
+          for (int bx = 0; bx < 2 * HALVES; ++bx)
+            tma_load_2d_hint(stage_w(s) + bx * W_BOX_BYTES, &tmap_w, &bars.full[s],
+                             tile * 128 * HALVES + bx * 64, kb * BK, w_policy);
           issued |= 1u << s;
           last_ph = (last_ph & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -297,7 +199,6 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
       uint32_t ph = 0;
       bool ok = true;
       int seg = 0;
-      int gi = 0;   // running iteration count (fp8 operand buffer rotation)
       for (long long it = it0; it < it1 && ok; ++seg) {
         const int tile = static_cast<int>(it / p.kblocks);
         const int kb0 = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
@@ -306,12 +207,10 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
         const uint32_t aph = (seg >> 1) & 1;
         if (!mbar_wait(&bars.acc_empty[b], aph ^ 1, ctl, kSiteMmaAccEmpty)) break;
         tc_fence_after();
-        for (int kb = kb0; kb < kb1; ++kb, ++gi) {
-          const int bb = gi & 1;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
-          if (FP8 && !mbar_wait(&bars.conv_full[bb], (gi >> 1) & 1, ctl, kSiteMmaConv)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t w0 = smem_u32(FP8 ? bufb(bb) : stage_w(s));
+          const uint32_t w0 = smem_u32(stage_w(s));
           const uint32_t x0 = smem_u32(stage_x(s));
 #pragma unroll
           for (int h = 0; h < HALVES; ++h) {
@@ -327,7 +226,6 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
             }
           }
           umma_commit(&bars.empty[s]);
-          if (FP8) umma_commit(&bars.conv_empty[bb]);
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
         if (!ok) break;
@@ -364,48 +262,6 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
       if (row < MPAD) bars.ssq[b][row] = acc;
       if (!(p.withhold && seg == 0)) mbar_arrive(&bars.ssq_full[b]);
       it += kb1 - kb0;
-    }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ fp8 converters
-    // e4m3 tile (64 k rows x 128*HALVES bytes, unswizzled) -> bf16 operand tile
-    // with the 128x128 block scale folded in: bf16(fp32(q) * s), one rounding.
-    if (FP8) {
-      const int ct = threadIdx.x - 256;                 // 0..127
-      constexpr int UNITS_PER_ROW = 8 * HALVES;         // 16-byte e4m3 chunks per k row
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      int gi = 0;
-      for (long long it = it0; it < it1 && ok;) {
-        const int tile = static_cast<int>(it / p.kblocks);
-        const int kb0 = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
-        const int kb1 = static_cast<int>(min(static_cast<long long>(p.kblocks), kb0 + (it1 - it)));
-        for (int kb = kb0; kb < kb1; ++kb, ++gi) {
-          const int bb = gi & 1;
-          const int scale_row = (kb * BK) >> 7;
-          float sc[HALVES];
-#pragma unroll
-          for (int h = 0; h < HALVES; ++h) sc[h] = __ldg(p.scales + static_cast<int64_t>(scale_row) * (p.ncols >> 7) +
-                                                         tile * HALVES + h);
-          bool ready = mbar_wait(&bars.full[s], ph, ctl, kSiteConvFull);
-          ready = ready && mbar_wait(&bars.conv_empty[bb], ((gi >> 1) & 1) ^ 1, ctl, kSiteConvFull);
-          if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
-          const uint8_t* e4 = stage_e4(s);
-          uint8_t* wt = bufb(bb);
-#pragma unroll
-          for (int i = 0; i < BK * UNITS_PER_ROW / 128; ++i) {
-            const int u = ct + 128 * i;
-            const int k = u / UNITS_PER_ROW;
-            const int n0 = (u % UNITS_PER_ROW) * 16;
-            const float scale = (HALVES == 2 && n0 >= 128) ? sc[HALVES - 1] : sc[0];
-            e4m3x16_scale_to_bf16_sw128(e4 + k * (128 * HALVES) + n0, scale, wt, k, n0);
-          }
-          fence_proxy_async_smem();   // generic-proxy writes -> visible to tcgen05.mma
-          mbar_arrive(&bars.conv_full[bb]);
-          if (++s == STAGES) { s = 0; ph ^= 1; }
-        }
-        it += kb1 - kb0;
-      }
     }
   } else {
     // ------------------------------------------------------------ epilogue / fix-up
@@ -449,7 +305,7 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
         }
         mbar_arrive(&bars.ssq_empty[b]);
         named_bar_sync(1, 128);
-        store_tile_rows(bars.ybuf, p, tile, et);
+        store_tile_rows(bars.ybuf, p, tile, et, 128);
         continue;
       }
       if (p.cluster > 1) {
@@ -540,92 +396,21 @@ __global__ void __launch_bounds__(num_threads<FP8>(), 1)
   }
 }
 
-// Fix-up of the tiles whose k range was split between CTAs.  One thread per
-// (tile, row group of 4, column): it loads the float4 partials of every
-// contributing CTA (up to four in flight at once), adds them in ascending k
-// order together with the partial sums of squares of its four rows, applies
-// 1/rms (and SwiGLU) and stores four bf16 outputs.
-constexpr int FIX_THREADS = 128;
-
-template <int MPAD, int HALVES>
-__global__ void __launch_bounds__(FIX_THREADS) decode_fixup_kernel(const Params p) {
-  using C = Cfg<MPAD, HALVES>;
-  // Let the next kernel in the stream launch now: its CTAs take SMs as the
-  // stream-K CTAs leave and prefetch their weights into L2 meanwhile.  All
-  // CTAs of the stream-K grid are resident by now (each triggered this
-  // launch after its own start), so no generation can starve another.
-  grid_launch_dependents();
-  grid_dependency_wait();        // the partials of the stream-K kernel are complete and visible
-  const int Q = (p.M + 3) >> 2;
-  const long long gid = static_cast<long long>(blockIdx.x) * FIX_THREADS + threadIdx.x;
-  const int n = static_cast<int>(gid & 127);
-  const long long rest = gid >> 7;
-  const int q = static_cast<int>(rest % Q);
-  const int tile = static_cast<int>(rest / Q);
-  if (tile >= p.tiles) return;
-  const long long t_it0 = static_cast<long long>(tile) * p.kblocks;
-  const int c_first = owner_of(t_it0, p);
-  const int c_last = owner_of(t_it0 + p.kblocks - 1, p);
-  if (c_first == c_last) return;   // finished by the stream-K kernel itself
-  float4 acc[HALVES];
-#pragma unroll
-  for (int h = 0; h < HALVES; ++h) acc[h] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float4 ss = make_float4(0.f, 0.f, 0.f, 0.f);
-  auto add = [](float4& t, const float4& v) { t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w; };
-  constexpr int CB = 4;
-  for (int c0 = c_first; c0 <= c_last; c0 += CB) {
-    float4 v[CB][HALVES], s4[CB];
-#pragma unroll
-    for (int j = 0; j < CB; ++j) {
-      const int c = c0 + j;
-      if (c <= c_last) {
-        const int slot = c * 2 + (it_begin(c, p) >= t_it0 ? 0 : 1);
-        const float4* base = reinterpret_cast<const float4*>(p.part + static_cast<int64_t>(slot) * C::SLOT_FLOATS);
-#pragma unroll
-        for (int h = 0; h < HALVES; ++h) v[j][h] = __ldcg(base + (h * (MPAD / 4) + q) * 128 + n);
-        s4[j] = __ldcg(base + HALVES * (MPAD / 4) * 128 + q);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < CB; ++j) {
-      if (c0 + j <= c_last) {
-#pragma unroll
-        for (int h = 0; h < HALVES; ++h) add(acc[h], v[j][h]);
-        add(ss, s4[j]);
-      }
-    }
-  }
-  const float a0[4] = {acc[0].x, acc[0].y, acc[0].z, acc[0].w};
-  const float a1[4] = {acc[HALVES - 1].x, acc[HALVES - 1].y, acc[HALVES - 1].z, acc[HALVES - 1].w};
-  const float sq[4] = {ss.x, ss.y, ss.z, ss.w};
-  const int col = tile * 128 + n;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = 4 * q + i;
-    if (m >= p.M) break;
-    const float r = inv_rms(sq[i], p.inv_d, p.eps);
-    float v = a0[i] * r;
-    if (HALVES == 2) v = silu_f32(v) * (a1[i] * r);
-    if (col < p.nout) p.y[static_cast<int64_t>(m) * p.nout + col] = __float2bfloat16_rn(v);
-  }
-}
-
 // The staging buffer is read as 16-byte vectors; the barrier block itself is
 // placed at a 1024-byte multiple.
 using BarsSmall = Bars<16, 1, 8>;
 using BarsLarge = Bars<64, 2, 5>;
 static_assert(offsetof(BarsSmall, ybuf) % 16 == 0 && offsetof(BarsLarge, ybuf) % 16 == 0,
               "ybuf must be 16-byte aligned");
-static_assert(Cfg<64, 2, true>::STAGES >= 2 && Cfg<64, 2, false>::STAGES >= 2, "pipeline needs two stages");
+static_assert(Cfg<64, 2>::STAGES >= 2, "pipeline needs two stages");
 // cluster mode reuses the ring for its partials: HALVES x MPAD x 128 floats + MPAD
-static_assert(Cfg<64, 2, true>::STAGES * Cfg<64, 2, true>::STAGE_BYTES >= (2 * 64 * 128 + 64) * 4 &&
-                  Cfg<64, 2, false>::STAGES * Cfg<64, 2, false>::STAGE_BYTES >= (2 * 64 * 128 + 64) * 4,
+static_assert(Cfg<64, 2>::STAGES * Cfg<64, 2>::STAGE_BYTES >= (2 * 64 * 128 + 64) * 4,
               "cluster partials must fit the ring");
 
-template <int MPAD, int HALVES, bool FP8>
+template <int MPAD, int HALVES>
 constexpr size_t smem_bytes() {
-  using C = Cfg<MPAD, HALVES, FP8>;
-  return 1024 + C::STAGES * C::STAGE_BYTES + C::NB * C::W_BYTES + sizeof(Bars<MPAD, HALVES, C::STAGES>);
+  using C = Cfg<MPAD, HALVES>;
+  return 1024 + C::STAGES * C::STAGE_BYTES + sizeof(Bars<MPAD, HALVES, C::STAGES>);
 }
 
 // Cluster size for split-K with a distributed-shared-memory reduction: as
@@ -670,101 +455,57 @@ bool clusters_fit(int S, int tiles, int threads, size_t smem) {
   return v - 1 >= tiles;
 }
 
-struct Layout {
-  int tiles, kblocks, grid;
-  long long total;
-  size_t part_off, bytes;
-};
-
 template <int MPAD, int HALVES>
-Layout layout_for(int64_t d, int64_t ncols, int num_sms) {
-  Layout L;
-  L.tiles = static_cast<int>(ncols / (128 * HALVES));
-  L.kblocks = static_cast<int>(d / BK);
-  L.total = static_cast<long long>(L.tiles) * L.kblocks;
-  L.grid = static_cast<int>(L.total < num_sms ? L.total : num_sms);
-  L.part_off = kWsHeaderBytes;
-  L.bytes = L.part_off + static_cast<size_t>(L.grid) * 2 * Cfg<MPAD, HALVES>::SLOT_FLOATS * 4;
-  return L;
-}
-
-template <int MPAD, int HALVES, bool FP8>
 cudaError_t launch_impl(const CallArgs& a) {
-  const Layout L = layout_for<MPAD, HALVES>(a.d, a.ncols, a.num_sms);
-  if (a.ws_bytes < L.bytes) return cudaErrorInvalidValue;
+  if (a.ws_bytes < workspace_bytes<MPAD, HALVES>(a.d, a.ncols, a.num_sms)) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, MPAD, BK)) return cudaErrorInvalidValue;
-  if (FP8) {
-    // e4m3 bytes, one unswizzled box of 128 * HALVES columns x 64 k rows per stage
-    if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.d, a.ncols, BK, 128 * HALVES, false))
-      return cudaErrorInvalidValue;
-  } else if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d, a.ncols, BK, 64)) {
-    return cudaErrorInvalidValue;
-  }
+  if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d, a.ncols, BK, 64)) return cudaErrorInvalidValue;
   Params p;
   p.M = static_cast<int>(a.M);
   p.d = static_cast<int>(a.d);
   p.ncols = static_cast<int>(a.ncols);
   p.nout = static_cast<int>(a.N);
-  p.kblocks = L.kblocks;
-  p.tiles = L.tiles;
-  p.total = L.total;
-  p.grid = L.grid;
+  p.kblocks = static_cast<int>(a.d / BK);
+  p.tiles = static_cast<int>(a.ncols / (128 * HALVES));
+  p.total = static_cast<long long>(p.tiles) * p.kblocks;
+  p.grid = static_cast<int>(p.total < a.num_sms ? p.total : a.num_sms);
   p.eps = a.eps;
   p.inv_d = 1.0f / static_cast<float>(a.d);
   p.y = static_cast<__nv_bfloat16*>(a.y);
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
   p.status = reinterpret_cast<unsigned int*>(ws);
-  p.part = reinterpret_cast<float*>(ws + L.part_off);
+  p.part = reinterpret_cast<float*>(ws + kWsHeaderBytes);
   p.budget_ns = a.budget_ns;
   p.withhold = a.withhold;
   p.wp = static_cast<const uint8_t*>(a.Wp);
   p.prefetch_iters = a.prefetch_iters;
   p.prefetch_mode = a.prefetch_mode;
-  p.scales = a.scales;
+  p.scales = nullptr;
   p.cluster = 1;
-  constexpr size_t SMEM = smem_bytes<MPAD, HALVES, FP8>();
-  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES, FP8>>(static_cast<int>(SMEM));
+  constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
+  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
   // Split K inside clusters when the tiles fill the GPU at least twice over
   // and every cluster can be resident at once; otherwise stream-K.
   // The largest cluster size whose clusters can all be resident (GPC sizes
   // decide that, not just the SM count), or the size forced by the caller.
-  int S = a.cluster_mode >= 2 ? a.cluster_mode : cluster_split(L.tiles, L.kblocks, a.num_sms);
-  if (S > L.kblocks) S = L.kblocks;
+  int S = a.cluster_mode >= 2 ? a.cluster_mode : cluster_split(p.tiles, p.kblocks, a.num_sms);
+  if (S > p.kblocks) S = p.kblocks;
   if (S > 8) S = 8;
-  while (S >= 2 && !clusters_fit<decode_kernel<MPAD, HALVES, FP8>>(S, L.tiles, num_threads<FP8>(), SMEM)) --S;
+  while (S >= 2 && !clusters_fit<decode_kernel<MPAD, HALVES>>(S, p.tiles, NUM_THREADS, SMEM)) --S;
   // Clusters only pay off when they occupy about as many SMs as stream-K
   // would: fewer SMs cannot pull the full HBM bandwidth.
-  const long long sk_ctas = L.total < a.num_sms ? L.total : a.num_sms;
-  if (S >= 2 && a.cluster_mode != 0 && (a.cluster_mode >= 2 || 10LL * L.tiles * S >= 9LL * sk_ctas)) {
+  if (S >= 2 && a.cluster_mode != 0 && (a.cluster_mode >= 2 || 10LL * p.tiles * S >= 9LL * p.grid)) {
     p.cluster = S;
-    p.grid = L.tiles * S;
-    return launch_pdl_cluster(decode_kernel<MPAD, HALVES, FP8>, static_cast<unsigned>(p.grid), S,
-                              num_threads<FP8>(), SMEM, a.stream, tx, tw, p);
+    p.grid = p.tiles * S;
+    return launch_pdl_cluster(decode_kernel<MPAD, HALVES>, static_cast<unsigned>(p.grid), S, NUM_THREADS, SMEM,
+                              a.stream, tx, tw, p);
   }
-  e = launch_pdl(decode_kernel<MPAD, HALVES, FP8>, L.grid, num_threads<FP8>(), SMEM, a.stream, tx, tw, p);
+  e = launch_pdl(decode_kernel<MPAD, HALVES>, p.grid, NUM_THREADS, SMEM, a.stream, tx, tw, p);
   if (e != cudaSuccess) return e;
-  if (L.grid <= L.tiles) {
-    // every CTA's range covers whole tiles only when the grid is at most the
-    // tile count and divides the iterations evenly; otherwise some tile is split
-    bool split = false;
-    for (int c = 0; c < L.grid && !split; ++c) {
-      const long long b0 = static_cast<long long>(c) * L.total / L.grid;
-      const long long b1 = static_cast<long long>(c + 1) * L.total / L.grid;
-      split = (b0 % L.kblocks) != 0 || (b1 % L.kblocks) != 0;
-    }
-    if (!split) return cudaSuccess;
-  }
-  const long long threads = static_cast<long long>(L.tiles) * 128 * ((a.M + 3) / 4);
-  const unsigned fgrid = static_cast<unsigned>((threads + FIX_THREADS - 1) / FIX_THREADS);
-  return launch_pdl(decode_fixup_kernel<MPAD, HALVES>, fgrid, FIX_THREADS, 0, a.stream, p);
-}
-
-template <int MPAD>
-cudaError_t launch_halves(const CallArgs& a) {
-  if (a.wtype == 1) return a.swiglu ? launch_impl<MPAD, 2, true>(a) : launch_impl<MPAD, 1, true>(a);
-  return a.swiglu ? launch_impl<MPAD, 2, false>(a) : launch_impl<MPAD, 1, false>(a);
+  if (!any_split_tile(p.grid, p.total, p.kblocks)) return cudaSuccess;
+  return launch_fixup<MPAD, HALVES>(p, a.stream);
 }
 
 }  // namespace dec
@@ -774,20 +515,21 @@ int decode_mpad(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms) {
   const int mp = decode_mpad(M);
   if (swiglu) {
-    if (mp == 16) return dec::layout_for<16, 2>(d, ncols, num_sms).bytes;
-    if (mp == 32) return dec::layout_for<32, 2>(d, ncols, num_sms).bytes;
-    return dec::layout_for<64, 2>(d, ncols, num_sms).bytes;
+    if (mp == 16) return dec::workspace_bytes<16, 2>(d, ncols, num_sms);
+    if (mp == 32) return dec::workspace_bytes<32, 2>(d, ncols, num_sms);
+    return dec::workspace_bytes<64, 2>(d, ncols, num_sms);
   }
-  if (mp == 16) return dec::layout_for<16, 1>(d, ncols, num_sms).bytes;
-  if (mp == 32) return dec::layout_for<32, 1>(d, ncols, num_sms).bytes;
-  return dec::layout_for<64, 1>(d, ncols, num_sms).bytes;
+  if (mp == 16) return dec::workspace_bytes<16, 1>(d, ncols, num_sms);
+  if (mp == 32) return dec::workspace_bytes<32, 1>(d, ncols, num_sms);
+  return dec::workspace_bytes<64, 1>(d, ncols, num_sms);
 }
 
 cudaError_t launch_decode(const CallArgs& a) {
   const int mp = decode_mpad(a.M);
-  if (mp == 16) return dec::launch_halves<16>(a);
-  if (mp == 32) return dec::launch_halves<32>(a);
-  return dec::launch_halves<64>(a);
+  if (a.wtype == 1) return launch_decode_fp8(a, mp);
+  if (mp == 16) return a.swiglu ? dec::launch_impl<16, 2>(a) : dec::launch_impl<16, 1>(a);
+  if (mp == 32) return a.swiglu ? dec::launch_impl<32, 2>(a) : dec::launch_impl<32, 1>(a);
+  return a.swiglu ? dec::launch_impl<64, 2>(a) : dec::launch_impl<64, 1>(a);
 }
 
 }  // namespace fn

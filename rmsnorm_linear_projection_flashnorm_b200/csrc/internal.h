@@ -55,6 +55,8 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, in
 int decode_mpad(int64_t M);
 size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms);
 cudaError_t launch_decode(const CallArgs& a);
+// fp8 weights on the decode path (decode_fp8.cu); mpad is decode_mpad(M).
+cudaError_t launch_decode_fp8(const CallArgs& a, int mpad);
 
 // Tensor-core tile path (M > 64): persistent 128x256 tiles, tcgen05 + TMEM.
 cudaError_t launch_tc(const CallArgs& a);

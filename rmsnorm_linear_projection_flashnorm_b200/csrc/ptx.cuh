@@ -236,6 +236,24 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint6
       : "memory");
 }
 
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B and an fp32
+// accumulator: the same fields as above with both operand formats 0 (e4m3).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem] with 8-bit operands (K = 32 per instruction).
+__device__ __forceinline__ void umma_e4m3(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when all previously issued tcgen05 operations of this
 // thread have completed (their smem operands may then be overwritten).
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -343,6 +361,26 @@ __device__ __forceinline__ void e4m3x16_scale_to_bf16_sw128(const uint8_t* src16
   uint8_t* row = wtile + (n0 >> 6) * 8192 + k * 128;
   *reinterpret_cast<uint4*>(row + ((j0 ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
   *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Split two fp32 values a0, a1 into e4m3 pairs hi + lo: hi = e4m3(a), lo =
+// e4m3(a - hi), both rounded to nearest even (packed two per 16 bits, a0 in
+// the low byte).  For a = (bf16 value) * 2^e with 0.25 <= |a| < 448 the
+// split is exact, a == hi + lo: hi keeps the top 4 significant bits, and
+// the remainder, at most 4 more bits of the 8-bit bf16 significand, is a
+// multiple of the e4m3 grid at its own magnitude.  The subtraction is exact
+// in fp32 (hi is a and rounded to 4 bits, within a factor of two of a).
+__device__ __forceinline__ void split_e4m3x2(float a0, float a1, uint16_t& hi, uint16_t& lo) {
+  uint16_t h, l;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(a1), "f"(a0));
+  uint32_t f2;   // the two e4m3 values back as f16 (exact)
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f2) : "h"(h));
+  float b0, b1;  // f16 -> f32 (exact)
+  asm("cvt.f32.f16 %0, %1;" : "=f"(b0) : "h"(static_cast<uint16_t>(f2 & 0xFFFFu)));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(b1) : "h"(static_cast<uint16_t>(f2 >> 16)));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(l) : "f"(a1 - b1), "f"(a0 - b0));
+  hi = h;
+  lo = l;
 }
 
 // 1 / sqrt(mean + eps) for a row, from its sum of squares over d columns.

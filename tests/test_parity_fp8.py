@@ -1,8 +1,10 @@
 """GPU parity with fp8 (e4m3, 128x128 block-scaled) folded weights.
 
-The activations stay bf16; the kernels convert each staged e4m3 weight tile
-to bf16 on chip (fp32 product with the block scale, one rounding) and run the
-bf16 MMA.  Kernel parity is against the oracle evaluated on the stored,
+The activations stay bf16.  At M > 64 the kernels convert each staged e4m3
+weight tile to bf16 on chip (fp32 product with the block scale, one rounding)
+and run the bf16 MMA; at M <= 64 the e4m3 codes go to the tensor cores as they
+are and the activations are split exactly into two e4m3 parts per 128-deep k
+block.  Kernel parity is against the oracle evaluated on the stored,
 dequantised weight W_deq = e4m3(q) * s (exact in fp64) with g = 1, within
 6e-2 (1 + |y_ref|).  The oracle's own fold provides W_deq; the GPU folds the
 same weights itself, and the fold's bit-exactness is a separate test.
@@ -15,7 +17,7 @@ import oracle as O
 import rmsnorm_linear_projection_flashnorm_b200 as fnb
 import workloads as WL
 from rmsnorm_linear_projection_flashnorm_b200 import torch_api as T
-from tests._util import FP8_TOL, fold_fp8_ref, gpu, rel_err, run, sample_cols
+from tests._util import BF16_TOL, FP8_TOL, fold_fp8_ref, gpu, rel_err, run, sample_cols
 
 pytestmark = pytest.mark.gpu
 FP8 = fnb.FN_W_FP8_E4M3_B128
@@ -40,8 +42,10 @@ def test_dequant_step_bit_exact():
     assert np.array_equal(got, O.dequant_fp8_bf16_bits(q, s))
 
 
-def _case(M, d, N, swiglu, seed):
+def _case(M, d, N, swiglu, seed, x=None):
     inp = WL.case(M, d, N, swiglu, seed=seed)
+    if x is not None:
+        inp["x"] = x
     x, g = inp["x"], inp["g"]
     if swiglu:
         Wq, s = T.fold(gpu(inp["W_gate"]), gpu(g), gpu(inp["W_up"]), wtype=FP8)
@@ -80,6 +84,61 @@ def test_fp8_both_paths_at_small_m(path):
             assert rel_err(y, ref) <= FP8_TOL
     finally:
         fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 0)
+
+
+@pytest.mark.parametrize("M", [1, 2, 15, 16, 17, 31, 32, 33, 63, 64])
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_fp8_decode_m_ladder(M, swiglu):
+    """Every padded row count of the decode kernel (16, 32, 64 rows) and both
+    scaler layouts (all rows per thread, or half of them)."""
+    y, ref = _case(M, 512, 768 if not swiglu else 384, swiglu, seed=140 + M)
+    assert rel_err(y, ref) <= FP8_TOL
+
+
+def test_fp8_decode_wide_dynamic_range_is_exact():
+    """Per row and 128-deep k block the decode kernel scales x by a power of
+    two and splits it into two e4m3 parts whose sum is the bf16 value; the
+    products with the e4m3 weight are then exact, so even activations that
+    span 2^-20 .. 2^12 inside one k block meet the bf16-weight bound."""
+    M, d, N = 6, 512, 384
+    x = WL.activations(M, d, 150).float()
+    mult = torch.ones(d)
+    mult[0::4] = 2.0 ** 10
+    mult[1::8] = 2.0 ** -12
+    mult[3::16] = 2.0 ** -18
+    x = (x * mult).to(torch.bfloat16)
+    for swiglu in (False, True):
+        y, ref = _case(M, d, N, swiglu, seed=150, x=x)
+        assert rel_err(y, ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("M", [3, 200])
+def test_fp8_non_finite_rows_give_nan_rows(M):
+    """An inf or NaN in a row makes that row's outputs NaN (its sum of squares
+    is not finite), as in the oracle; the other rows are unaffected."""
+    d, N = 256, 256
+    x = WL.activations(M, d, 151).clone()
+    x[1, 7] = float("inf")
+    x[2, 200] = float("nan")
+    y, ref = _case(M, d, N, False, seed=151, x=x)
+    assert torch.all(torch.isnan(y[1:3].float()))
+    assert rel_err(y, ref) <= FP8_TOL      # NaN positions coincide, the rest within bound
+
+
+@pytest.mark.parametrize("M,swiglu", [(1, True), (40, False), (64, True)])
+def test_fp8_decode_repeated_calls_bit_identical(M, swiglu):
+    d, N = 1024, 1024
+    inp = WL.case(M, d, N, swiglu, seed=152)
+    if swiglu:
+        Wq, s = T.fold(gpu(inp["W_gate"]), gpu(inp["g"]), gpu(inp["W_up"]), wtype=FP8)
+    else:
+        Wq, s = T.fold(gpu(inp["W"]), gpu(inp["g"]), wtype=FP8)
+    x = gpu(inp["x"])
+    ws = T.Workspace()
+    first = run(x, Wq, N, 1e-6, swiglu=swiglu, scales=s, ws=ws).clone()
+    for _ in range(200):
+        assert torch.equal(run(x, Wq, N, 1e-6, swiglu=swiglu, scales=s, ws=ws), first)
+    assert ws.status()[0] == fnb.FN_OK
 
 
 @pytest.fixture(scope="module")
