@@ -17,10 +17,14 @@
 // hi = e4m3(a) and lo = e4m3(a - hi), with a == hi + lo for every |a| >= 1/4
 // (a bf16 value has 8 significant bits, hi keeps the top 4 and lo the rest).
 // Elements below 1/4, under 2^-9 of the block's largest, are off by at most
-// 2^-10 in the scaled units.  Two MMAs per k step (hi and lo) accumulate into
-// one TMEM buffer per k block, so the block's partial sums are the exact
-// products in fp32.  Scaler warps read each block's buffer back, multiply by
-// s[b, n] * 2^-e and add it to fp32 running sums in registers.  This converts
+// 2^-10 in the scaled units.  x_hi and x_lo are stacked as the 2 x MPAD
+// columns of one B operand, so one MMA per k step gives both halves of the
+// split; each k block has its own TMEM buffer, whose partial sums are exact
+// products in fp32.  Scaler warps read each block's buffer back, add the hi
+// and lo columns, multiply by s[b, n] * 2^-e and add the result to fp32
+// running sums in registers.  (Small-N tcgen05.mma instructions cost nearly
+// as much as large ones, so the stacking halves the tensor-core time per
+// weight byte.)  This converts
 // MPAD x 128 activations per k block instead of 128 x 128 (or 128 x 256)
 // weight codes: 8 to 64 times fewer conversions (Marlin explainer, section
 // 4: the conversion must hide under the memory stream).
@@ -65,7 +69,8 @@ struct Cfg {
   static constexpr int STAGE_BYTES = W_BYTES + XB_BYTES + 2 * XQ_BYTES;   // multiple of 1024
   static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-  static constexpr int TMEM_COLS = 2 * HALVES * MPAD;      // two k-block buffers: 32..256
+  static constexpr int ACC_COLS = HALVES * 2 * MPAD;       // one k-block buffer: hi and lo columns
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;           // two k-block buffers: 64..512
   static constexpr int TPR = CONV_THREADS / MPAD;          // converter threads per row: 8, 4 or 2
   static constexpr int EPT = BKQ / TPR;                    // k elements per converter thread
 };
@@ -86,14 +91,15 @@ struct alignas(16) Bars {
   int warp_ok[8];
 };
 
-// One activation row's share of a k block: load this thread's EPT bf16
-// values from the two 64-column x boxes (128-byte swizzle), reduce the row's
-// largest magnitude and sum of squares over the row's TPR threads, and write
-// the exact e4m3 split of x * 2^e into the x_hi / x_lo operand rows
-// (K-major, 128-byte swizzle: 16-byte chunk j of row m at chunk j ^ (m & 7)).
-// Returns the row's sum of squares; *factor receives 2^-e (NaN when the
-// block holds a non-finite value, so the row's outputs become NaN as the bf16
-// path's would).
+// One activation row's share of a k block: this thread's EPT bf16 values,
+// read from the two 64-column x boxes (128-byte swizzle).  First pass: the
+// row's largest magnitude over its TPR threads, on the raw bit patterns
+// (|x| orders like its bits; inf and NaN sort above every finite value).
+// Second pass: the exact e4m3 split of x * 2^e into the x_hi / x_lo operand
+// rows (K-major, 128-byte swizzle: 16-byte chunk j of row m at chunk
+// j ^ (m & 7)) and the row's sum of squares.  Returns the sum of squares;
+// *factor receives 2^-e (NaN when the block holds a non-finite value, so the
+// row's outputs become NaN as the bf16 path's would).
 template <int MPAD, int TPR, int EPT>
 __device__ __forceinline__ float convert_row_block(const uint8_t* xb, uint8_t* xh, uint8_t* xl, int row, int sub,
                                                    bool live, float* factor) {
@@ -104,34 +110,27 @@ __device__ __forceinline__ float convert_row_block(const uint8_t* xb, uint8_t* x
     return *reinterpret_cast<const uint4*>(xb + (g >> 3) * (MPAD * 128) + row * 128 + (((g & 7) ^ (row & 7)) << 4));
   };
   uint32_t amax2 = 0;                   // |x| bit patterns, two bf16 lanes
-  float ss0 = 0.f, ss1 = 0.f;
   if (live) {
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const uint4 v = chunk(i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        amax2 = __vmaxu2(amax2, w[j] & 0x7FFF7FFFu);
-        const float lo = bf16lo_to_f32(w[j]), hi = bf16hi_to_f32(w[j]);
-        ss0 = fmaf(lo, lo, ss0);
-        ss1 = fmaf(hi, hi, ss1);
-      }
+      amax2 = __vmaxu2(amax2, v.x & 0x7FFF7FFFu);
+      amax2 = __vmaxu2(amax2, v.y & 0x7FFF7FFFu);
+      amax2 = __vmaxu2(amax2, v.z & 0x7FFF7FFFu);
+      amax2 = __vmaxu2(amax2, v.w & 0x7FFF7FFFu);
     }
   }
   uint32_t amax = max(amax2 & 0xFFFFu, amax2 >> 16);
-  float ss = ss0 + ss1;
 #pragma unroll
-  for (int o = 1; o < TPR; o <<= 1) {
-    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  }
+  for (int o = 1; o < TPR; o <<= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   // amax is a bf16 bit pattern: exponent field in bits 7..14 (255: inf / NaN)
   const int E = static_cast<int>(amax >> 7);
   int e = amax == 0 ? 0 : 134 - E;      // amax * 2^e in [128, 256)
   e = e > 126 ? 126 : (e < -126 ? -126 : e);
   const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+  const uint64_t sc2 = f2_pack(sc, sc);
   *factor = E == 255 ? __int_as_float(0x7fc00000) : __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+  uint64_t ss2 = 0;                     // two partial sums of squares (+0.0f, +0.0f)
 #pragma unroll
   for (int oc = 0; oc < EPT / 16; ++oc) {
     uint4 hv = make_uint4(0u, 0u, 0u, 0u), lv = hv;   // padding rows (TMA filled zeros) stay zero
@@ -143,11 +142,16 @@ __device__ __forceinline__ float convert_row_block(const uint8_t* xb, uint8_t* x
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          uint16_t h0, l0, h1, l1;
-          split_e4m3x2(bf16lo_to_f32(w[2 * q]) * sc, bf16hi_to_f32(w[2 * q]) * sc, h0, l0);
-          split_e4m3x2(bf16lo_to_f32(w[2 * q + 1]) * sc, bf16hi_to_f32(w[2 * q + 1]) * sc, h1, l1);
-          hw[2 * c + q] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-          lw[2 * c + q] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+          uint16_t h[2], l[2];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const uint32_t x2 = w[2 * q + t];
+            const uint64_t xf = f2_pack_u(x2 << 16, x2 & 0xFFFF0000u);   // two bf16 -> fp32 (exact)
+            ss2 = f2_fma(xf, xf, ss2);
+            split_e4m3x2(f2_mul(xf, sc2), h[t], l[t]);
+          }
+          hw[2 * c + q] = static_cast<uint32_t>(h[0]) | (static_cast<uint32_t>(h[1]) << 16);
+          lw[2 * c + q] = static_cast<uint32_t>(l[0]) | (static_cast<uint32_t>(l[1]) << 16);
         }
       }
       hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
@@ -158,6 +162,9 @@ __device__ __forceinline__ float convert_row_block(const uint8_t* xb, uint8_t* x
     *reinterpret_cast<uint4*>(xh + off) = hv;
     *reinterpret_cast<uint4*>(xl + off) = lv;
   }
+  float ss = f2_lo(ss2) + f2_hi(ss2);
+#pragma unroll
+  for (int o = 1; o < TPR; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   return ss;
 }
 
@@ -267,8 +274,9 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
     if (lane == 0) {
       // A = q^T: 128 weight columns (one 128-byte swizzle row), MN-major; 8-row
       //     k groups 1024 B apart, so K = 32 is 4096 B.
-      // B = x_hi / x_lo: MPAD activation rows of 128 e4m3 k values, K-major.
-      constexpr uint32_t IDESC = idesc_e4m3_f32(128, MPAD, /*a MN-major*/ true, /*b MN-major*/ false);
+      // B = [x_hi; x_lo]: 2 x MPAD rows of 128 e4m3 k values, K-major (x_lo's
+      //     rows follow x_hi's, so both are one operand of N = 2 x MPAD).
+      constexpr uint32_t IDESC = idesc_e4m3_f32(128, 2 * MPAD, /*a MN-major*/ true, /*b MN-major*/ false);
       int s = 0;
       uint32_t ph = 0;
       long long gi = 0;
@@ -281,15 +289,13 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
         tc_fence_after();
         const uint32_t w0 = smem_u32(stage_w(s));
         const uint32_t xh = smem_u32(stage_xh(s));
-        const uint32_t xl = smem_u32(stage_xl(s));
 #pragma unroll
         for (int h = 0; h < HALVES; ++h) {
-          const uint32_t d_tmem = tmem_base + (ab * HALVES + h) * MPAD;
+          const uint32_t d_tmem = tmem_base + (ab * HALVES + h) * 2 * MPAD;
 #pragma unroll
           for (int kk = 0; kk < BKQ / 32; ++kk) {
             const uint64_t adesc = sdesc_sw128(w0 + h * WQ_BOX + kk * 4096, WQ_BOX, 1024);
             umma_e4m3(d_tmem, adesc, sdesc_sw128(xh + kk * 32, 16, 1024), IDESC, kk != 0 ? 1u : 0u);
-            umma_e4m3(d_tmem, adesc, sdesc_sw128(xl + kk * 32, 16, 1024), IDESC, 1u);
           }
         }
         umma_commit(&bars.empty[s]);
@@ -341,12 +347,26 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
   } else {
     // ------------------------------------------------------------ scalers / epilogue
     constexpr int RPS = C::RPS;
+    constexpr int CH = HALVES * RPS >= 64 ? 8 : 16;   // TMEM columns per load
     const int st = threadIdx.x - FIRST_SCALER;        // 0 .. SCALE_THREADS-1
     const int wq = warp & 3;                          // TMEM lane quarter this warp may read
     const int n = wq * 32 + lane;                     // weight column within a 128-column half
     const int m0 = (st >> 7) * RPS;                   // first activation row of this thread
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const int scale_cols = p.ncols >> 7;
+    // Block scales of iteration `it`, loaded three iterations ahead so that
+    // the global-load latency never sits between two k blocks.
+    auto load_scales = [&](long long it, float (&sv)[HALVES]) {
+      const int t = static_cast<int>(it / p.kblocks);
+      const int k = static_cast<int>(it - static_cast<long long>(t) * p.kblocks);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h)
+        sv[h] = it < it1 ? __ldg(p.scales + static_cast<int64_t>(k) * scale_cols + t * HALVES + h) : 0.f;
+    };
+    float s0[HALVES], s1[HALVES], s2[HALVES];
+    load_scales(it0, s0);
+    load_scales(it0 + 1, s1);
+    load_scales(it0 + 2, s2);
     bool ok = true;
     long long gi = 0;
     int seg = 0;
@@ -355,18 +375,22 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
       const int kb0 = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
       const int kb1 = static_cast<int>(min(static_cast<long long>(p.kblocks), kb0 + (it1 - it)));
       it += kb1 - kb0;
-      float acc[HALVES][RPS];
+      uint64_t acc[HALVES][RPS / 2];   // fp32 running sums, rows in pairs
 #pragma unroll
       for (int h = 0; h < HALVES; ++h)
 #pragma unroll
-        for (int j = 0; j < RPS; ++j) acc[h][j] = 0.f;
+        for (int j = 0; j < RPS / 2; ++j) acc[h][j] = 0;
       for (int kb = kb0; kb < kb1; ++kb, ++gi) {
         const int ab = static_cast<int>(gi & 1);
         const int xr = static_cast<int>(gi & (XR - 1));
         float sw[HALVES];
 #pragma unroll
-        for (int h = 0; h < HALVES; ++h)
-          sw[h] = __ldg(p.scales + static_cast<int64_t>(kb) * scale_cols + tile * HALVES + h);
+        for (int h = 0; h < HALVES; ++h) {
+          sw[h] = s0[h];
+          s0[h] = s1[h];
+          s1[h] = s2[h];
+        }
+        load_scales(it0 + gi + 3, s2);
         if (ok) {
           bool ready = mbar_wait(&bars.accf[ab], static_cast<uint32_t>((gi >> 1) & 1), ctl, dec::kSiteEpiAccFull);
           ready = ready && mbar_wait(&bars.xsf[xr], static_cast<uint32_t>((gi / XR) & 1), ctl, dec::kSiteScaleFull);
@@ -374,13 +398,29 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
         }
         if (!ok) continue;    // no further waits; the group decides at the segment end
         tc_fence_after();
-        const float* f = bars.xs[xr] + m0;   // 2^-e of this thread's rows (shared-memory broadcast)
+        // 2^-e of this thread's rows, as fp32 pairs (shared-memory broadcast)
+        const uint64_t* f2 = reinterpret_cast<const uint64_t*>(bars.xs[xr] + m0);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h) {
-          float part[RPS];
-          dec::tmem_ld_cols<RPS>(tmem_base + lane_base + (ab * HALVES + h) * MPAD + m0, part);
+          const uint64_t s2 = f2_pack(sw[h], sw[h]);
+          const uint32_t col = tmem_base + lane_base + (ab * HALVES + h) * 2 * MPAD + m0;
 #pragma unroll
-          for (int j = 0; j < RPS; ++j) acc[h][j] = fmaf(part[j], sw[h] * f[j], acc[h][j]);
+          for (int c = 0; c < RPS; c += CH) {   // CH columns at a time keeps register use low
+            uint32_t ph[CH], pl[CH];            // x_hi and x_lo products of the same rows
+            if constexpr (CH == 16) {
+              tmem_ld16(col + c, ph);
+              tmem_ld16(col + MPAD + c, pl);
+            } else {
+              tmem_ld8(col + c, ph);
+              tmem_ld8(col + MPAD + c, pl);
+            }
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < CH / 2; ++j) {
+              const uint64_t sum = f2_add(f2_pack_u(ph[2 * j], ph[2 * j + 1]), f2_pack_u(pl[2 * j], pl[2 * j + 1]));
+              acc[h][c / 2 + j] = f2_fma(sum, f2_mul(f2[c / 2 + j], s2), acc[h][c / 2 + j]);
+            }
+          }
         }
         tc_fence_before();
         mbar_arrive(&bars.acce[ab]);
@@ -405,9 +445,9 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
           const int m = m0 + j;
           if (m >= p.M) break;
           const float r = inv_rms(bars.ssq[b][m], p.inv_d, p.eps);
-          float v;
-          if (HALVES == 2) v = silu_f32(acc[0][j] * r) * (acc[1][j] * r);
-          else v = acc[0][j] * r;
+          const float a0 = (j & 1) ? f2_hi(acc[0][j / 2]) : f2_lo(acc[0][j / 2]);
+          float v = a0 * r;
+          if (HALVES == 2) v = silu_f32(v) * (((j & 1) ? f2_hi(acc[1][j / 2]) : f2_lo(acc[1][j / 2])) * r);
           bars.ybuf[m * 128 + n] = __float2bfloat16_rn(v);
         }
       } else {
@@ -424,7 +464,8 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
           for (int q4 = 0; q4 < RPS / 4; ++q4)
             if (m0 / 4 + q4 < Q)
               __stcg(part4 + (h * (MPAD / 4) + m0 / 4 + q4) * 128 + n,
-                     make_float4(acc[h][4 * q4], acc[h][4 * q4 + 1], acc[h][4 * q4 + 2], acc[h][4 * q4 + 3]));
+                     make_float4(f2_lo(acc[h][2 * q4]), f2_hi(acc[h][2 * q4]), f2_lo(acc[h][2 * q4 + 1]),
+                                 f2_hi(acc[h][2 * q4 + 1])));
         if (st < MPAD) __stcg(part + HALVES * MPAD * 128 + st, bars.ssq[b][st]);
       }
       named_bar_sync(1, C::SCALE_THREADS);   // sums of squares read, staging complete
@@ -451,7 +492,7 @@ static_assert(smem_bytes<64, 2>() <= 227 * 1024 && smem_bytes<64, 1>() <= 227 * 
                   smem_bytes<16, 2>() <= 227 * 1024 && smem_bytes<32, 2>() <= 227 * 1024,
               "shared memory per CTA");
 static_assert(Cfg<64, 2>::STAGES >= 2, "pipeline needs two stages");
-static_assert(Cfg<16, 1>::TMEM_COLS == 32 && Cfg<64, 2>::TMEM_COLS == 256, "TMEM allocation is a power of two");
+static_assert(Cfg<16, 1>::TMEM_COLS == 64 && Cfg<64, 2>::TMEM_COLS == 512, "TMEM allocation: a power of two <= 512");
 
 template <int MPAD, int HALVES>
 cudaError_t launch_impl(const CallArgs& a) {

@@ -277,6 +277,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -363,22 +369,52 @@ __device__ __forceinline__ void e4m3x16_scale_to_bf16_sw128(const uint8_t* src16
   *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Split two fp32 values a0, a1 into e4m3 pairs hi + lo: hi = e4m3(a), lo =
-// e4m3(a - hi), both rounded to nearest even (packed two per 16 bits, a0 in
-// the low byte).  For a = (bf16 value) * 2^e with 0.25 <= |a| < 448 the
-// split is exact, a == hi + lo: hi keeps the top 4 significant bits, and
-// the remainder, at most 4 more bits of the 8-bit bf16 significand, is a
-// multiple of the e4m3 grid at its own magnitude.  The subtraction is exact
-// in fp32 (hi is a and rounded to 4 bits, within a factor of two of a).
-__device__ __forceinline__ void split_e4m3x2(float a0, float a1, uint16_t& hi, uint16_t& lo) {
+// Packed fp32 pairs (sm_100a paired arithmetic): lane 0 in bits 0-31.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_pack_u(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// Split two values a = (a0, a1) into e4m3 pairs hi + lo: hi = e4m3(a),
+// lo = e4m3(a - hi), rounded to nearest even, packed two per 16 bits (a0 in
+// the low byte).  The inputs are fp32 values a = (bf16 value) * 2^e with
+// |a| < 256; they pass through f16, which holds every such value with
+// |a| >= 2^-14 exactly (11 significant bits >= 8).  For |a| >= 1/4 the split
+// is exact, a == hi + lo: hi keeps the top 4 significant bits and the rest,
+// at most 4 more bits, is a multiple of the e4m3 grid at its own magnitude.
+// The f16 subtraction is exact as well (hi is within a factor of two of a,
+// or both lie on the f16 subnormal grid).  Values below 2^-10 give hi = lo = 0.
+__device__ __forceinline__ void split_e4m3x2(uint64_t a, uint16_t& hi, uint16_t& lo) {
+  uint32_t a16, b16, r16;
   uint16_t h, l;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(a1), "f"(a0));
-  uint32_t f2;   // the two e4m3 values back as f16 (exact)
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f2) : "h"(h));
-  float b0, b1;  // f16 -> f32 (exact)
-  asm("cvt.f32.f16 %0, %1;" : "=f"(b0) : "h"(static_cast<uint16_t>(f2 & 0xFFFFu)));
-  asm("cvt.f32.f16 %0, %1;" : "=f"(b1) : "h"(static_cast<uint16_t>(f2 >> 16)));
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(l) : "f"(a1 - b1), "f"(a0 - b0));
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(a16) : "f"(f2_hi(a)), "f"(f2_lo(a)));
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(h) : "r"(a16));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(b16) : "h"(h));   // hi back in f16 (exact)
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r16) : "r"(a16), "r"(b16));
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(l) : "r"(r16));
   hi = h;
   lo = l;
 }
