@@ -110,6 +110,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, but the thread may stay suspended in the barrier unit for up
+// to `suspend_ns` (it resumes as soon as the phase completes), so waiting
+// warps do not spin on the issue slots that the working warps need.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; false on timeout or
 // when another role of this CTA has already given up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c,
@@ -117,7 +132,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
     if (*c.abort_flag) return false;
     if (globaltimer_ns() - t0 > c.budget_ns) {
       raise_timeout(c, site);
@@ -406,7 +421,8 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 // is exact, a == hi + lo: hi keeps the top 4 significant bits and the rest,
 // at most 4 more bits, is a multiple of the e4m3 grid at its own magnitude.
 // The f16 subtraction is exact as well (hi is within a factor of two of a,
-// or both lie on the f16 subnormal grid).  Values below 2^-10 give hi = lo = 0.
+// or both lie on the f16 subnormal grid).  Below 1/4 the error is at most
+// 2^-10, and values below 2^-10 give hi = lo = 0.
 __device__ __forceinline__ void split_e4m3x2(uint64_t a, uint16_t& hi, uint16_t& lo) {
   uint32_t a16, b16, r16;
   uint16_t h, l;
