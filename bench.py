@@ -501,17 +501,22 @@ def main():
     kernel_avg_ms = kernel_ms / max(kernel_n, 1)
     per_launch_bytes = bytes_per_step / len(Ms)
     per_launch_flops = flops_per_step / len(Ms)
-    src_hash = kernel_source_hash(["decode.cu" if hbm_bound else "tc.cu", "ptx.cuh"])
-    prof_name = f"{'decode_kernel' if hbm_bound else 'tc_kernel'}_{wl.name}.md"
-    traffic = profile_traffic(prof_name, src_hash)
+    if hbm_bound:
+        kname = "decode_kernel" if wl.wtype == "bf16" else "decode_fp8_kernel"
+        sources = ["decode.cu" if wl.wtype == "bf16" else "decode_fp8.cu", "decode_common.cuh", "ptx.cuh"]
+    else:
+        kname, sources = "tc_kernel", ["tc.cu", "ptx.cuh"]
+    src_hash = kernel_source_hash(sources)
+    traffic = profile_traffic(f"{kname}_{wl.name}.md", src_hash)
     if hbm_bound:
         peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
         achieved = per_launch_bytes / (kernel_avg_ms / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": traffic, "kernel": "decode_kernel (+ decode_fixup_kernel): one fn_norm_proj call",
+                    "traffic": traffic, "kernel": f"{kname} (+ decode_fixup_kernel): one fn_norm_proj call",
                     "peak_source": f"hbm_gbs ({peaks_kind})",
                     "bytes_per_launch": per_launch_bytes, "avg_launch_us": kernel_avg_ms * 1e3,
-                    "stream_us_per_call": job_ms / K / n_calls * 1e3}
+                    "stream_us_per_call": job_ms / K / n_calls * 1e3,
+                    "frac_stream": per_launch_bytes / (job_ms / K / n_calls / 1e3) / 1e9 / peak}
         value, unit = value_bytes / 1e9, "GB/s"
     else:
         # burst peak for a kernel that ran at full clock, sustained when the

@@ -483,6 +483,7 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.prefetch_mode = a.prefetch_mode;
   p.scales = nullptr;
   p.cluster = 1;
+  p.narrow = partition_is_narrow(p.total, p.grid) ? 1 : 0;
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
   cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
@@ -499,6 +500,7 @@ cudaError_t launch_impl(const CallArgs& a) {
   if (S >= 2 && a.cluster_mode != 0 && (a.cluster_mode >= 2 || 10LL * p.tiles * S >= 9LL * p.grid)) {
     p.cluster = S;
     p.grid = p.tiles * S;
+    p.narrow = partition_is_narrow(p.total, p.grid) ? 1 : 0;
     return launch_pdl_cluster(decode_kernel<MPAD, HALVES>, static_cast<unsigned>(p.grid), S, NUM_THREADS, SMEM,
                               a.stream, tx, tw, p);
   }

@@ -43,6 +43,7 @@ struct Params {
   int prefetch_mode;         // 0 none, 1 TMA prefetch, 2 per-thread prefetch from idle warps
   const float* scales;       // fp8: block scales [d/128][ncols/128]
   int cluster;               // > 1: split-K inside clusters of this many CTAs, one tile each
+  int narrow;                // (total + 1) * grid fits 32 bits: partition arithmetic in 32 bits
 };
 
 // One partial-result slot: float4 groups [half][row / 4][column] for the
@@ -52,12 +53,21 @@ __host__ __device__ constexpr int slot_floats() {
   return ((HALVES * MPAD * 128 + MPAD) + 31) / 32 * 32;
 }
 
+// First iteration of CTA c.  The 32-bit forms give the same values; they only
+// avoid 64-bit division where the products fit.
 __host__ __device__ __forceinline__ long long it_begin(int c, const Params& p) {
+  if (p.narrow) return static_cast<unsigned>(c) * static_cast<unsigned>(p.total) / static_cast<unsigned>(p.grid);
   return static_cast<long long>(c) * p.total / p.grid;
 }
 // CTA whose iteration range holds iteration `it`
 __device__ __forceinline__ int owner_of(long long it, const Params& p) {
+  if (p.narrow)
+    return static_cast<int>((static_cast<unsigned>(it + 1) * static_cast<unsigned>(p.grid) - 1u) /
+                            static_cast<unsigned>(p.total));
   return static_cast<int>(((it + 1) * p.grid - 1) / p.total);
+}
+inline bool partition_is_narrow(long long total, int grid) {
+  return (total + 1) * static_cast<long long>(grid) < (1ll << 32);
 }
 
 // Wait for a teardown barrier without reporting: the kernel is leaving anyway.

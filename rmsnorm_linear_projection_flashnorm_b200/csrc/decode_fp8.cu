@@ -524,6 +524,7 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.prefetch_mode = a.prefetch_mode;
   p.scales = a.scales;
   p.cluster = 1;
+  p.narrow = dec::partition_is_narrow(p.total, p.grid) ? 1 : 0;
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
   cudaError_t e = ensure_smem_limit<decode_fp8_kernel<MPAD, HALVES>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
