@@ -251,19 +251,38 @@ class Setup:
             raise RuntimeError(f"norm_proj failed: {self.fnb.status_string(st)}")
 
     def chain(self, M, stream=None):
-        """Unfused chain: standalone RMSNorm kernel -> cuBLAS GEMM -> (silu * up)."""
-        if self.W_unf is None:
-            W0, W1 = self._W_src
-            Wcat = torch.cat([W0, W1], dim=1) if self.wl.swiglu else W0
-            self.W_unf = [Wcat] + [Wcat.clone() for _ in range(self.copies - 1)]
+        """Unfused chain: standalone RMSNorm kernel -> cuBLAS GEMM -> (silu * up).
+        bf16 weights: the norm applies g and the GEMM uses the original W.  fp8
+        weights: a dequantisation kernel first turns the stored e4m3 W' (g
+        already folded in) into bf16, the norm runs without a gain, and the
+        GEMM's interleaved gate/up columns are separated for silu * up."""
         wl, c = self.wl, self.i % self.copies
         self.i += 1
+        fp8 = self.wtype != self.fnb.FN_W_BF16
+        if fp8:
+            if self.W_unf is None:
+                self.W_unf = torch.empty_like(self.Wp[0], dtype=torch.bfloat16)
+                self.g_one = torch.ones_like(self.g)
+            ncols = self.Wp[c].shape[1]
+            st = self.fnb.fn_dequant_fp8(self.Wp[c], self.scales[c], wl.d, ncols, self.W_unf, stream)
+            if st != 0:
+                raise RuntimeError(self.fnb.status_string(st))
+            W, g = self.W_unf, self.g_one
+        else:
+            if self.W_unf is None:
+                W0, W1 = self._W_src
+                Wcat = torch.cat([W0, W1], dim=1) if self.wl.swiglu else W0
+                self.W_unf = [Wcat] + [Wcat.clone() for _ in range(self.copies - 1)]
+            W, g = self.W_unf[c], self.g
         h = torch.empty((M, wl.d), dtype=torch.bfloat16, device=self.dev)
-        st = self.fnb.fn_rmsnorm(self.x[M], M, wl.d, self.g, WL.EPS, h, stream)
+        st = self.fnb.fn_rmsnorm(self.x[M], M, wl.d, g, WL.EPS, h, stream)
         if st != 0:
             raise RuntimeError(self.fnb.status_string(st))
-        z = torch.matmul(h, self.W_unf[c])
+        z = torch.matmul(h, W)
         if wl.swiglu:
+            if fp8:   # stored layout: 128-column gate and up blocks alternate
+                z4 = z.view(M, wl.N // 128, 2, 128)
+                return (torch.nn.functional.silu(z4[:, :, 0]) * z4[:, :, 1]).reshape(M, wl.N)
             return torch.nn.functional.silu(z[:, :wl.N]) * z[:, wl.N:]
         return z
 
@@ -581,7 +600,9 @@ def main():
         torch.cuda.synchronize()
         chain_ms = c0.elapsed_time(c1) / c_steps
         chain = {"ms_per_step": chain_ms, "fused_speedup": chain_ms / (elapsed_ms / K),
-                 "what": "fn_rmsnorm kernel -> torch.matmul (cuBLAS) with unfolded W"
+                 "what": ("fn_dequant_fp8 kernel (e4m3 W' -> bf16) -> fn_rmsnorm kernel (no gain) -> "
+                          "torch.matmul (cuBLAS)" if wl.wtype != "bf16" else
+                          "fn_rmsnorm kernel -> torch.matmul (cuBLAS) with unfolded W")
                          + (" -> silu(gate)*up" if wl.swiglu else "")}
 
     _stage("chain done")
