@@ -239,3 +239,31 @@ def test_decode_cluster_and_stream_k_agree_with_oracle(cluster, M, d, N, swiglu)
         assert rel_err(y, ref) <= BF16_TOL
     finally:
         fnb.fn_set_debug(fnb.FN_DEBUG_CLUSTER, 1)
+
+
+@pytest.mark.parametrize("M", [3, 200])
+def test_non_finite_rows_give_nan_rows(M):
+    """An inf or NaN in a row makes that row's outputs NaN (its sum of squares
+    is not finite), as in the oracle; the other rows are unaffected."""
+    d, N = 256, 256
+    x = WL.activations(M, d, 96).clone()
+    x[1, 7] = float("inf")
+    x[2, 200] = float("nan")
+    inp = WL.case(M, d, N, False, seed=96)
+    Wp, _ = T.fold(gpu(inp["W"]), gpu(inp["g"]))
+    y = run(gpu(x), Wp, N, 1e-6)
+    ref = O.norm_proj(x, np.ones(d), fold_ref_bf16(inp["W"], inp["g"]), 1e-6)
+    assert torch.all(torch.isnan(y[1:3].float()))
+    assert rel_err(y, ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("M,swiglu", [(1, False), (48, True), (130, False)])
+def test_long_k(M, swiglu):
+    """d = 16384: 256 k blocks per column tile, so stream-K ranges span many
+    blocks and the tile kernel runs a long main loop."""
+    d, N = 16384, 256
+    if swiglu:
+        y, ref, _ = _swiglu_case(M, d, N, seed=94)
+    else:
+        y, ref, _ = _plain_case(M, d, N, seed=94)
+    assert rel_err(y, ref) <= BF16_TOL
