@@ -154,7 +154,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   fn_status st = check_device(sms);
   if (st != FN_OK) return st;
   const bool dequant_once = wt == FN_W_FP8_E4M3_B128 && !use_decode && M >= kFp8DequantOnceM;
-  const size_t need = use_decode     ? decode_workspace_bytes(M, d, ncols, swiglu, sms)
+  const size_t need = use_decode     ? decode_workspace_bytes(M, d, ncols, swiglu, sms, wt == FN_W_FP8_E4M3_B128)
                       : dequant_once ? kWsHeaderBytes + wbytes * 2
                                      : kWsHeaderBytes;
   if (ws_bytes < need) return FN_ERR_WORKSPACE;
@@ -236,7 +236,7 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
       return kWsHeaderBytes + static_cast<size_t>(d) * static_cast<size_t>(ncols) * 2;
     return kWsHeaderBytes;
   }
-  return decode_workspace_bytes(M, d, ncols, swiglu != 0, current_sms_or_default());
+  return decode_workspace_bytes(M, d, ncols, swiglu != 0, current_sms_or_default(), wt == FN_W_FP8_E4M3_B128);
 }
 
 fn_status fn_norm_proj(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,

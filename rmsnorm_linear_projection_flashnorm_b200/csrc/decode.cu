@@ -484,6 +484,9 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.scales = nullptr;
   p.cluster = 1;
   p.narrow = partition_is_narrow(p.total, p.grid) ? 1 : 0;
+  p.x = static_cast<const __nv_bfloat16*>(a.x);
+  p.xhilo = nullptr;
+  p.xfac = nullptr;
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
   cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
@@ -514,16 +517,17 @@ cudaError_t launch_impl(const CallArgs& a) {
 
 int decode_mpad(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
-size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms) {
+size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms, bool fp8) {
   const int mp = decode_mpad(M);
+  const size_t extra = fp8 ? decode_fp8_presplit_bytes(M, d) : 0;
   if (swiglu) {
-    if (mp == 16) return dec::workspace_bytes<16, 2>(d, ncols, num_sms);
-    if (mp == 32) return dec::workspace_bytes<32, 2>(d, ncols, num_sms);
-    return dec::workspace_bytes<64, 2>(d, ncols, num_sms);
+    if (mp == 16) return dec::workspace_bytes<16, 2>(d, ncols, num_sms) + extra;
+    if (mp == 32) return dec::workspace_bytes<32, 2>(d, ncols, num_sms) + extra;
+    return dec::workspace_bytes<64, 2>(d, ncols, num_sms) + extra;
   }
-  if (mp == 16) return dec::workspace_bytes<16, 1>(d, ncols, num_sms);
-  if (mp == 32) return dec::workspace_bytes<32, 1>(d, ncols, num_sms);
-  return dec::workspace_bytes<64, 1>(d, ncols, num_sms);
+  if (mp == 16) return dec::workspace_bytes<16, 1>(d, ncols, num_sms) + extra;
+  if (mp == 32) return dec::workspace_bytes<32, 1>(d, ncols, num_sms) + extra;
+  return dec::workspace_bytes<64, 1>(d, ncols, num_sms) + extra;
 }
 
 cudaError_t launch_decode(const CallArgs& a) {

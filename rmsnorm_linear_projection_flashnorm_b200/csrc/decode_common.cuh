@@ -44,6 +44,9 @@ struct Params {
   const float* scales;       // fp8: block scales [d/128][ncols/128]
   int cluster;               // > 1: split-K inside clusters of this many CTAs, one tile each
   int narrow;                // (total + 1) * grid fits 32 bits: partition arithmetic in 32 bits
+  const __nv_bfloat16* x;    // the activations (read directly by the x-splitting kernel)
+  uint8_t* xhilo;            // fp8, split once per call: e4m3 x_hi / x_lo rows [kblocks][2 MPAD][128]
+  float* xfac;               // fp8, split once per call: 2^-e per [kblock][row]
 };
 
 // One partial-result slot: float4 groups [half][row / 4][column] for the

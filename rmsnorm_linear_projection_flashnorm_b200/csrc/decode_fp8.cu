@@ -32,6 +32,14 @@
 // The work split is the stream-K partition of decode.cu, and tiles whose k
 // range spans CTAs are finished by the shared fix-up kernel.
 //
+// With 17 to 64 activation rows every CTA would split the same x blocks again
+// for each column tile it visits, and the conversion, a short dependent chain
+// per element, becomes the bottleneck.  There a small kernel splits x once per
+// call into the workspace (the same codes and scales, and each row's sum of
+// squares per k block), and the main kernel stages those operand rows with TMA
+// beside the weight; its converter warps then only add up each row's sums of
+// squares over the k blocks of a segment, alongside the MMAs.
+//
 // Layout:
 //   warp 0        TMA producer
 //   warp 1        TMEM owner and MMA issuer
@@ -56,7 +64,13 @@ constexpr int FIRST_SCALER = 64 + CONV_THREADS;
 constexpr int SMEM_BUDGET = 200 * 1024;  // pipeline stages; barriers and staging come on top
 constexpr int XR = 4;                    // ring of per-row activation scales (converters -> scalers)
 
-template <int MPAD, int HALVES>
+// Workspace for splitting x once per call: x_hi / x_lo slabs, then 2^-e and
+// the sum of squares per (k block, row).
+inline size_t presplit_bytes(int mpad, int64_t d) {
+  return (static_cast<size_t>(2 * mpad) * d + static_cast<size_t>(2 * mpad) * (d / BKQ) * 4 + 255) / 256 * 256;
+}
+
+template <int MPAD, int HALVES, bool PRE = false>
 struct Cfg {
   static constexpr int SCALE_WARPS = HALVES * MPAD >= 64 ? 8 : 4;
   static constexpr int SCALE_THREADS = 32 * SCALE_WARPS;
@@ -64,7 +78,7 @@ struct Cfg {
   static constexpr int RPS = MPAD / (SCALE_WARPS / 4);    // activation rows per scaler thread
   static constexpr int W_BYTES = HALVES * WQ_BOX;          // e4m3 weight: 16 or 32 KB
   static constexpr int XB_BOX = MPAD * 128;                // bf16 x box: MPAD rows x 64 columns
-  static constexpr int XB_BYTES = 2 * XB_BOX;
+  static constexpr int XB_BYTES = PRE ? 0 : 2 * XB_BOX;    // x split once per call: no bf16 x tile
   static constexpr int XQ_BYTES = MPAD * BKQ;              // e4m3 x_hi (or x_lo): MPAD rows x 128 B
   static constexpr int STAGE_BYTES = W_BYTES + XB_BYTES + 2 * XQ_BYTES;   // multiple of 1024
   static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
@@ -168,11 +182,58 @@ __device__ __forceinline__ float convert_row_block(const uint8_t* xb, uint8_t* x
   return ss;
 }
 
-template <int MPAD, int HALVES>
-__global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
+// Split x once per call (the 17..64-row case): one warp per (128-deep k block,
+// padded row); lane l takes k values 4l .. 4l+3.  Codes and scale factors are
+// those convert_row_block computes, written as the operand rows the decode
+// kernel stages: x_hi at row r, x_lo at row MPAD + r of the k block's
+// [2 MPAD][128-byte] slab; padding rows are zero.
+template <int MPAD>
+__global__ void __launch_bounds__(256) xsplit_kernel(const Params p) {
+  grid_launch_dependents();     // the decode kernel may set up meanwhile
+  grid_dependency_wait();       // x may have been written by the preceding kernel
+  const int wg = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int kb = wg / MPAD, row = wg % MPAD;
+  if (kb >= p.kblocks) return;
+  const bool live = row < p.M;
+  uint2 v = make_uint2(0u, 0u);
+  if (live) v = *reinterpret_cast<const uint2*>(p.x + static_cast<int64_t>(row) * p.d + kb * BKQ + lane * 4);
+  uint32_t amax = max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu), max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const int E = static_cast<int>(amax >> 7);
+  int e = amax == 0 ? 0 : 134 - E;
+  e = e > 126 ? 126 : (e < -126 ? -126 : e);
+  const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+  const uint64_t sc2 = f2_pack(sc, sc);
+  uint16_t h0 = 0, l0 = 0, h1 = 0, l1 = 0;
+  uint64_t ss2 = 0;
+  if (live) {
+    const uint64_t a = f2_pack_u(v.x << 16, v.x & 0xFFFF0000u), b = f2_pack_u(v.y << 16, v.y & 0xFFFF0000u);
+    ss2 = f2_fma(b, b, f2_fma(a, a, ss2));
+    split_e4m3x2(f2_mul(a, sc2), h0, l0);
+    split_e4m3x2(f2_mul(b, sc2), h1, l1);
+  }
+  float ss = f2_lo(ss2) + f2_hi(ss2);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  uint8_t* slab = p.xhilo + static_cast<int64_t>(kb) * 2 * MPAD * 128;
+  *reinterpret_cast<uint32_t*>(slab + row * 128 + lane * 4) = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+  *reinterpret_cast<uint32_t*>(slab + (MPAD + row) * 128 + lane * 4) =
+      static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+  if (lane == 0) {
+    p.xfac[kb * MPAD + row] = !live ? 0.f
+                              : (E == 255 ? __int_as_float(0x7fc00000)
+                                          : __uint_as_float(static_cast<uint32_t>(127 - e) << 23));
+    p.xfac[(p.kblocks + kb) * MPAD + row] = ss;   // the block's sum of squares
+  }
+}
+
+template <int MPAD, int HALVES, bool PRESPLIT>
+__global__ void __launch_bounds__(Cfg<MPAD, HALVES, PRESPLIT>::THREADS, 1)
     decode_fp8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                      const Params p) {
-  using C = Cfg<MPAD, HALVES>;
+                      const __grid_constant__ CUtensorMap tmap_q, const Params p) {
+  using C = Cfg<MPAD, HALVES, PRESPLIT>;
   constexpr int STAGES = C::STAGES;
   using B = Bars<MPAD, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -212,6 +273,7 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_x);
+    if (PRESPLIT) tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_w);
   }
   if (warp == 1) {
@@ -254,9 +316,13 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
         const int tile = static_cast<int>(it / p.kblocks);
         const int kb = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
         if (!mbar_wait(&bars.empty[s], ph ^ 1, ctl, dec::kSiteProdEmpty)) break;
-        mbar_arrive_expect_tx(&bars.full[s], C::XB_BYTES + C::W_BYTES);
-        tma_load_2d(stage_xb(s), &tmap_x, &bars.full[s], kb * BKQ, 0);
-        tma_load_2d(stage_xb(s) + C::XB_BOX, &tmap_x, &bars.full[s], kb * BKQ + 64, 0);
+        mbar_arrive_expect_tx(&bars.full[s], C::XB_BYTES + C::W_BYTES + (PRESPLIT ? 2 * C::XQ_BYTES : 0));
+        if (!PRESPLIT) {
+          tma_load_2d(stage_xb(s), &tmap_x, &bars.full[s], kb * BKQ, 0);
+          tma_load_2d(stage_xb(s) + C::XB_BOX, &tmap_x, &bars.full[s], kb * BKQ + 64, 0);
+        }
+        // pre-split operand rows: x_hi and x_lo of this k block, one box
+        if (PRESPLIT) tma_load_2d(stage_xh(s), &tmap_q, &bars.full[s], 0, kb * 2 * MPAD);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
           tma_load_2d_hint(stage_w(s) + h * WQ_BOX, &tmap_w, &bars.full[s], (tile * HALVES + h) * 128, kb * BKQ,
@@ -311,6 +377,22 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
     const int ct = threadIdx.x - 64;
     const int row = ct / C::TPR, sub = ct % C::TPR;
     const bool live = row < p.M;
+    // x split once per call: this row's scale factor and sum of squares for
+    // iteration `it`, loaded three iterations ahead
+    auto load_pre = [&](long long it, float& f, float& ss) {
+      f = ss = 0.f;
+      if (PRESPLIT && it < it1) {
+        const int kb = static_cast<int>(it % p.kblocks);
+        f = p.xfac[kb * MPAD + row];
+        ss = p.xfac[(p.kblocks + kb) * MPAD + row];
+      }
+    };
+    float pre_f[3] = {0.f, 0.f, 0.f}, pre_ss[3] = {0.f, 0.f, 0.f};
+    if (PRESPLIT && sub == 0) {
+      load_pre(it0, pre_f[0], pre_ss[0]);
+      load_pre(it0 + 1, pre_f[1], pre_ss[1]);
+      load_pre(it0 + 2, pre_f[2], pre_ss[2]);
+    }
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -327,11 +409,21 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
         ready = ready && mbar_wait(&bars.xse[xr], static_cast<uint32_t>((gi / XR) & 1) ^ 1u, ctl,
                                    dec::kSiteConvScaleEmpty);
         if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
-        float factor;
-        rss += convert_row_block<MPAD, C::TPR, C::EPT>(stage_xb(s), stage_xh(s), stage_xl(s), row, sub, live,
-                                                       &factor);
-        if (sub == 0) bars.xs[xr][row] = factor;
-        fence_proxy_async_smem();   // generic-proxy operand writes -> visible to tcgen05.mma
+        if (PRESPLIT) {
+          if (sub == 0) {
+            rss += pre_ss[0];
+            bars.xs[xr][row] = pre_f[0];
+            pre_f[0] = pre_f[1]; pre_ss[0] = pre_ss[1];
+            pre_f[1] = pre_f[2]; pre_ss[1] = pre_ss[2];
+            load_pre(it0 + gi + 3, pre_f[2], pre_ss[2]);
+          }
+        } else {
+          float factor;
+          rss += convert_row_block<MPAD, C::TPR, C::EPT>(stage_xb(s), stage_xh(s), stage_xl(s), row, sub, live,
+                                                         &factor);
+          if (sub == 0) bars.xs[xr][row] = factor;
+          fence_proxy_async_smem();   // generic-proxy operand writes -> visible to tcgen05.mma
+        }
         mbar_arrive(&bars.conv[s]);
         mbar_arrive(&bars.xsf[xr]);
         if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -482,9 +574,9 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES>::THREADS, 1)
   }
 }
 
-template <int MPAD, int HALVES>
+template <int MPAD, int HALVES, bool PRE = false>
 constexpr size_t smem_bytes() {
-  using C = Cfg<MPAD, HALVES>;
+  using C = Cfg<MPAD, HALVES, PRE>;
   return 1024 + C::STAGES * C::STAGE_BYTES + sizeof(Bars<MPAD, C::STAGES>);
 }
 
@@ -494,11 +586,17 @@ static_assert(smem_bytes<64, 2>() <= 227 * 1024 && smem_bytes<64, 1>() <= 227 * 
 static_assert(Cfg<64, 2>::STAGES >= 2, "pipeline needs two stages");
 static_assert(Cfg<16, 1>::TMEM_COLS == 64 && Cfg<64, 2>::TMEM_COLS == 512, "TMEM allocation: a power of two <= 512");
 
+// Whether calls with this padded row count split x once per call.
+template <int MPAD>
+constexpr bool presplit() { return MPAD >= 32; }
+
 template <int MPAD, int HALVES>
 cudaError_t launch_impl(const CallArgs& a) {
-  using C = Cfg<MPAD, HALVES>;
-  if (a.ws_bytes < dec::workspace_bytes<MPAD, HALVES>(a.d, a.ncols, a.num_sms)) return cudaErrorInvalidValue;
-  CUtensorMap tx, tw;
+  constexpr bool PRE = presplit<MPAD>();
+  using C = Cfg<MPAD, HALVES, PRE>;
+  const size_t part_bytes = dec::workspace_bytes<MPAD, HALVES>(a.d, a.ncols, a.num_sms);
+  if (a.ws_bytes < part_bytes + (PRE ? presplit_bytes(MPAD, a.d) : 0)) return cudaErrorInvalidValue;
+  CUtensorMap tx, tw, tq;
   if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, MPAD, 64)) return cudaErrorInvalidValue;
   // e4m3 codes as bytes: 128 columns (one 128-byte swizzle row) x 128 k rows per box
   if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.d, a.ncols, BKQ, 128)) return cudaErrorInvalidValue;
@@ -525,16 +623,40 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.scales = a.scales;
   p.cluster = 1;
   p.narrow = dec::partition_is_narrow(p.total, p.grid) ? 1 : 0;
-  constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
-  cudaError_t e = ensure_smem_limit<decode_fp8_kernel<MPAD, HALVES>>(static_cast<int>(SMEM));
+  p.x = static_cast<const __nv_bfloat16*>(a.x);
+  p.xhilo = nullptr;
+  p.xfac = nullptr;
+  tq = tw;   // unused unless x is split once per call
+  if (PRE) {
+    // after the partial slots: x_hi / x_lo slabs, then the scale factors
+    p.xhilo = ws + part_bytes;
+    p.xfac = reinterpret_cast<float*>(ws + part_bytes + static_cast<size_t>(2 * MPAD) * a.d);
+    if (!make_tmap_2d(&tq, p.xhilo, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(p.kblocks) * 2 * MPAD,
+                      BKQ, 2 * MPAD, BKQ))
+      return cudaErrorInvalidValue;
+  }
+  constexpr size_t SMEM = smem_bytes<MPAD, HALVES, PRE>();
+  cudaError_t e = ensure_smem_limit<decode_fp8_kernel<MPAD, HALVES, PRE>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
-  e = launch_pdl(decode_fp8_kernel<MPAD, HALVES>, p.grid, C::THREADS, SMEM, a.stream, tx, tw, p);
+  if (PRE) {
+    const int warps = p.kblocks * MPAD;
+    e = launch_pdl(xsplit_kernel<MPAD>, static_cast<unsigned>((warps + 7) / 8), 256, 0, a.stream, p);
+    if (e != cudaSuccess) return e;
+  }
+  e = launch_pdl(decode_fp8_kernel<MPAD, HALVES, PRE>, p.grid, C::THREADS, SMEM, a.stream, tx, tw, tq, p);
   if (e != cudaSuccess) return e;
   if (!dec::any_split_tile(p.grid, p.total, p.kblocks)) return cudaSuccess;
   return dec::launch_fixup<MPAD, HALVES>(p, a.stream);
 }
 
 }  // namespace dec8
+
+size_t decode_fp8_presplit_bytes(int64_t M, int64_t d) {
+  const int mp = decode_mpad(M);
+  if (mp == 32) return dec8::presplit<32>() ? dec8::presplit_bytes(32, d) : 0;
+  if (mp == 64) return dec8::presplit<64>() ? dec8::presplit_bytes(64, d) : 0;
+  return dec8::presplit<16>() ? dec8::presplit_bytes(16, d) : 0;
+}
 
 cudaError_t launch_decode_fp8(const CallArgs& a, int mpad) {
   if (mpad == 16) return a.swiglu ? dec8::launch_impl<16, 2>(a) : dec8::launch_impl<16, 1>(a);

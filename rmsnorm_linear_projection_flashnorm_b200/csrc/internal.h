@@ -53,7 +53,9 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, in
 // Decode (M <= 64) path: stream-K split over all SMs with a deterministic
 // in-kernel fix-up through workspace partials.
 int decode_mpad(int64_t M);
-size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms);
+size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms, bool fp8);
+// fp8 weights, 17..64 rows: workspace for x split once per call (decode_fp8.cu)
+size_t decode_fp8_presplit_bytes(int64_t M, int64_t d);
 cudaError_t launch_decode(const CallArgs& a);
 // fp8 weights on the decode path (decode_fp8.cu); mpad is decode_mpad(M).
 cudaError_t launch_decode_fp8(const CallArgs& a, int mpad);
