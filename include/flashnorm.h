@@ -87,10 +87,12 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
  * fn_workspace_size — bytes of workspace a call with these sizes needs.
  * The workspace holds a 256-byte header (the device status word) and, for
  * M <= 64, the per-CTA partial sums of the split-K decode path; with fp8
- * weights and M >= 1024 it also holds one bf16 copy of the weight, converted
- * once per call with the same rounding the on-chip conversion uses
- * (bf16(fp32(q) * s)), because converting each weight tile once per 128-row
- * tile would repeat that work M/128 times.  Zero it once
+ * weights and 17 <= M <= 64 also the activations split once per call into
+ * the two e4m3 operand parts (2 x 64 x d bytes at most) with their scale
+ * factors and per-block sums of squares; with fp8 weights and M >= 1024 one
+ * bf16 copy of the weight, converted once per call with the same rounding the
+ * on-chip conversion uses (bf16(fp32(q) * s)), because converting each weight
+ * tile once per 128-row tile would repeat that work M/128 times.  Zero it once
  * before its first use (the status word must start at zero); the calls keep
  * the status word at zero unless a device-side wait times out.  Depends on
  * the SM count of the current device (148 is assumed when no device is
