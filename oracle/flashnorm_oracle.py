@@ -33,6 +33,21 @@ oracle spells out their rounding steps from the formats' definitions:
     SwiGLU storage: 128-column tiles of the gate and up halves alternate,
             W'_cat[:, 256j : 256j+128]       = W'_gate[:, 128j : 128j+128]
             W'_cat[:, 256j+128 : 256j+256]   = W'_up  [:, 128j : 128j+128]
+
+The quantising SwiGLU epilogue writes its output in NVFP4 for the next
+projection (FlashInfer PR #4040 analysis: silu_and_mul fused with the NVFP4
+quantisation, a block of SF_VEC_SIZE = 16 elements per scale factor and a
+caller-supplied global scale).  That page names the parts but prints no
+formula; the reading used here, per row m and block b of 16 consecutive
+output columns, with gs the fp32 global scale:
+
+    amax_b = max |y[m, 16b : 16b+16]|
+    sf_b   = RN_e4m3_satfinite( gs * amax_b / 6 )     6: the largest e2m1 value
+    q      = RN_e2m1_satfinite( y * gs / sf_b )        q = 0 where sf_b = 0
+    a block holding a non-finite value: sf_b = the e4m3 NaN code, q = 0
+    dequantised: e2m1(q) * e4m3(sf_b) / gs
+    storage: two codes per byte, the even column in the low nibble;
+             scale codes row-major [M, N/16]
 """
 from __future__ import annotations
 
@@ -47,6 +62,8 @@ __all__ = [
     "rms_inv", "rmsnorm", "norm_proj", "silu", "norm_proj_swiglu",
     "fold_bf16", "interleave128", "deinterleave128", "fold_fp8", "dequant_fp8", "dequant_fp8_bf16_bits",
     "FP8_BLOCK", "E4M3_MAX",
+    "E2M1", "E2M1_MAX", "NVFP4_BLOCK", "e2m1_round", "e2m1_encode", "e2m1_decode",
+    "nvfp4_quantize", "nvfp4_pack", "nvfp4_unpack", "nvfp4_dequantize",
 ]
 
 FP8_BLOCK = 128
@@ -76,6 +93,11 @@ BF16 = _Format("bf16", 7, 8, 127, (2.0 - 2.0 ** -7) * 2.0 ** 127, "inf")
 # S.1111.111 is NaN, so the largest finite value is 1.75 * 2^8 = 448.
 # Conversions here saturate to +-448 (the "satfinite" rounding).
 E4M3 = _Format("e4m3", 3, 4, 7, 448.0, "sat")
+# e2m1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; no inf and no NaN.  The
+# exponent field 0 holds the subnormal 0.5; the largest value is 1.5 * 2^2 = 6.
+E2M1 = _Format("e2m1", 1, 2, 1, 6.0, "sat")
+E2M1_MAX = 6.0
+NVFP4_BLOCK = 16
 
 
 def round_to_format(v, fmt: _Format) -> np.ndarray:
@@ -287,3 +309,79 @@ def dequant_fp8_bf16_bits(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     s_full = np.repeat(np.repeat(np.asarray(s, dtype=np.float32), FP8_BLOCK, axis=0), FP8_BLOCK, axis=1)
     prod = e4m3_decode(q).astype(np.float32) * s_full        # fp32 IEEE product
     return bf16_bits(prod.astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 output encoding (quantising SwiGLU epilogue)
+# ---------------------------------------------------------------------------
+def e2m1_round(v) -> np.ndarray:
+    return round_to_format(v, E2M1)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """4-bit codes (uint8 0..15) of RN_e2m1_satfinite(v): sign | exponent
+    field (2 bits) | mantissa bit.  NaN has no code here; callers keep it out."""
+    r = e2m1_round(v)
+    sign = np.signbit(r).astype(np.uint8) << 3
+    a = np.abs(np.where(np.isnan(r), 0.0, r))
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    e = ex.astype(np.int64) - 1                     # floor(log2 a)
+    normal = a >= 1.0                               # smallest normal: 2^(1 - bias)
+    exp_field = np.where(normal, e + E2M1.bias, 0)
+    # normal: a = (1 + m/2) * 2^e; subnormal (field 0): a = m * 0.5
+    mant_field = np.where(normal, np.rint((np.ldexp(a, -e) - 1.0) * 2.0), np.rint(a * 2.0)).astype(np.int64)
+    code = (exp_field << 1) | mant_field
+    return (np.where(a == 0, 0, code).astype(np.uint8) | sign).astype(np.uint8)
+
+
+def e2m1_decode(code) -> np.ndarray:
+    """float64 value of each 4-bit e2m1 code."""
+    c = np.asarray(code, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x8, -1.0, 1.0)
+    ef = (c >> 1) & 0x3
+    mf = c & 0x1
+    val = np.where(ef == 0, mf * 0.5, np.ldexp(1.0 + mf / 2.0, ef - E2M1.bias))
+    return s * val
+
+
+def nvfp4_quantize(y, global_scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """NVFP4 encoding of y [M, N] (N a multiple of 16) with the fp32 global
+    scale gs, following the reading in the module docstring.  Returns the
+    4-bit codes [M, N] (one per uint8) and the e4m3 scale codes [M, N/16].
+    The arithmetic is float64; gs is taken as its fp32 value."""
+    y = np.asarray(y, dtype=np.float64)
+    M, N = y.shape
+    assert N % NVFP4_BLOCK == 0
+    gs = float(np.float32(global_scale))
+    blocks = y.reshape(M, N // NVFP4_BLOCK, NVFP4_BLOCK)
+    finite = np.all(np.isfinite(blocks), axis=2)                     # [M, N/16]
+    amax = np.max(np.abs(np.where(np.isfinite(blocks), blocks, 0.0)), axis=2)
+    sf = e4m3_encode(gs * amax / E2M1_MAX)
+    sf = np.where(finite, sf, np.uint8(0x7F)).astype(np.uint8)
+    sf_val = np.where(finite, e4m3_decode(np.where(finite, sf, 0)), 0.0)
+    enc = np.where(sf_val > 0, gs / np.where(sf_val > 0, sf_val, 1.0), 0.0)
+    scaled = np.where(finite[:, :, None], np.where(np.isfinite(blocks), blocks, 0.0) * enc[:, :, None], 0.0)
+    codes = e2m1_encode(scaled).reshape(M, N)
+    return codes, sf
+
+
+def nvfp4_pack(codes) -> np.ndarray:
+    """[M, N] 4-bit codes -> [M, N/2] bytes, the even column in the low nibble."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[:, 0::2] & 0xF) | ((c[:, 1::2] & 0xF) << 4)
+
+
+def nvfp4_unpack(packed) -> np.ndarray:
+    """[M, N/2] bytes -> [M, N] 4-bit codes."""
+    b = np.asarray(packed, dtype=np.uint8)
+    out = np.empty((b.shape[0], b.shape[1] * 2), dtype=np.uint8)
+    out[:, 0::2] = b & 0xF
+    out[:, 1::2] = b >> 4
+    return out
+
+
+def nvfp4_dequantize(codes, sf, global_scale: float) -> np.ndarray:
+    """float64 e2m1(q) * e4m3(sf) / gs for codes [M, N] and scale codes [M, N/16]."""
+    gs = float(np.float32(global_scale))
+    scale = np.repeat(e4m3_decode(sf), NVFP4_BLOCK, axis=1)
+    return e2m1_decode(codes) * scale / gs
