@@ -171,9 +171,12 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # workload setup
 # ---------------------------------------------------------------------------
-def algorithmic(M: int, d: int, N: int, swiglu: bool, wbytes_per_elem: int = 2):
+def algorithmic(M: int, d: int, N: int, swiglu: bool, wbytes_per_elem: int = 2, out: str = "bf16"):
+    """Bytes (x and W' read once, the output written once) and flops of one call.
+    NVFP4 output: half a byte per element plus one scale byte per 16."""
     ncols = 2 * N if swiglu else N
-    by = M * d * 2 + d * ncols * wbytes_per_elem + M * N * 2
+    out_bytes = M * N // 2 + M * N // 16 if out == "nvfp4" else M * N * 2
+    by = M * d * 2 + d * ncols * wbytes_per_elem + out_bytes
     fl = 2.0 * M * d * ncols
     return by, fl
 
@@ -205,7 +208,7 @@ def profile_traffic(profile_name: str, src_hash: str):
 
 
 class Setup:
-    def __init__(self, wl: WL.Workload, Ms, device):
+    def __init__(self, wl: WL.Workload, Ms, device, out: str = "bf16"):
         import rmsnorm_linear_projection_flashnorm_b200 as fnb
         from rmsnorm_linear_projection_flashnorm_b200 import torch_api as T
         self.fnb, self.T = fnb, T
@@ -231,8 +234,18 @@ class Setup:
         x_all = WL.activations(Mmax, d, wl.seed, wl.outliers)
         self.x_host = {M: x_all[:M].contiguous().pin_memory() for M in self.Ms}
         self.x = {M: self.x_host[M].to(device) for M in self.Ms}
-        self.y = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in self.Ms}
-        self.y_host = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in self.Ms}
+        self.out = out
+        if out == "nvfp4":
+            # codes [M, N/2] and scale bytes [M, N/16], copied to one host buffer
+            # per M; a fixed global scale (its value does not change the work)
+            self.y = {M: torch.empty((M, N // 2 + N // 16), dtype=torch.uint8, device=device) for M in self.Ms}
+            self.y_host = {M: torch.empty((M, N // 2 + N // 16), dtype=torch.uint8).pin_memory() for M in self.Ms}
+            self.yq = {M: torch.empty((M, N // 2), dtype=torch.uint8, device=device) for M in self.Ms}
+            self.ysf = {M: torch.empty((M, N // 16), dtype=torch.uint8, device=device) for M in self.Ms}
+            self.gscale = torch.tensor([448.0 * 6.0 / 8.0], dtype=torch.float32, device=device)
+        else:
+            self.y = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in self.Ms}
+            self.y_host = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in self.Ms}
         self.ws = T.Workspace(device)
         for M in self.Ms:
             self.ws.get(M, d, N, self.wtype, sw)
@@ -245,10 +258,24 @@ class Setup:
         self.i += 1
         x = self.x[M] if x is None else x
         y = self.y[M] if y is None else y
-        st = self.fn(x, M, wl.d, self.Wp[c], self.scales[c], self.wtype, wl.N, WL.EPS, y, self.ws.buf,
-                     self.ws.buf.numel(), stream)
+        if self.out == "nvfp4":
+            st = self.fnb.fn_norm_proj_swiglu_nvfp4(x, M, wl.d, self.Wp[c], self.scales[c], self.wtype, wl.N,
+                                                    WL.EPS, self.gscale, self.yq[M], self.ysf[M], self.ws.buf,
+                                                    self.ws.buf.numel(), stream)
+        else:
+            st = self.fn(x, M, wl.d, self.Wp[c], self.scales[c], self.wtype, wl.N, WL.EPS, y, self.ws.buf,
+                         self.ws.buf.numel(), stream)
         if st != 0:
             raise RuntimeError(f"norm_proj failed: {self.fnb.status_string(st)}")
+
+    def fetch(self, M):
+        """Copy the call's output to pinned host memory (asynchronous)."""
+        if self.out == "nvfp4":
+            n = self.yq[M].shape[1]
+            self.y_host[M][:, :n].copy_(self.yq[M], non_blocking=True)
+            self.y_host[M][:, n:].copy_(self.ysf[M], non_blocking=True)
+        else:
+            self.y_host[M].copy_(self.y[M], non_blocking=True)
 
     def chain(self, M, stream=None):
         """Unfused chain: standalone RMSNorm kernel -> cuBLAS GEMM -> (silu * up).
@@ -396,6 +423,8 @@ def main():
     ap.add_argument("--m", type=int, default=0, help="run a single batch size of the workload")
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU oracle baseline")
     ap.add_argument("--skip-chain", action="store_true", help="omit the unfused-chain baseline")
+    ap.add_argument("--out", default="bf16", choices=["bf16", "nvfp4"],
+                    help="output format; nvfp4 (SwiGLU workloads) runs the quantising epilogue")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -416,15 +445,17 @@ def main():
     fnb.lib()
 
     wl = WL.WORKLOADS[args.workload]
+    if args.out == "nvfp4" and not wl.swiglu:
+        raise SystemExit("--out nvfp4 needs a SwiGLU workload")
     Ms = [args.m] if args.m else list(wl.Ms)
     _stage("setup")
-    S = Setup(wl, Ms, dev)
+    S = Setup(wl, Ms, dev, args.out)
     _stage("setup done")
     stream = torch.cuda.current_stream()
     peaks, peaks_kind = load_peaks()
     wbyte = 2 if wl.wtype == "bf16" else 1
-    bytes_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte)[0] for M in Ms)
-    flops_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte)[1] for M in Ms)
+    bytes_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte, args.out)[0] for M in Ms)
+    flops_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte, args.out)[1] for M in Ms)
     hbm_bound = max(Ms) <= 64
 
     # warm-up
@@ -522,11 +553,12 @@ def main():
     per_launch_flops = flops_per_step / len(Ms)
     if hbm_bound:
         kname = "decode_kernel" if wl.wtype == "bf16" else "decode_fp8_kernel"
-        sources = ["decode.cu" if wl.wtype == "bf16" else "decode_fp8.cu", "decode_common.cuh", "ptx.cuh"]
+        sources = ["decode.cu" if wl.wtype == "bf16" else "decode_fp8.cu", "decode_common.cuh", "ptx.cuh",
+                   "nvfp4.cuh"]
     else:
-        kname, sources = "tc_kernel", ["tc.cu", "ptx.cuh"]
+        kname, sources = "tc_kernel", ["tc.cu", "ptx.cuh", "nvfp4.cuh"]
     src_hash = kernel_source_hash(sources)
-    traffic = profile_traffic(f"{kname}_{wl.name}.md", src_hash)
+    traffic = profile_traffic(f"{kname}_{wl.name}{'_nvfp4' if args.out == 'nvfp4' else ''}.md", src_hash)
     if hbm_bound:
         peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
         achieved = per_launch_bytes / (kernel_avg_ms / 1e3) / 1e9
@@ -558,13 +590,13 @@ def main():
     # end to end through the public API: pinned host x -> device -> call -> host y
     e2e_steps = max(1, min(K, 2000))
     h2d = sum(S.x_host[M].numel() * 2 for M in Ms)
-    d2h = sum(S.y_host[M].numel() * 2 for M in Ms)
+    d2h = sum(S.y_host[M].numel() * S.y_host[M].element_size() for M in Ms)
     xs = {M: torch.empty_like(S.x[M]) for M in Ms}
     for _ in range(3):
         for M in Ms:
             xs[M].copy_(S.x_host[M], non_blocking=True)
             S.call(M, x=xs[M])
-            S.y_host[M].copy_(S.y[M], non_blocking=True)
+            S.fetch(M)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -573,7 +605,7 @@ def main():
         for M in Ms:
             xs[M].copy_(S.x_host[M], non_blocking=True)
             S.call(M, x=xs[M])
-            S.y_host[M].copy_(S.y[M], non_blocking=True)
+            S.fetch(M)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_units, e2e_ms = aggregate(float(bytes_per_step if hbm_bound else flops_per_step) * e2e_steps,
@@ -585,7 +617,7 @@ def main():
 
     # unfused chain (same rotation of weight copies): rmsnorm -> cuBLAS -> silu*up
     chain = None
-    if not args.skip_chain:
+    if not args.skip_chain and args.out == "bf16":
         for _ in range(3):
             for M in Ms:
                 S.chain(M)
@@ -616,7 +648,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": job_ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if wl.wtype == "bf16" else "bf16 (e4m3 weights)",
             "data": "synthetic (seeded workloads recipe; random-init weights)",
-            "config": {"workload": wl.name, "M": Ms, "d": wl.d, "N": wl.N, "swiglu": wl.swiglu,
+            "config": {"workload": wl.name, "M": Ms, "d": wl.d, "N": wl.N, "swiglu": wl.swiglu, "output": args.out,
                        "weights": wl.wtype, "parallelism": f"replicas x{world} (rows shard, no collective)",
                        "l2": f"{S.copies} rotating W' copies ({S.copies * S.Wp[0].numel() * S.Wp[0].element_size() / 1e6:.0f} MB > L2)",
                        "step": f"{len(Ms)} fused calls, one per M; CUDA graphs of {G} steps",

@@ -128,6 +128,31 @@ fn_status fn_norm_proj_swiglu(const void* x, int64_t M, int64_t d, const void* W
                               fn_stream_t stream);
 
 /*
+ * fn_norm_proj_swiglu_nvfp4 — the SwiGLU output of fn_norm_proj_swiglu written
+ * in NVFP4 for the projection that follows, from the epilogue registers (no
+ * bf16 intermediate in memory), as the FlashInfer PR #4040 analysis fuses
+ * silu_and_mul with its NVFP4 quantisation (16 elements per scale factor, a
+ * global scale).  For each row m and block b of 16 consecutive output columns,
+ * with v the fp32 SwiGLU value and gs = *global_scale:
+ *   sf[m, b] = RN_e4m3_satfinite(gs * max|v| / 6)         (6: largest e2m1 value)
+ *   q[m, n]  = RN_e2m1_satfinite(v * (gs / sf[m, b]))      (0 where sf is 0)
+ * A block holding a non-finite value gets sf = 0x7F (e4m3 NaN) and zero codes.
+ * The consumer dequantises as e2m1(q) * e4m3(sf) / gs.
+ *   global_scale  device pointer to one fp32 value, > 0 and finite (read on
+ *                 the device, so a CUDA graph may keep it while it changes)
+ *   out_q         [M, N/2] bytes: two e2m1 codes per byte, the even column in
+ *                 the low nibble; 16-byte aligned
+ *   out_sf        [M, N/16] e4m3 scale bytes, row-major (not the swizzled
+ *                 tensor-core layout); 16-byte aligned
+ * Other arguments and the workspace as fn_norm_proj_swiglu.  The outputs must
+ * not overlap each other, the inputs, global_scale or the workspace
+ * (FN_ERR_ALIAS).  M == 0 is a no-op.
+ */
+fn_status fn_norm_proj_swiglu_nvfp4(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                                    fn_wtype wt, int64_t N, float eps, const float* global_scale, void* out_q,
+                                    void* out_sf, void* workspace, size_t ws_bytes, fn_stream_t stream);
+
+/*
  * fn_norm_proj_static — fn_norm_proj for callers that cannot allocate device
  * memory, so cannot pass a workspace: code recording work under a CUDA stream
  * capture (where cudaMalloc is not permitted), plug-ins whose host application

@@ -42,6 +42,8 @@ _SIGNATURES = {
     "fn_workspace_size": (_sz, [_i64, _i64, _i64, _int, _int]),
     "fn_norm_proj": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp, _sz, _vp]),
     "fn_norm_proj_swiglu": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp, _sz, _vp]),
+    "fn_norm_proj_swiglu_nvfp4": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp, _vp, _vp, _sz,
+                                         _vp]),
     "fn_norm_proj_static": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp]),
     "fn_query_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_uint), _vp]),
     "fn_rmsnorm": (_int, [_vp, _i64, _i64, _vp, _f32, _vp, _vp]),
@@ -137,6 +139,12 @@ def fn_norm_proj_swiglu(x, M: int, d: int, Wp, scales, wt: int, N: int, eps: flo
                         ws_bytes: int, stream=None) -> int:
     return lib().fn_norm_proj_swiglu(_ptr(x), M, d, _ptr(Wp), _ptr(scales), wt, N, eps, _ptr(out),
                                      _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def fn_norm_proj_swiglu_nvfp4(x, M: int, d: int, Wp, scales, wt: int, N: int, eps: float, global_scale, out_q,
+                              out_sf, workspace, ws_bytes: int, stream=None) -> int:
+    return lib().fn_norm_proj_swiglu_nvfp4(_ptr(x), M, d, _ptr(Wp), _ptr(scales), wt, N, eps, _ptr(global_scale),
+                                           _ptr(out_q), _ptr(out_sf), _ptr(workspace), ws_bytes, _stream(stream))
 
 
 def fn_norm_proj_static(x, M: int, d: int, Wp, scales, wt: int, N: int, eps: float, y, stream=None) -> int:

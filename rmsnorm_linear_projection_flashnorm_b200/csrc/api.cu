@@ -116,9 +116,12 @@ fn_status check_device(int& sms) {
   return FN_OK;
 }
 
+// Fused call.  Output: bf16 y, or (SwiGLU only) NVFP4 codes yq, scale bytes
+// ysf and the global scale gscale, with y null.
 fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
                            int64_t N, float eps, void* y, void* ws, size_t ws_bytes, fn_stream_t stream,
-                           bool swiglu) {
+                           bool swiglu, void* yq = nullptr, void* ysf = nullptr, const float* gscale = nullptr) {
+  const bool fp4 = yq != nullptr || ysf != nullptr || gscale != nullptr;
   if (M < 0 || d <= 0 || N <= 0) return FN_ERR_INVALID_ARG;
   if (wt != FN_W_BF16 && wt != FN_W_FP8_E4M3_B128) return FN_ERR_INVALID_ARG;
   if (!eps_ok(eps)) return FN_ERR_INVALID_ARG;
@@ -127,19 +130,32 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   const int64_t ncols = swiglu ? 2 * N : N;
   if (M > kMaxDim || d > kMaxDim || ncols > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FN_OK;
-  if (!x || !Wp || !y) return FN_ERR_INVALID_ARG;
+  if (!x || !Wp) return FN_ERR_INVALID_ARG;
+  if (fp4 ? (!yq || !ysf || !gscale || y || !swiglu) : !y) return FN_ERR_INVALID_ARG;
   if (!ws) return FN_ERR_WORKSPACE;
   if (wt == FN_W_FP8_E4M3_B128 && !scales) return FN_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(Wp) || !aligned16(y) || !aligned16(ws)) return FN_ERR_ALIGNMENT;
+  if (!aligned16(x) || !aligned16(Wp) || !aligned16(ws)) return FN_ERR_ALIGNMENT;
+  if (fp4 ? (!aligned16(yq) || !aligned16(ysf) || (reinterpret_cast<uintptr_t>(gscale) & 3u)) : !aligned16(y))
+    return FN_ERR_ALIGNMENT;
   if (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return FN_ERR_ALIGNMENT;
 
   const size_t wbytes = static_cast<size_t>(d) * ncols * (wt == FN_W_BF16 ? 2 : 1);
   const size_t xbytes = static_cast<size_t>(M) * d * 2;
   const size_t ybytes = static_cast<size_t>(M) * N * 2;
   const size_t sbytes = scales ? static_cast<size_t>(d / 128) * (ncols / 128) * 4 : 0;
-  if (overlaps(y, ybytes, x, xbytes) || overlaps(y, ybytes, Wp, wbytes) || overlaps(y, ybytes, scales, sbytes) ||
-      overlaps(y, ybytes, ws, ws_bytes) || overlaps(ws, ws_bytes, x, xbytes) || overlaps(ws, ws_bytes, Wp, wbytes))
-    return FN_ERR_ALIAS;
+  if (overlaps(ws, ws_bytes, x, xbytes) || overlaps(ws, ws_bytes, Wp, wbytes)) return FN_ERR_ALIAS;
+  // every output region against every input region, the workspace and each other
+  const size_t qbytes = static_cast<size_t>(M) * (N / 2), fbytes = static_cast<size_t>(M) * (N / 16);
+  const struct { const void* p; size_t n; } outs[3] = {{y, ybytes}, {yq, qbytes}, {ysf, fbytes}};
+  for (int i = 0; i < 3; ++i) {
+    if (!outs[i].p) continue;
+    if (overlaps(outs[i].p, outs[i].n, x, xbytes) || overlaps(outs[i].p, outs[i].n, Wp, wbytes) ||
+        overlaps(outs[i].p, outs[i].n, scales, sbytes) || overlaps(outs[i].p, outs[i].n, ws, ws_bytes) ||
+        overlaps(outs[i].p, outs[i].n, gscale, gscale ? 4 : 0))
+      return FN_ERR_ALIAS;
+    for (int j = i + 1; j < 3; ++j)
+      if (outs[j].p && overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return FN_ERR_ALIAS;
+  }
 
   int force = g_force_path.load();
   bool use_decode = M <= 64;
@@ -171,6 +187,9 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.swiglu = swiglu;
   a.eps = eps;
   a.y = y;
+  a.yq = yq;
+  a.ysf = ysf;
+  a.gscale = gscale;
   a.ws = ws;
   a.ws_bytes = ws_bytes;
   a.stream = reinterpret_cast<cudaStream_t>(stream);
@@ -248,6 +267,14 @@ fn_status fn_norm_proj_swiglu(const void* x, int64_t M, int64_t d, const void* W
                               fn_wtype wt, int64_t N, float eps, void* out, void* workspace, size_t ws_bytes,
                               fn_stream_t stream) {
   return norm_proj_common(x, M, d, Wp, scales, wt, N, eps, out, workspace, ws_bytes, stream, true);
+}
+
+fn_status fn_norm_proj_swiglu_nvfp4(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                                    fn_wtype wt, int64_t N, float eps, const float* global_scale, void* out_q,
+                                    void* out_sf, void* workspace, size_t ws_bytes, fn_stream_t stream) {
+  if (M > 0 && (!out_q || !out_sf || !global_scale)) return FN_ERR_INVALID_ARG;
+  return norm_proj_common(x, M, d, Wp, scales, wt, N, eps, nullptr, workspace, ws_bytes, stream, true, out_q,
+                          out_sf, global_scale);
 }
 
 fn_status fn_query_device_status(void* workspace, unsigned int* detail, fn_stream_t stream) {

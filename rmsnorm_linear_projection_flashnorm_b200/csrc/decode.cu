@@ -73,10 +73,12 @@ struct alignas(16) Bars {
   float rfix[MPAD];          // cluster mode: 1/rms of each row
 };
 
-template <int MPAD, int HALVES>
+// FP4: write the SwiGLU output in NVFP4 (yq, ysf) instead of bf16 y.
+template <int MPAD, int HALVES, bool FP4 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   const Params p) {
+  static_assert(!FP4 || HALVES == 2, "NVFP4 output is a SwiGLU epilogue");
   using C = Cfg<MPAD, HALVES>;
   constexpr int STAGES = C::STAGES;
   using B = Bars<MPAD, HALVES, STAGES>;
@@ -294,6 +296,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive(&bars.acc_empty[b]);
       const bool whole = (kb0 == 0 && kb1 == p.kblocks);
       if (whole) {
+        uint8_t* qbuf = reinterpret_cast<uint8_t*>(bars.ybuf);   // NVFP4 staging
+        const float gs = FP4 ? __ldg(p.gscale) : 0.f;
 #pragma unroll
         for (int m = 0; m < MPAD; ++m) {
           if (m >= p.M) break;
@@ -301,11 +305,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           float v;
           if (HALVES == 2) v = silu_f32(acc[0][m] * r) * (acc[1][m] * r);
           else v = acc[0][m] * r;
-          bars.ybuf[m * 128 + n] = __float2bfloat16_rn(v);
+          if constexpr (FP4) stage_fp4(qbuf, MPAD, m, n, v, gs);
+          else bars.ybuf[m * 128 + n] = __float2bfloat16_rn(v);
         }
         mbar_arrive(&bars.ssq_empty[b]);
         named_bar_sync(1, 128);
-        store_tile_rows(bars.ybuf, p, tile, et, 128);
+        if constexpr (FP4) store_tile_fp4(qbuf, MPAD, p, tile, et, 128);
+        else store_tile_rows(bars.ybuf, p, tile, et, 128);
         continue;
       }
       if (p.cluster > 1) {
@@ -455,7 +461,7 @@ bool clusters_fit(int S, int tiles, int threads, size_t smem) {
   return v - 1 >= tiles;
 }
 
-template <int MPAD, int HALVES>
+template <int MPAD, int HALVES, bool FP4 = false>
 cudaError_t launch_impl(const CallArgs& a) {
   if (a.ws_bytes < workspace_bytes<MPAD, HALVES>(a.d, a.ncols, a.num_sms)) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
@@ -487,30 +493,34 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.x = static_cast<const __nv_bfloat16*>(a.x);
   p.xhilo = nullptr;
   p.xfac = nullptr;
+  p.yq = static_cast<uint8_t*>(a.yq);
+  p.ysf = static_cast<uint8_t*>(a.ysf);
+  p.gscale = a.gscale;
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
-  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES>>(static_cast<int>(SMEM));
+  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES, FP4>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
   // Split K inside clusters when the tiles fill the GPU at least twice over
   // and every cluster can be resident at once; otherwise stream-K.
   // The largest cluster size whose clusters can all be resident (GPC sizes
   // decide that, not just the SM count), or the size forced by the caller.
   int S = a.cluster_mode >= 2 ? a.cluster_mode : cluster_split(p.tiles, p.kblocks, a.num_sms);
+  if (FP4) S = 1;   // the cluster finish writes bf16 only: NVFP4 output takes the stream-K path
   if (S > p.kblocks) S = p.kblocks;
   if (S > 8) S = 8;
-  while (S >= 2 && !clusters_fit<decode_kernel<MPAD, HALVES>>(S, p.tiles, NUM_THREADS, SMEM)) --S;
+  while (S >= 2 && !clusters_fit<decode_kernel<MPAD, HALVES, FP4>>(S, p.tiles, NUM_THREADS, SMEM)) --S;
   // Clusters only pay off when they occupy about as many SMs as stream-K
   // would: fewer SMs cannot pull the full HBM bandwidth.
   if (S >= 2 && a.cluster_mode != 0 && (a.cluster_mode >= 2 || 10LL * p.tiles * S >= 9LL * p.grid)) {
     p.cluster = S;
     p.grid = p.tiles * S;
     p.narrow = partition_is_narrow(p.total, p.grid) ? 1 : 0;
-    return launch_pdl_cluster(decode_kernel<MPAD, HALVES>, static_cast<unsigned>(p.grid), S, NUM_THREADS, SMEM,
+    return launch_pdl_cluster(decode_kernel<MPAD, HALVES, FP4>, static_cast<unsigned>(p.grid), S, NUM_THREADS, SMEM,
                               a.stream, tx, tw, p);
   }
-  e = launch_pdl(decode_kernel<MPAD, HALVES>, p.grid, NUM_THREADS, SMEM, a.stream, tx, tw, p);
+  e = launch_pdl(decode_kernel<MPAD, HALVES, FP4>, p.grid, NUM_THREADS, SMEM, a.stream, tx, tw, p);
   if (e != cudaSuccess) return e;
   if (!any_split_tile(p.grid, p.total, p.kblocks)) return cudaSuccess;
-  return launch_fixup<MPAD, HALVES>(p, a.stream);
+  return launch_fixup<MPAD, HALVES, FP4>(p, a.stream);
 }
 
 }  // namespace dec
@@ -533,6 +543,11 @@ size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, 
 cudaError_t launch_decode(const CallArgs& a) {
   const int mp = decode_mpad(a.M);
   if (a.wtype == 1) return launch_decode_fp8(a, mp);
+  if (a.yq) {   // NVFP4 output (SwiGLU only)
+    if (mp == 16) return dec::launch_impl<16, 2, true>(a);
+    if (mp == 32) return dec::launch_impl<32, 2, true>(a);
+    return dec::launch_impl<64, 2, true>(a);
+  }
   if (mp == 16) return a.swiglu ? dec::launch_impl<16, 2>(a) : dec::launch_impl<16, 1>(a);
   if (mp == 32) return a.swiglu ? dec::launch_impl<32, 2>(a) : dec::launch_impl<32, 1>(a);
   return a.swiglu ? dec::launch_impl<64, 2>(a) : dec::launch_impl<64, 1>(a);

@@ -15,6 +15,7 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 
 namespace fn {
@@ -47,6 +48,9 @@ struct Params {
   const __nv_bfloat16* x;    // the activations (read directly by the x-splitting kernel)
   uint8_t* xhilo;            // fp8, split once per call: e4m3 x_hi / x_lo rows [kblocks][2 MPAD][128]
   float* xfac;               // fp8, split once per call: 2^-e per [kblock][row]
+  uint8_t* yq;               // NVFP4 output (SwiGLU only; y is null then): codes [M][nout / 2]
+  uint8_t* ysf;              //   and e4m3 scale codes [M][nout / 16]
+  const float* gscale;       //   global scale (one fp32 value in device memory)
 };
 
 // One partial-result slot: float4 groups [half][row / 4][column] for the
@@ -97,6 +101,33 @@ __device__ __forceinline__ void store_tile_rows(const __nv_bfloat16* ybuf, const
   }
 }
 
+// NVFP4 form of store_tile_rows: the staged codes ([MPAD rows][64 bytes], the
+// tile's 128 columns) and scale bytes ([MPAD rows][8 bytes] after them) go to
+// yq and ysf with 16- and 8-byte stores.
+__device__ __forceinline__ void store_tile_fp4(const uint8_t* qbuf, int mpad, const Params& p, int tile, int et,
+                                               int nthr) {
+  const int64_t qrow = p.nout / 2, srow = p.nout / kFp4Block;
+  for (int i = et; i < p.M * 5; i += nthr) {
+    const int m = i / 5, c = i - 5 * (i / 5);
+    if (c < 4) {
+      *reinterpret_cast<uint4*>(p.yq + m * qrow + tile * 64 + c * 16) =
+          *reinterpret_cast<const uint4*>(qbuf + m * 64 + c * 16);
+    } else {
+      *reinterpret_cast<uint2*>(p.ysf + m * srow + tile * 8) =
+          *reinterpret_cast<const uint2*>(qbuf + mpad * 64 + m * 8);
+    }
+  }
+}
+
+// Stage row m of a tile's NVFP4 output from the 128 epilogue threads that
+// hold column n's value v (n = 0..127 across 4 warps; all lanes call).
+__device__ __forceinline__ void stage_fp4(uint8_t* qbuf, int mpad, int m, int n, float v, float gs) {
+  uint32_t pair;
+  const uint32_t sf = fp4_quantize_lane16(v, gs, pair);
+  if ((n & 1) == 0) qbuf[m * 64 + (n >> 1)] = static_cast<uint8_t>(pair);
+  if ((n & 15) == 0) qbuf[mpad * 64 + m * 8 + (n >> 4)] = static_cast<uint8_t>(sf);
+}
+
 // COLS consecutive fp32 TMEM columns of this warp's 32 lanes (16 or a
 // multiple of 32).
 template <int COLS>
@@ -127,8 +158,10 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[COLS]) {
 // 1/rms (and SwiGLU) and stores four bf16 outputs.
 constexpr int FIX_THREADS = 128;
 
-template <int MPAD, int HALVES>
+// FP4: write the SwiGLU output in NVFP4 (yq, ysf) instead of bf16 y.
+template <int MPAD, int HALVES, bool FP4 = false>
 __global__ void __launch_bounds__(FIX_THREADS) decode_fixup_kernel(const Params p) {
+  static_assert(!FP4 || HALVES == 2, "NVFP4 output is a SwiGLU epilogue");
   constexpr int SLOT = slot_floats<MPAD, HALVES>();
   // Let the next kernel in the stream launch now: its CTAs take SMs as the
   // stream-K CTAs leave and prefetch their weights into L2 meanwhile.  All
@@ -179,14 +212,24 @@ __global__ void __launch_bounds__(FIX_THREADS) decode_fixup_kernel(const Params 
   const float a1[4] = {acc[HALVES - 1].x, acc[HALVES - 1].y, acc[HALVES - 1].z, acc[HALVES - 1].w};
   const float sq[4] = {ss.x, ss.y, ss.z, ss.w};
   const int col = tile * 128 + n;
+  const float gs = FP4 ? __ldg(p.gscale) : 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int m = 4 * q + i;
-    if (m >= p.M) break;
+    if (m >= p.M) break;            // uniform: the block is one (tile, row group)
     const float r = inv_rms(sq[i], p.inv_d, p.eps);
     float v = a0[i] * r;
     if (HALVES == 2) v = silu_f32(v) * (a1[i] * r);
-    if (col < p.nout) p.y[static_cast<int64_t>(m) * p.nout + col] = __float2bfloat16_rn(v);
+    if constexpr (FP4) {
+      // NVFP4 output (SwiGLU: every tile column is an output column)
+      uint32_t pair;
+      const uint32_t sf = fp4_quantize_lane16(v, gs, pair);
+      if ((n & 1) == 0) p.yq[static_cast<int64_t>(m) * (p.nout / 2) + (col >> 1)] = static_cast<uint8_t>(pair);
+      if ((n & 15) == 0)
+        p.ysf[static_cast<int64_t>(m) * (p.nout / kFp4Block) + (col >> 4)] = static_cast<uint8_t>(sf);
+    } else if (col < p.nout) {
+      p.y[static_cast<int64_t>(m) * p.nout + col] = __float2bfloat16_rn(v);
+    }
   }
 }
 
@@ -203,11 +246,11 @@ inline bool any_split_tile(int grid, long long total, int kblocks) {
 }
 
 // Launch the fix-up for the stream-K grid described by `p`.
-template <int MPAD, int HALVES>
+template <int MPAD, int HALVES, bool FP4 = false>
 cudaError_t launch_fixup(const Params& p, cudaStream_t stream) {
   const long long threads = static_cast<long long>(p.tiles) * 128 * ((p.M + 3) / 4);
   const unsigned fgrid = static_cast<unsigned>((threads + FIX_THREADS - 1) / FIX_THREADS);
-  return launch_pdl(decode_fixup_kernel<MPAD, HALVES>, fgrid, FIX_THREADS, 0, stream, p);
+  return launch_pdl(decode_fixup_kernel<MPAD, HALVES, FP4>, fgrid, FIX_THREADS, 0, stream, p);
 }
 
 // Workspace needed by a decode call: the header and two partial slots per CTA

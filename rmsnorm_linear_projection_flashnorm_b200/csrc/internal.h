@@ -28,7 +28,10 @@ struct CallArgs {
   int64_t ncols;          // stored weight columns: N or 2N (SwiGLU)
   bool swiglu;
   float eps;
-  void* y;                // bf16 [M, N]
+  void* y;                // bf16 [M, N] (null with NVFP4 output)
+  void* yq;               // NVFP4 output, SwiGLU only: e2m1 codes [M, N/2] bytes, or null
+  void* ysf;              //   e4m3 scale codes [M, N/16]
+  const float* gscale;    //   global scale, one fp32 value in device memory
   void* ws;               // workspace (status word + decode scratch)
   size_t ws_bytes;
   cudaStream_t stream;

@@ -31,6 +31,7 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 
 namespace fn {
@@ -65,6 +66,9 @@ struct Params {
   unsigned long long budget_ns;
   int withhold;
   const float* scales;   // fp8: block scales [d/128][ncols/128]
+  uint8_t* yq;           // NVFP4 output (SwiGLU only; y is null then): codes [M][nout / 2]
+  uint8_t* ysf;          //   and e4m3 scale codes [M][nout / 16]
+  const float* gscale;   //   global scale (one fp32 value in device memory)
 };
 
 template <int STAGES>
@@ -104,10 +108,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
   }
 }
 
-template <bool SWIGLU, bool FP8>
+// FP4: write the SwiGLU output in NVFP4 (yq, ysf) instead of bf16 y.
+template <bool SWIGLU, bool FP8, bool FP4 = false>
 __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
               const Params p) {
+  static_assert(!FP4 || SWIGLU, "NVFP4 output is a SwiGLU epilogue");
   constexpr int STAGES = Cfg<FP8>::STAGES;
   constexpr int STAGE_BYTES = Cfg<FP8>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
@@ -303,7 +309,38 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
       const int grow = mb * BM + row;
       const bool row_ok = grow < p.M;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
-      if (SWIGLU) {
+      if constexpr (FP4) {
+        // NVFP4 output: this thread's row holds whole 16-column blocks
+        const float gs = __ldg(p.gscale);
+        uint8_t* qrow = p.yq + static_cast<int64_t>(grow) * (p.nout / 2) + nb * (BN / 4);
+        uint64_t sfw = 0;   // the tile row's 8 scale bytes
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t gv[32], uv[32];
+          tmem_ld32(taddr + c, gv);
+          tmem_ld32(taddr + BN / 2 + c, uv);
+          tmem_ld_wait();
+          uint32_t w[4];
+#pragma unroll
+          for (int blk = 0; blk < 2; ++blk) {
+            float o[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float g = __uint_as_float(gv[16 * blk + j]) * r, u = __uint_as_float(uv[16 * blk + j]) * r;
+              o[j] = silu_f32(g) * u;
+            }
+            uint2 q;
+            const uint32_t sf = fp4_quantize16(o, gs, q);
+            w[2 * blk] = q.x;
+            w[2 * blk + 1] = q.y;
+            sfw |= static_cast<uint64_t>(sf) << (8 * (c / 16 + blk));
+          }
+          if (row_ok) *reinterpret_cast<uint4*>(qrow + c / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        if (row_ok)
+          *reinterpret_cast<uint2*>(p.ysf + static_cast<int64_t>(grow) * (p.nout / kFp4Block) + nb * (BN / 32)) =
+              make_uint2(static_cast<uint32_t>(sfw), static_cast<uint32_t>(sfw >> 32));
+      } else if constexpr (SWIGLU) {
         __nv_bfloat16* yrow = p.y + static_cast<int64_t>(grow) * p.nout + nb * (BN / 2);
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
@@ -356,7 +393,7 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
   }
 }
 
-template <bool SWIGLU, bool FP8>
+template <bool SWIGLU, bool FP8, bool FP4 = false>
 cudaError_t launch_impl(const CallArgs& a) {
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, BM, BK)) return cudaErrorInvalidValue;
@@ -382,16 +419,20 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.budget_ns = a.budget_ns;
   p.withhold = a.withhold;
   p.scales = a.scales;
+  p.yq = static_cast<uint8_t*>(a.yq);
+  p.ysf = static_cast<uint8_t*>(a.ysf);
+  p.gscale = a.gscale;
   constexpr size_t SMEM_BYTES = smem_bytes<FP8>();
-  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU, FP8>>(static_cast<int>(SMEM_BYTES));
+  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU, FP8, FP4>>(static_cast<int>(SMEM_BYTES));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
-  return launch_pdl(tc_kernel<SWIGLU, FP8>, grid, Cfg<FP8>::NUM_THREADS, SMEM_BYTES, a.stream, tx, tw, p);
+  return launch_pdl(tc_kernel<SWIGLU, FP8, FP4>, grid, Cfg<FP8>::NUM_THREADS, SMEM_BYTES, a.stream, tx, tw, p);
 }
 
 }  // namespace tc
 
 cudaError_t launch_tc(const CallArgs& a) {
+  if (a.yq) return a.wtype == 1 ? tc::launch_impl<true, true, true>(a) : tc::launch_impl<true, false, true>(a);
   if (a.wtype == 1) return a.swiglu ? tc::launch_impl<true, true>(a) : tc::launch_impl<false, true>(a);
   return a.swiglu ? tc::launch_impl<true, false>(a) : tc::launch_impl<false, false>(a);
 }

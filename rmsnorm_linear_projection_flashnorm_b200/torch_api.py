@@ -8,7 +8,7 @@ from typing import Optional, Tuple
 import torch
 
 from . import (FN_W_BF16, FN_W_FP8_E4M3_B128, check, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
-               fn_query_device_status, fn_workspace_size)
+               fn_norm_proj_swiglu_nvfp4, fn_query_device_status, fn_workspace_size)
 
 
 def fold(W0: torch.Tensor, g: torch.Tensor, W1: Optional[torch.Tensor] = None, wtype: int = FN_W_BF16,
@@ -58,3 +58,23 @@ def norm_proj(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float, swiglu: boo
     fn = fn_norm_proj_swiglu if swiglu else fn_norm_proj
     check(fn(x, M, d, Wp, scales, wt, N, eps, out, buf, buf.numel(), stream), fn.__name__)
     return out
+
+
+def norm_proj_swiglu_nvfp4(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float, global_scale: torch.Tensor,
+                           scales: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None,
+                           out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """SwiGLU output in NVFP4: (codes uint8 [M, N/2], e4m3 scale bytes uint8
+    [M, N/16]); global_scale is a one-element fp32 device tensor."""
+    M, d = x.shape
+    wt = FN_W_BF16 if Wp.dtype == torch.bfloat16 else FN_W_FP8_E4M3_B128
+    if ws is None:
+        ws = Workspace(x.device)
+    buf = ws.get(M, d, N, wt, True)
+    if out is None:
+        out = (torch.empty((M, N // 2), dtype=torch.uint8, device=x.device),
+               torch.empty((M, N // 16), dtype=torch.uint8, device=x.device))
+    q, sf = out
+    check(fn_norm_proj_swiglu_nvfp4(x, M, d, Wp, scales, wt, N, eps, global_scale, q, sf, buf, buf.numel(), stream),
+          "fn_norm_proj_swiglu_nvfp4")
+    return q, sf

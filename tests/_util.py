@@ -74,3 +74,50 @@ def fold_fp8_ref(W0, g, W1=None, col_chunk: int = 1024):
     s = np.empty((sg.shape[0], 2 * sg.shape[1]), dtype=np.float32)
     s[:, 0::2], s[:, 1::2] = sg, su
     return O.interleave128(qg, qu), s
+
+
+def check_nvfp4(q_packed, sf, ref, gs: float, tol: float, min_exact: float = 0.97) -> float:
+    """Check the kernel's NVFP4 output (codes [M, N/2] bytes, scale bytes
+    [M, N/16]) against the oracle's fp64 SwiGLU values `ref` [M, N].
+
+    The kernel's fp32 value v lies within t = tol * (1 + |ref|) of ref, and a
+    quantised code is a decision on v, so the check accepts every code some v
+    in that band could give:
+      * the scale byte must lie between the oracle's scale codes for the
+        smallest and largest block maximum the band allows;
+      * given the kernel's scale, each element's e2m1 value must lie between
+        the oracle's roundings of the band's two ends;
+      * blocks where ref holds a non-finite value must carry the NaN scale
+        code 0x7F and zero codes.
+    Returns the fraction of codes (scale and element) equal to the oracle's
+    own encoding of ref, which must be at least `min_exact`."""
+    q = O.nvfp4_unpack(np.asarray(q_packed, dtype=np.uint8))
+    sf = np.asarray(sf, dtype=np.uint8)
+    ref = np.asarray(ref, dtype=np.float64)
+    M, N = ref.shape
+    assert q.shape == (M, N) and sf.shape == (M, N // 16)
+    gs = float(np.float32(gs))
+    blocks = ref.reshape(M, N // 16, 16)
+    bad_blk = ~np.all(np.isfinite(blocks), axis=2)
+    assert np.all(sf[bad_blk] == 0x7F), "non-finite blocks must carry the NaN scale"
+    assert np.all(q.reshape(M, N // 16, 16)[bad_blk] == 0), "non-finite blocks must carry zero codes"
+    fin = np.where(np.isfinite(blocks), blocks, 0.0)
+    t = tol * (1.0 + np.abs(fin))
+    amax_lo = np.max(np.maximum(np.abs(fin) - t, 0.0), axis=2)
+    amax_hi = np.max(np.abs(fin) + t, axis=2)
+    s_lo = O.e4m3_decode(O.e4m3_encode(gs * amax_lo / O.E2M1_MAX))
+    s_hi = O.e4m3_decode(O.e4m3_encode(gs * amax_hi / O.E2M1_MAX))
+    s_got = np.where(bad_blk, 0.0, O.e4m3_decode(np.where(bad_blk, 0, sf)))
+    ok_s = bad_blk | ((s_got >= s_lo) & (s_got <= s_hi))
+    assert ok_s.all(), f"{int((~ok_s).sum())} scale codes outside the band"
+    enc = np.where(s_got > 0, gs / np.where(s_got > 0, s_got, 1.0), 0.0)[:, :, None]
+    v_lo = O.e2m1_round((fin - t) * enc)
+    v_hi = O.e2m1_round((fin + t) * enc)
+    v_got = O.e2m1_decode(q).reshape(M, N // 16, 16)
+    ok_v = bad_blk[:, :, None] | ((v_got >= v_lo) & (v_got <= v_hi))
+    assert ok_v.all(), f"{int((~ok_v).sum())} element codes outside the band"
+    q_ref, sf_ref = O.nvfp4_quantize(ref, gs)
+    same = np.count_nonzero(sf == sf_ref) + np.count_nonzero(O.e2m1_decode(q) == O.e2m1_decode(q_ref))
+    frac = same / (sf.size + q.size)
+    assert frac >= min_exact, f"only {frac:.4f} of the codes equal the oracle's encoding"
+    return frac

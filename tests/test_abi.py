@@ -90,6 +90,39 @@ def test_empty_batch_is_a_noop(L):
     assert np_(M=0, swiglu=True, x=None, y=None, ws=None) == fnb.FN_OK
 
 
+GS = (1 << 37) + 4096     # global scale: 4-byte aligned
+Q = 1 << 38
+SF = 1 << 39
+
+
+def nvfp4_(x=A, M=4, d=256, Wp=B, scales=None, wt=0, N=512, eps=1e-6, gs=GS, q=Q, sf=SF, ws=WS,
+           ws_bytes=1 << 30):
+    return fnb.fn_norm_proj_swiglu_nvfp4(x, M, d, Wp, scales, wt, N, eps, gs, q, sf, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(M=-1), fnb.FN_ERR_INVALID_ARG),
+    (dict(gs=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(q=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(sf=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(N=500), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(q=Q + 8), fnb.FN_ERR_ALIGNMENT),
+    (dict(sf=SF + 8), fnb.FN_ERR_ALIGNMENT),
+    (dict(gs=GS + 2), fnb.FN_ERR_ALIGNMENT),
+    (dict(q=A + 16), fnb.FN_ERR_ALIAS),          # codes overlap x
+    (dict(sf=B + 64), fnb.FN_ERR_ALIAS),         # scale bytes overlap W'
+    (dict(sf=Q + 512), fnb.FN_ERR_ALIAS),        # codes [4, 256] bytes: 1 KB
+    (dict(gs=SF + 4), fnb.FN_ERR_ALIAS),         # global scale inside the scale bytes
+    (dict(q=WS + 256), fnb.FN_ERR_ALIAS),        # codes inside the workspace
+])
+def test_nvfp4_rejects_bad_arguments(L, kw, code):
+    assert nvfp4_(**kw) == code
+
+
+def test_nvfp4_empty_batch_is_a_noop(L):
+    assert nvfp4_(M=0, x=None, gs=None, q=None, sf=None, ws=None) == fnb.FN_OK
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(d=0), fnb.FN_ERR_INVALID_ARG),
     (dict(W0=None), fnb.FN_ERR_INVALID_ARG),

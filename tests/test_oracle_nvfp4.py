@@ -183,3 +183,48 @@ def test_planted_swapped_nibbles_fail(monkeypatch):
     monkeypatch.setattr(O, "nvfp4_pack", OF.nvfp4_pack)
     with pytest.raises(AssertionError):
         test_nvfp4_pack_layout()
+
+
+# ---------------------------------------------------------------------------
+# the GPU tests' band check, exercised on oracle encodings
+# ---------------------------------------------------------------------------
+def _band_case():
+    rng = np.random.default_rng(5)
+    ref = rng.standard_normal((8, 64)) * np.exp(rng.uniform(-2, 2, (8, 1)))
+    ref[3, 5] = np.nan
+    tol = 1e-2
+    gs = float(np.float32(448.0 * 6.0 / np.nanmax(np.abs(ref))))
+    # a stand-in for the kernel's value: anywhere inside the tolerance band
+    v = ref + rng.uniform(-0.9, 0.9, ref.shape) * tol * (1.0 + np.abs(ref))
+    q, sf = O.nvfp4_quantize(v, gs)
+    return ref, tol, gs, q, sf
+
+
+def test_band_check_accepts_values_inside_the_band():
+    from tests._util import check_nvfp4
+    ref, tol, gs, q, sf = _band_case()
+    frac = check_nvfp4(O.nvfp4_pack(q), sf, ref, gs, tol, min_exact=0.8)
+    assert 0.8 <= frac <= 1.0
+
+
+@pytest.mark.parametrize("mistake", ["swap_nibbles", "scale_up", "wrong_gs", "nan_scale_lost", "code_flip"])
+def test_band_check_rejects_planted_mistakes(mistake):
+    from tests._util import check_nvfp4
+    ref, tol, gs, q, sf = _band_case()
+    q, sf = q.copy(), sf.copy()
+    if mistake == "swap_nibbles":
+        packed = O.nvfp4_pack(q)
+        packed = ((packed & 0xF) << 4) | (packed >> 4)
+    else:
+        if mistake == "scale_up":
+            sf[0, 0] += 2                   # two e4m3 steps above the band
+        elif mistake == "wrong_gs":
+            q, sf = O.nvfp4_quantize(ref, gs * 3.0)
+        elif mistake == "nan_scale_lost":
+            sf[3, 0] = 0x30
+        elif mistake == "code_flip":
+            i = int(np.argmax(np.abs(O.e2m1_decode(q[0]))))
+            q[0, i] ^= 0x8                  # the sign of the largest element
+        packed = O.nvfp4_pack(q)
+    with pytest.raises(AssertionError):
+        check_nvfp4(packed, sf, ref, gs, tol, min_exact=0.8)

@@ -1,0 +1,136 @@
+"""GPU parity of the quantising SwiGLU epilogue (NVFP4 output) against the
+fp64 oracle, through the C ABI.
+
+The kernels encode their fp32 SwiGLU value; the oracle encodes its fp64
+value.  A code is a decision taken on that value, so the check (see
+tests/_util.check_nvfp4) accepts every code a value within the kernel
+tolerance could give, requires nearly all codes to equal the oracle's own
+encoding, and checks the non-finite blocks exactly.  Cases cover the decode
+kernel (bf16 and fp8 weights, whole tiles and tiles finished by the fix-up
+kernel), the tile kernel (bf16, fp8 converted per tile and fp8 dequantised
+once), ragged M, several global scales (including saturation and subnormal
+scales), NaN rows and repeated calls.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import rmsnorm_linear_projection_flashnorm_b200 as fnb
+import workloads as WL
+from rmsnorm_linear_projection_flashnorm_b200 import torch_api as T
+from tests._util import BF16_TOL, FP8_TOL, check_nvfp4, fold_fp8_ref, fold_ref_bf16, gpu
+
+pytestmark = pytest.mark.gpu
+FP8 = fnb.FN_W_FP8_E4M3_B128
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    fnb.build()
+    fnb.lib()
+    torch.cuda.init()
+    yield
+    fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 0)
+
+
+def _prepare(M, d, N, wt, seed, x=None, eps=None):
+    inp = WL.case(M, d, N, True, seed=seed)
+    if x is not None:
+        inp["x"] = x
+    if eps is not None:
+        inp["eps"] = eps
+    g = inp["g"]
+    if wt == FP8:
+        Wq, s = T.fold(gpu(inp["W_gate"]), gpu(g), gpu(inp["W_up"]), wtype=FP8)
+        q, sr = fold_fp8_ref(inp["W_gate"], g, inp["W_up"])
+        Wg, Wu = O.deinterleave128(O.dequant_fp8(q, sr))
+    else:
+        Wq, _ = T.fold(gpu(inp["W_gate"]), gpu(g), gpu(inp["W_up"]))
+        s = None
+        Wg, Wu = fold_ref_bf16(inp["W_gate"], g), fold_ref_bf16(inp["W_up"], g)
+    ref = O.norm_proj_swiglu(inp["x"], np.ones(d), Wg, Wu, inp["eps"])
+    return inp, Wq, s, ref
+
+
+def _run_nvfp4(inp, Wq, s, N, gs, ws=None):
+    gsd = torch.tensor([gs], dtype=torch.float32, device="cuda")
+    q, sf = T.norm_proj_swiglu_nvfp4(gpu(inp["x"]), Wq, N, inp["eps"], gsd, scales=s, ws=ws)
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), sf.cpu().numpy()
+
+
+def _gs_for(ref):
+    """The usual choice: the tensor maximum maps to the largest scale x value."""
+    amax = np.max(np.abs(ref[np.isfinite(ref)]))
+    return float(np.float32(448.0 * 6.0 / amax))
+
+
+@pytest.mark.parametrize("M,d,N,wt", [
+    (1, 512, 256, 0),        # decode: every tile split, finished by the fix-up kernel
+    (5, 256, 19200, 0),      # decode: 150 tiles on 148 SMs, whole tiles in the decode kernel
+    (33, 384, 640, 0),
+    (64, 256, 19200, 0),
+    (65, 256, 512, 0),       # tile kernel
+    (200, 512, 384, 0),      # tile kernel, ragged M
+    (3, 256, 19200, FP8),    # fp8 decode, whole tiles
+    (40, 384, 256, FP8),     # fp8 decode with the activations split once per call, fix-up
+    (64, 512, 640, FP8),
+    (130, 256, 384, FP8),    # fp8 tile kernel (per-tile conversion)
+    (1100, 256, 256, FP8),   # fp8, weight dequantised once into the workspace
+])
+def test_nvfp4_small(M, d, N, wt):
+    inp, Wq, s, ref = _prepare(M, d, N, wt, seed=401)
+    gs = _gs_for(ref)
+    q, sf = _run_nvfp4(inp, Wq, s, N, gs)
+    check_nvfp4(q, sf, ref, gs, FP8_TOL if wt == FP8 else BF16_TOL)
+
+
+@pytest.mark.parametrize("gs", [1.0, 1e6, 1e-3])
+@pytest.mark.parametrize("M", [4, 96])
+def test_nvfp4_global_scales(M, gs):
+    """gs = 1 gives scales near one, 1e6 saturates every scale at 448 and the
+    large elements at +-6, 1e-3 puts the scales in e4m3's subnormal range
+    (the smallest round to zero)."""
+    inp, Wq, s, ref = _prepare(M, 256, 512, 0, seed=402)
+    q, sf = _run_nvfp4(inp, Wq, s, 512, gs)
+    check_nvfp4(q, sf, ref, gs, BF16_TOL)
+    if gs == 1e6:
+        assert np.all(sf == 0x7E)
+
+
+@pytest.mark.parametrize("M,wt", [(6, 0), (70, 0), (6, FP8), (70, FP8)])
+def test_nvfp4_nan_rows(M, wt):
+    """A zero row with eps = 0 has no finite 1/rms: its blocks carry the NaN
+    scale code and zero codes; the other rows are unaffected."""
+    inp = WL.case(M, 256, 256, True, seed=403)
+    x = inp["x"].clone()
+    x[1] = 0
+    x[M - 1] = 0
+    inp, Wq, s, ref = _prepare(M, 256, 256, wt, seed=403, x=x, eps=0.0)
+    assert np.all(np.isnan(ref[1])) and np.all(np.isfinite(ref[0]))
+    gs = _gs_for(ref)
+    q, sf = _run_nvfp4(inp, Wq, s, 256, gs)
+    check_nvfp4(q, sf, ref, gs, FP8_TOL if wt == FP8 else BF16_TOL)
+    assert np.all(sf[1] == 0x7F) and np.all(sf[0] != 0x7F)
+
+
+def test_nvfp4_ffn_decode_workload():
+    w = WL.WORKLOADS["ffn_swiglu"]
+    inp, Wq, s, ref = _prepare(16, w.d, w.N, 0, seed=w.seed)
+    gs = _gs_for(ref)
+    q, sf = _run_nvfp4(inp, Wq, s, w.N, gs)
+    frac = check_nvfp4(q, sf, ref, gs, BF16_TOL)
+    assert frac > 0.99
+
+
+@pytest.mark.parametrize("M,wt", [(16, 0), (300, 0), (48, FP8)])
+def test_nvfp4_repeated_calls_bit_identical(M, wt):
+    inp, Wq, s, ref = _prepare(M, 512, 1024, wt, seed=404)
+    ws = T.Workspace()
+    gs = _gs_for(ref)
+    q0, sf0 = _run_nvfp4(inp, Wq, s, 1024, gs, ws=ws)
+    for _ in range(20):
+        q1, sf1 = _run_nvfp4(inp, Wq, s, 1024, gs, ws=ws)
+        assert np.array_equal(q0, q1) and np.array_equal(sf0, sf1)
+    assert ws.status()[0] == fnb.FN_OK
