@@ -134,3 +134,57 @@ def test_nvfp4_repeated_calls_bit_identical(M, wt):
         q1, sf1 = _run_nvfp4(inp, Wq, s, 1024, gs, ws=ws)
         assert np.array_equal(q0, q1) and np.array_equal(sf0, sf1)
     assert ws.status()[0] == fnb.FN_OK
+
+
+def _sample_blocks(N: int, seed: int) -> np.ndarray:
+    """One whole 16-column block in every 128-column output tile."""
+    rng = np.random.default_rng(30_000 + seed)
+    return np.array([t * 8 + int(rng.integers(0, 8)) for t in range(N // 128)], dtype=np.int64)
+
+
+def _check_sampled(q, sf, rows, blocks, ref, gs, tol):
+    cols = (blocks[:, None] * 16 + np.arange(16)[None, :]).reshape(-1)
+    codes = O.nvfp4_unpack(q[rows])[:, cols]
+    return check_nvfp4(O.nvfp4_pack(codes), sf[rows][:, blocks], ref, gs, tol)
+
+
+def test_nvfp4_ffn_prefill_workload_sampled():
+    """FFN SwiGLU at M = 4096 (tile kernel) on the full workload, checked on
+    the deterministic row sample and one whole scale block per output tile."""
+    w = WL.WORKLOADS["ffn_swiglu"]
+    M = 4096
+    inp = WL.workload_case("ffn_swiglu", M)
+    x, g, Wg, Wu = inp["x"], inp["g"], inp["W_gate"], inp["W_up"]
+    Wp, _ = T.fold(gpu(Wg), gpu(g), gpu(Wu))
+    rows = WL.sample_rows(M, w.seed)
+    blocks = _sample_blocks(w.N, w.seed)
+    cols = (blocks[:, None] * 16 + np.arange(16)[None, :]).reshape(-1)
+    ref = O.norm_proj_swiglu(x[rows], np.ones(w.d), fold_ref_bf16(Wg[:, cols], g), fold_ref_bf16(Wu[:, cols], g),
+                             inp["eps"])
+    gs = _gs_for(ref)
+    q, sf = _run_nvfp4(inp, Wp, None, w.N, gs)
+    assert _check_sampled(q, sf, rows, blocks, ref, gs, BF16_TOL) > 0.99
+
+
+@pytest.fixture(scope="module")
+def fp8_workload():
+    w = WL.WORKLOADS["fp8_swiglu"]
+    inp = WL.workload_case("fp8_swiglu", 256)
+    g = inp["g"]
+    Wq, s = T.fold(gpu(inp["W_gate"]), gpu(g), gpu(inp["W_up"]), wtype=FP8)
+    q, sr = fold_fp8_ref(inp["W_gate"], g, inp["W_up"])
+    Wg, Wu = O.deinterleave128(O.dequant_fp8(q, sr))
+    torch.cuda.synchronize()
+    return w, inp, Wq, s, Wg, Wu
+
+
+@pytest.mark.parametrize("M", [1, 64, 256])
+def test_nvfp4_fp8_workload(fp8_workload, M):
+    """The fp8 SwiGLU workload (d = 5120, N = 13824): decode kernel with the
+    in-kernel and the once-per-call activation split, and the tile kernel."""
+    w, inp, Wq, s, Wg, Wu = fp8_workload
+    x = inp["x"][:M]
+    ref = O.norm_proj_swiglu(x, np.ones(w.d), Wg, Wu, inp["eps"])
+    gs = _gs_for(ref)
+    q, sf = _run_nvfp4({"x": x, "eps": inp["eps"]}, Wq, s, w.N, gs)
+    assert check_nvfp4(q, sf, ref, gs, FP8_TOL) > 0.99
