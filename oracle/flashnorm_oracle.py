@@ -64,6 +64,7 @@ __all__ = [
     "FP8_BLOCK", "E4M3_MAX",
     "E2M1", "E2M1_MAX", "NVFP4_BLOCK", "e2m1_round", "e2m1_encode", "e2m1_decode",
     "nvfp4_quantize", "nvfp4_pack", "nvfp4_unpack", "nvfp4_dequantize",
+    "rowparallel_partial", "rowparallel_finish",
 ]
 
 FP8_BLOCK = 128
@@ -385,3 +386,28 @@ def nvfp4_dequantize(codes, sf, global_scale: float) -> np.ndarray:
     gs = float(np.float32(global_scale))
     scale = np.repeat(e4m3_decode(sf), NVFP4_BLOCK, axis=1)
     return e2m1_decode(codes) * scale / gs
+
+
+# ---------------------------------------------------------------------------
+# Row-parallel (d-split) form of the deferred normalisation
+# ---------------------------------------------------------------------------
+def rowparallel_partial(x_local, W_local) -> Tuple[np.ndarray, np.ndarray]:
+    """One rank's share when the input width d is split across ranks: the
+    unscaled products over this rank's columns of x (rows of W) and the sums
+    of squares of those columns.  Proposal 2 (deferred normalisation) applies
+    1/rms after the matmul, and both quantities are sums over k, so the shares
+    of all ranks add up to the single-device values."""
+    x = to_f64(x_local)
+    return x @ to_f64(W_local), np.sum(x * x, axis=1)
+
+
+def rowparallel_finish(acc, ssq, d_total: int, eps: float, swiglu: bool = False) -> np.ndarray:
+    """The post-scale after the shares were summed: r = 1/sqrt(ssq/d + eps)
+    with d the full width, then r * acc, or silu(r * gate) * (r * up) with the
+    gate and up columns in the interleaved stored order."""
+    acc = np.asarray(acc, dtype=np.float64)
+    r = 1.0 / np.sqrt(np.asarray(ssq, dtype=np.float64) / d_total + eps)
+    if not swiglu:
+        return acc * r[:, None]
+    gate, up = deinterleave128(acc)
+    return silu(gate * r[:, None]) * (up * r[:, None])

@@ -383,3 +383,43 @@ def test_pins_catch_planted_swiglu_mistakes():
     assert not _pins_pass(O.norm_proj, silu_sign, O.interleave128)
     swapped_interleave = lambda A, B: O.interleave128(B, A)
     assert not _pins_pass(O.norm_proj, O.norm_proj_swiglu, swapped_interleave)
+
+
+# ---------------------------------------------------------------------------
+# row-parallel (d-split) form: shares over any partition of d add up to the
+# single-device result (the definition computed the unfolded way)
+# ---------------------------------------------------------------------------
+def _partition(d, parts, rng):
+    cuts = np.sort(rng.choice(np.arange(1, d), size=parts - 1, replace=False)) if parts > 1 else np.array([], int)
+    edges = np.concatenate([[0], cuts, [d]])
+    return list(zip(edges[:-1], edges[1:]))
+
+
+@pytest.mark.parametrize("parts", [1, 2, 3, 7])
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_rowparallel_shares_add_up(parts, swiglu):
+    rng = np.random.default_rng(parts * 10 + swiglu)
+    M, d, N = 5, 48, 256
+    x = rng.standard_normal((M, d)) * np.exp(rng.uniform(-2, 2, (M, 1)))
+    Wg = rng.standard_normal((d, N)) / np.sqrt(d)
+    Wu = rng.standard_normal((d, N)) / np.sqrt(d)
+    W = O.interleave128(Wg, Wu) if swiglu else Wg
+    acc = np.zeros((M, W.shape[1]))
+    ssq = np.zeros(M)
+    for k0, k1 in _partition(d, parts, rng):
+        a, s = O.rowparallel_partial(x[:, k0:k1], W[k0:k1])
+        acc += a
+        ssq += s
+    y = O.rowparallel_finish(acc, ssq, d, 1e-6, swiglu)
+    want = (O.norm_proj_swiglu(x, np.ones(d), Wg, Wu, 1e-6) if swiglu else O.norm_proj(x, np.ones(d), Wg, 1e-6))
+    assert np.max(np.abs(y - want) / (1 + np.abs(want))) < 1e-12
+
+
+def test_rowparallel_finish_closed_form():
+    """A constant row c with eps = 0: r = 1/|c|, so y = sign(c) * sum_k W[k]."""
+    d, N = 16, 128
+    W = np.random.default_rng(2).standard_normal((d, N))
+    x = np.full((1, d), -3.0)
+    acc, ssq = O.rowparallel_partial(x, W)
+    y = O.rowparallel_finish(acc, ssq, d, 0.0)
+    assert np.allclose(y[0], -W.sum(axis=0), rtol=1e-13, atol=1e-13)
