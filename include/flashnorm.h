@@ -153,6 +153,49 @@ fn_status fn_norm_proj_swiglu_nvfp4(const void* x, int64_t M, int64_t d, const v
                                     void* out_sf, void* workspace, size_t ws_bytes, fn_stream_t stream);
 
 /*
+ * Row-parallel (d-split) projection, for tensor parallelism that shards the
+ * input width d across ranks.  The deferred normalisation (FlashNorm talk
+ * summary, Proposal 2) makes 1/rms a per-row factor applied after the matmul,
+ * and sum_k x[m,k]^2 splits over k like the matmul, so each rank computes the
+ * unscaled products and the sum of squares of its own k range, one all-reduce
+ * (sum) of one buffer per rank combines them, and fn_post_scale finishes.
+ *
+ * fn_norm_proj_partial — this rank's share:
+ *   x         bf16 [M, d] — this rank's contiguous columns of the activations
+ *             (d = the rank's width: % 64, % 128 with fp8 weights)
+ *   Wp        this rank's rows of the folded weight [d, ncols] (a row slice of
+ *             fn_fold_weights' output; for fp8 the matching rows of scales, so
+ *             the slice starts on a 128-row boundary)
+ *   ncols     stored columns: N for a plain projection, 2N for a SwiGLU weight
+ *             (computed as a plain projection of its stored columns here)
+ *   partial   fp32, M * ncols + M values, 16-byte aligned: [M, ncols] sums
+ *             x @ Wp in stored column order, then [M] sums of x^2 over this
+ *             rank's columns; nothing is post-scaled
+ *   workspace >= fn_workspace_size(M, d, ncols, wt, 0)
+ *   M == 0 is a no-op.  The partial buffer must not overlap the inputs or the
+ *   workspace (FN_ERR_ALIAS).
+ */
+fn_status fn_norm_proj_partial(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                               fn_wtype wt, int64_t ncols, float* partial, void* workspace, size_t ws_bytes,
+                               fn_stream_t stream);
+
+/*
+ * fn_post_scale — finish a row-parallel projection from the summed partial
+ * buffer (the all-reduce of every rank's fn_norm_proj_partial output):
+ *   r[m] = 1/sqrt(ssq[m] / d_total + eps), d_total the full input width;
+ *   y = r * acc (plain), or silu(r * gate) * (r * up) for swiglu != 0, with
+ *   the gate and up columns read from the interleaved stored order;
+ *   one round to bf16 into y [M, N], 16-byte aligned, not overlapping partial.
+ * With one rank (d_total = d) the result equals fn_norm_proj on the same
+ * inputs up to the rounding order of the sums: bit for bit for M > 64 (every
+ * column tile reduces a row's sum of squares in the same k order), while for
+ * M <= 64 the fused call may cut different column tiles' k ranges at
+ * different points, and the partial buffer carries one sum of squares per row.
+ */
+fn_status fn_post_scale(const float* partial, int64_t M, int64_t N, int swiglu, int64_t d_total, float eps, void* y,
+                        fn_stream_t stream);
+
+/*
  * fn_norm_proj_static — fn_norm_proj for callers that cannot allocate device
  * memory, so cannot pass a workspace: code recording work under a CUDA stream
  * capture (where cudaMalloc is not permitted), plug-ins whose host application

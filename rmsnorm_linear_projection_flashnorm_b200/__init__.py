@@ -44,6 +44,8 @@ _SIGNATURES = {
     "fn_norm_proj_swiglu": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp, _sz, _vp]),
     "fn_norm_proj_swiglu_nvfp4": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp, _vp, _vp, _sz,
                                          _vp]),
+    "fn_norm_proj_partial": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _vp, _vp, _sz, _vp]),
+    "fn_post_scale": (_int, [_vp, _i64, _i64, _int, _i64, _f32, _vp, _vp]),
     "fn_norm_proj_static": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp]),
     "fn_query_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_uint), _vp]),
     "fn_rmsnorm": (_int, [_vp, _i64, _i64, _vp, _f32, _vp, _vp]),
@@ -145,6 +147,16 @@ def fn_norm_proj_swiglu_nvfp4(x, M: int, d: int, Wp, scales, wt: int, N: int, ep
                               out_sf, workspace, ws_bytes: int, stream=None) -> int:
     return lib().fn_norm_proj_swiglu_nvfp4(_ptr(x), M, d, _ptr(Wp), _ptr(scales), wt, N, eps, _ptr(global_scale),
                                            _ptr(out_q), _ptr(out_sf), _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def fn_norm_proj_partial(x, M: int, d: int, Wp, scales, wt: int, ncols: int, partial, workspace, ws_bytes: int,
+                         stream=None) -> int:
+    return lib().fn_norm_proj_partial(_ptr(x), M, d, _ptr(Wp), _ptr(scales), wt, ncols, _ptr(partial),
+                                      _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def fn_post_scale(partial, M: int, N: int, swiglu: int, d_total: int, eps: float, y, stream=None) -> int:
+    return lib().fn_post_scale(_ptr(partial), M, N, swiglu, d_total, eps, _ptr(y), _stream(stream))
 
 
 def fn_norm_proj_static(x, M: int, d: int, Wp, scales, wt: int, N: int, eps: float, y, stream=None) -> int:

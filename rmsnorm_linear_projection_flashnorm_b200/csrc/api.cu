@@ -120,8 +120,10 @@ fn_status check_device(int& sms) {
 // ysf and the global scale gscale, with y null.
 fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
                            int64_t N, float eps, void* y, void* ws, size_t ws_bytes, fn_stream_t stream,
-                           bool swiglu, void* yq = nullptr, void* ysf = nullptr, const float* gscale = nullptr) {
+                           bool swiglu, void* yq = nullptr, void* ysf = nullptr, const float* gscale = nullptr,
+                           float* part_out = nullptr) {
   const bool fp4 = yq != nullptr || ysf != nullptr || gscale != nullptr;
+  const bool partial = part_out != nullptr;
   if (M < 0 || d <= 0 || N <= 0) return FN_ERR_INVALID_ARG;
   if (wt != FN_W_BF16 && wt != FN_W_FP8_E4M3_B128) return FN_ERR_INVALID_ARG;
   if (!eps_ok(eps)) return FN_ERR_INVALID_ARG;
@@ -131,11 +133,14 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   if (M > kMaxDim || d > kMaxDim || ncols > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FN_OK;
   if (!x || !Wp) return FN_ERR_INVALID_ARG;
-  if (fp4 ? (!yq || !ysf || !gscale || y || !swiglu) : !y) return FN_ERR_INVALID_ARG;
+  if (partial ? (y || fp4 || swiglu) : fp4 ? (!yq || !ysf || !gscale || y || !swiglu) : !y)
+    return FN_ERR_INVALID_ARG;
   if (!ws) return FN_ERR_WORKSPACE;
   if (wt == FN_W_FP8_E4M3_B128 && !scales) return FN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wp) || !aligned16(ws)) return FN_ERR_ALIGNMENT;
-  if (fp4 ? (!aligned16(yq) || !aligned16(ysf) || (reinterpret_cast<uintptr_t>(gscale) & 3u)) : !aligned16(y))
+  if (partial ? !aligned16(part_out)
+              : fp4 ? (!aligned16(yq) || !aligned16(ysf) || (reinterpret_cast<uintptr_t>(gscale) & 3u))
+                    : !aligned16(y))
     return FN_ERR_ALIGNMENT;
   if (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return FN_ERR_ALIGNMENT;
 
@@ -146,14 +151,15 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   if (overlaps(ws, ws_bytes, x, xbytes) || overlaps(ws, ws_bytes, Wp, wbytes)) return FN_ERR_ALIAS;
   // every output region against every input region, the workspace and each other
   const size_t qbytes = static_cast<size_t>(M) * (N / 2), fbytes = static_cast<size_t>(M) * (N / 16);
-  const struct { const void* p; size_t n; } outs[3] = {{y, ybytes}, {yq, qbytes}, {ysf, fbytes}};
-  for (int i = 0; i < 3; ++i) {
+  const size_t pbytes = partial ? (static_cast<size_t>(M) * ncols + M) * 4 : 0;
+  const struct { const void* p; size_t n; } outs[4] = {{y, ybytes}, {yq, qbytes}, {ysf, fbytes}, {part_out, pbytes}};
+  for (int i = 0; i < 4; ++i) {
     if (!outs[i].p) continue;
     if (overlaps(outs[i].p, outs[i].n, x, xbytes) || overlaps(outs[i].p, outs[i].n, Wp, wbytes) ||
         overlaps(outs[i].p, outs[i].n, scales, sbytes) || overlaps(outs[i].p, outs[i].n, ws, ws_bytes) ||
         overlaps(outs[i].p, outs[i].n, gscale, gscale ? 4 : 0))
       return FN_ERR_ALIAS;
-    for (int j = i + 1; j < 3; ++j)
+    for (int j = i + 1; j < 4; ++j)
       if (outs[j].p && overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return FN_ERR_ALIAS;
   }
 
@@ -190,6 +196,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.yq = yq;
   a.ysf = ysf;
   a.gscale = gscale;
+  a.part_out = part_out;
   a.ws = ws;
   a.ws_bytes = ws_bytes;
   a.stream = reinterpret_cast<cudaStream_t>(stream);
@@ -275,6 +282,34 @@ fn_status fn_norm_proj_swiglu_nvfp4(const void* x, int64_t M, int64_t d, const v
   if (M > 0 && (!out_q || !out_sf || !global_scale)) return FN_ERR_INVALID_ARG;
   return norm_proj_common(x, M, d, Wp, scales, wt, N, eps, nullptr, workspace, ws_bytes, stream, true, out_q,
                           out_sf, global_scale);
+}
+
+fn_status fn_norm_proj_partial(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                               fn_wtype wt, int64_t ncols, float* partial, void* workspace, size_t ws_bytes,
+                               fn_stream_t stream) {
+  if (M > 0 && !partial) return FN_ERR_INVALID_ARG;
+  return norm_proj_common(x, M, d, Wp, scales, wt, ncols, 0.0f, nullptr, workspace, ws_bytes, stream, false,
+                          nullptr, nullptr, nullptr, partial);
+}
+
+fn_status fn_post_scale(const float* partial, int64_t M, int64_t N, int swiglu, int64_t d_total, float eps, void* y,
+                        fn_stream_t stream) {
+  if (M < 0 || N <= 0 || d_total <= 0) return FN_ERR_INVALID_ARG;
+  if (!eps_ok(eps)) return FN_ERR_INVALID_ARG;
+  if (N % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
+  const int64_t ncols = swiglu ? 2 * N : N;
+  if (M > kMaxDim || ncols > kMaxDim || d_total > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return FN_OK;
+  if (!partial || !y) return FN_ERR_INVALID_ARG;
+  if (!aligned16(partial) || !aligned16(y)) return FN_ERR_ALIGNMENT;
+  if (overlaps(y, static_cast<size_t>(M) * N * 2, partial, (static_cast<size_t>(M) * ncols + M) * 4))
+    return FN_ERR_ALIAS;
+  int sms = 0;
+  const fn_status st = check_device(sms);
+  if (st != FN_OK) return st;
+  const cudaError_t e =
+      launch_post_scale(partial, M, N, swiglu != 0, d_total, eps, y, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FN_OK : FN_ERR_CUDA;
 }
 
 fn_status fn_query_device_status(void* workspace, unsigned int* detail, fn_stream_t stream) {

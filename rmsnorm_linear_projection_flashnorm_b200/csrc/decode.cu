@@ -73,12 +73,13 @@ struct alignas(16) Bars {
   float rfix[MPAD];          // cluster mode: 1/rms of each row
 };
 
-// FP4: write the SwiGLU output in NVFP4 (yq, ysf) instead of bf16 y.
-template <int MPAD, int HALVES, bool FP4 = false>
+// OUT: bf16 y, NVFP4 codes and scales (SwiGLU only), or fp32 partials (OutKind).
+template <int MPAD, int HALVES, int OUT = kOutBf16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   const Params p) {
-  static_assert(!FP4 || HALVES == 2, "NVFP4 output is a SwiGLU epilogue");
+  static_assert(OUT != kOutNvfp4 || HALVES == 2, "NVFP4 output is a SwiGLU epilogue");
+  static_assert(OUT != kOutPartial || HALVES == 1, "partial output: plain projection of the stored columns");
   using C = Cfg<MPAD, HALVES>;
   constexpr int STAGES = C::STAGES;
   using B = Bars<MPAD, HALVES, STAGES>;
@@ -295,9 +296,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       mbar_arrive(&bars.acc_empty[b]);
       const bool whole = (kb0 == 0 && kb1 == p.kblocks);
+      if (whole && OUT == kOutPartial) {
+        // the tile's fp32 accumulators and (tile 0) the sums of squares, not post-scaled
+#pragma unroll
+        for (int m = 0; m < MPAD; ++m) {
+          if (m >= p.M) break;
+          p.part_out[static_cast<int64_t>(m) * p.ncols + tile * 128 + n] = acc[0][m];
+        }
+        if (tile == 0 && et < p.M) p.part_out[static_cast<int64_t>(p.M) * p.ncols + et] = bars.ssq[b][et];
+        mbar_arrive(&bars.ssq_empty[b]);
+        continue;
+      }
       if (whole) {
         uint8_t* qbuf = reinterpret_cast<uint8_t*>(bars.ybuf);   // NVFP4 staging
-        const float gs = FP4 ? __ldg(p.gscale) : 0.f;
+        const float gs = OUT == kOutNvfp4 ? __ldg(p.gscale) : 0.f;
 #pragma unroll
         for (int m = 0; m < MPAD; ++m) {
           if (m >= p.M) break;
@@ -305,12 +317,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           float v;
           if (HALVES == 2) v = silu_f32(acc[0][m] * r) * (acc[1][m] * r);
           else v = acc[0][m] * r;
-          if constexpr (FP4) stage_fp4(qbuf, MPAD, m, n, v, gs);
+          if constexpr (OUT == kOutNvfp4) stage_fp4(qbuf, MPAD, m, n, v, gs);
           else bars.ybuf[m * 128 + n] = __float2bfloat16_rn(v);
         }
         mbar_arrive(&bars.ssq_empty[b]);
         named_bar_sync(1, 128);
-        if constexpr (FP4) store_tile_fp4(qbuf, MPAD, p, tile, et, 128);
+        if constexpr (OUT == kOutNvfp4) store_tile_fp4(qbuf, MPAD, p, tile, et, 128);
         else store_tile_rows(bars.ybuf, p, tile, et, 128);
         continue;
       }
@@ -461,7 +473,7 @@ bool clusters_fit(int S, int tiles, int threads, size_t smem) {
   return v - 1 >= tiles;
 }
 
-template <int MPAD, int HALVES, bool FP4 = false>
+template <int MPAD, int HALVES, int OUT = kOutBf16>
 cudaError_t launch_impl(const CallArgs& a) {
   if (a.ws_bytes < workspace_bytes<MPAD, HALVES>(a.d, a.ncols, a.num_sms)) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
@@ -496,31 +508,32 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.yq = static_cast<uint8_t*>(a.yq);
   p.ysf = static_cast<uint8_t*>(a.ysf);
   p.gscale = a.gscale;
+  p.part_out = a.part_out;
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
-  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES, FP4>>(static_cast<int>(SMEM));
+  cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES, OUT>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
   // Split K inside clusters when the tiles fill the GPU at least twice over
   // and every cluster can be resident at once; otherwise stream-K.
   // The largest cluster size whose clusters can all be resident (GPC sizes
   // decide that, not just the SM count), or the size forced by the caller.
   int S = a.cluster_mode >= 2 ? a.cluster_mode : cluster_split(p.tiles, p.kblocks, a.num_sms);
-  if (FP4) S = 1;   // the cluster finish writes bf16 only: NVFP4 output takes the stream-K path
+  if (OUT != kOutBf16) S = 1;   // the cluster finish writes bf16 only: other outputs take the stream-K path
   if (S > p.kblocks) S = p.kblocks;
   if (S > 8) S = 8;
-  while (S >= 2 && !clusters_fit<decode_kernel<MPAD, HALVES, FP4>>(S, p.tiles, NUM_THREADS, SMEM)) --S;
+  while (S >= 2 && !clusters_fit<decode_kernel<MPAD, HALVES, OUT>>(S, p.tiles, NUM_THREADS, SMEM)) --S;
   // Clusters only pay off when they occupy about as many SMs as stream-K
   // would: fewer SMs cannot pull the full HBM bandwidth.
   if (S >= 2 && a.cluster_mode != 0 && (a.cluster_mode >= 2 || 10LL * p.tiles * S >= 9LL * p.grid)) {
     p.cluster = S;
     p.grid = p.tiles * S;
     p.narrow = partition_is_narrow(p.total, p.grid) ? 1 : 0;
-    return launch_pdl_cluster(decode_kernel<MPAD, HALVES, FP4>, static_cast<unsigned>(p.grid), S, NUM_THREADS, SMEM,
+    return launch_pdl_cluster(decode_kernel<MPAD, HALVES, OUT>, static_cast<unsigned>(p.grid), S, NUM_THREADS, SMEM,
                               a.stream, tx, tw, p);
   }
-  e = launch_pdl(decode_kernel<MPAD, HALVES, FP4>, p.grid, NUM_THREADS, SMEM, a.stream, tx, tw, p);
+  e = launch_pdl(decode_kernel<MPAD, HALVES, OUT>, p.grid, NUM_THREADS, SMEM, a.stream, tx, tw, p);
   if (e != cudaSuccess) return e;
   if (!any_split_tile(p.grid, p.total, p.kblocks)) return cudaSuccess;
-  return launch_fixup<MPAD, HALVES, FP4>(p, a.stream);
+  return launch_fixup<MPAD, HALVES, OUT>(p, a.stream);
 }
 
 }  // namespace dec
@@ -543,10 +556,15 @@ size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, 
 cudaError_t launch_decode(const CallArgs& a) {
   const int mp = decode_mpad(a.M);
   if (a.wtype == 1) return launch_decode_fp8(a, mp);
+  if (a.part_out) {   // partial output: a plain projection of the stored columns
+    if (mp == 16) return dec::launch_impl<16, 1, kOutPartial>(a);
+    if (mp == 32) return dec::launch_impl<32, 1, kOutPartial>(a);
+    return dec::launch_impl<64, 1, kOutPartial>(a);
+  }
   if (a.yq) {   // NVFP4 output (SwiGLU only)
-    if (mp == 16) return dec::launch_impl<16, 2, true>(a);
-    if (mp == 32) return dec::launch_impl<32, 2, true>(a);
-    return dec::launch_impl<64, 2, true>(a);
+    if (mp == 16) return dec::launch_impl<16, 2, kOutNvfp4>(a);
+    if (mp == 32) return dec::launch_impl<32, 2, kOutNvfp4>(a);
+    return dec::launch_impl<64, 2, kOutNvfp4>(a);
   }
   if (mp == 16) return a.swiglu ? dec::launch_impl<16, 2>(a) : dec::launch_impl<16, 1>(a);
   if (mp == 32) return a.swiglu ? dec::launch_impl<32, 2>(a) : dec::launch_impl<32, 1>(a);

@@ -51,6 +51,7 @@ struct Params {
   uint8_t* yq;               // NVFP4 output (SwiGLU only; y is null then): codes [M][nout / 2]
   uint8_t* ysf;              //   and e4m3 scale codes [M][nout / 16]
   const float* gscale;       //   global scale (one fp32 value in device memory)
+  float* part_out;           // partial output: fp32 [M][ncols] accumulators, then [M] sums of squares
 };
 
 // One partial-result slot: float4 groups [half][row / 4][column] for the
@@ -158,10 +159,11 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[COLS]) {
 // 1/rms (and SwiGLU) and stores four bf16 outputs.
 constexpr int FIX_THREADS = 128;
 
-// FP4: write the SwiGLU output in NVFP4 (yq, ysf) instead of bf16 y.
-template <int MPAD, int HALVES, bool FP4 = false>
+// OUT: bf16 y, NVFP4 codes and scales (SwiGLU only), or fp32 partials (OutKind).
+template <int MPAD, int HALVES, int OUT = kOutBf16>
 __global__ void __launch_bounds__(FIX_THREADS) decode_fixup_kernel(const Params p) {
-  static_assert(!FP4 || HALVES == 2, "NVFP4 output is a SwiGLU epilogue");
+  static_assert(OUT != kOutNvfp4 || HALVES == 2, "NVFP4 output is a SwiGLU epilogue");
+  static_assert(OUT != kOutPartial || HALVES == 1, "partial output: plain projection of the stored columns");
   constexpr int SLOT = slot_floats<MPAD, HALVES>();
   // Let the next kernel in the stream launch now: its CTAs take SMs as the
   // stream-K CTAs leave and prefetch their weights into L2 meanwhile.  All
@@ -212,7 +214,18 @@ __global__ void __launch_bounds__(FIX_THREADS) decode_fixup_kernel(const Params 
   const float a1[4] = {acc[HALVES - 1].x, acc[HALVES - 1].y, acc[HALVES - 1].z, acc[HALVES - 1].w};
   const float sq[4] = {ss.x, ss.y, ss.z, ss.w};
   const int col = tile * 128 + n;
-  const float gs = FP4 ? __ldg(p.gscale) : 0.f;
+  if constexpr (OUT == kOutPartial) {
+    // the summed fp32 accumulators and sums of squares, not post-scaled
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = 4 * q + i;
+      if (m >= p.M) break;
+      p.part_out[static_cast<int64_t>(m) * p.ncols + col] = a0[i];
+      if (tile == 0 && n == 0) p.part_out[static_cast<int64_t>(p.M) * p.ncols + m] = sq[i];
+    }
+    return;
+  }
+  const float gs = OUT == kOutNvfp4 ? __ldg(p.gscale) : 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int m = 4 * q + i;
@@ -220,7 +233,7 @@ __global__ void __launch_bounds__(FIX_THREADS) decode_fixup_kernel(const Params 
     const float r = inv_rms(sq[i], p.inv_d, p.eps);
     float v = a0[i] * r;
     if (HALVES == 2) v = silu_f32(v) * (a1[i] * r);
-    if constexpr (FP4) {
+    if constexpr (OUT == kOutNvfp4) {
       // NVFP4 output (SwiGLU: every tile column is an output column)
       uint32_t pair;
       const uint32_t sf = fp4_quantize_lane16(v, gs, pair);
@@ -246,11 +259,11 @@ inline bool any_split_tile(int grid, long long total, int kblocks) {
 }
 
 // Launch the fix-up for the stream-K grid described by `p`.
-template <int MPAD, int HALVES, bool FP4 = false>
+template <int MPAD, int HALVES, int OUT = kOutBf16>
 cudaError_t launch_fixup(const Params& p, cudaStream_t stream) {
   const long long threads = static_cast<long long>(p.tiles) * 128 * ((p.M + 3) / 4);
   const unsigned fgrid = static_cast<unsigned>((threads + FIX_THREADS - 1) / FIX_THREADS);
-  return launch_pdl(decode_fixup_kernel<MPAD, HALVES, FP4>, fgrid, FIX_THREADS, 0, stream, p);
+  return launch_pdl(decode_fixup_kernel<MPAD, HALVES, OUT>, fgrid, FIX_THREADS, 0, stream, p);
 }
 
 // Workspace needed by a decode call: the header and two partial slots per CTA

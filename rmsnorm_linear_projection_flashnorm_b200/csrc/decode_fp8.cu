@@ -229,12 +229,13 @@ __global__ void __launch_bounds__(256) xsplit_kernel(const Params p) {
   }
 }
 
-// FP4: write the SwiGLU output in NVFP4 (yq, ysf) instead of bf16 y.
-template <int MPAD, int HALVES, bool PRESPLIT, bool FP4 = false>
+// OUT: bf16 y, NVFP4 codes and scales (SwiGLU only), or fp32 partials (OutKind).
+template <int MPAD, int HALVES, bool PRESPLIT, int OUT = kOutBf16>
 __global__ void __launch_bounds__(Cfg<MPAD, HALVES, PRESPLIT>::THREADS, 1)
     decode_fp8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_q, const Params p) {
-  static_assert(!FP4 || HALVES == 2, "NVFP4 output is a SwiGLU epilogue");
+  static_assert(OUT != kOutNvfp4 || HALVES == 2, "NVFP4 output is a SwiGLU epilogue");
+  static_assert(OUT != kOutPartial || HALVES == 1, "partial output: plain projection of the stored columns");
   using C = Cfg<MPAD, HALVES, PRESPLIT>;
   constexpr int STAGES = C::STAGES;
   using B = Bars<MPAD, STAGES>;
@@ -534,8 +535,18 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES, PRESPLIT>::THREADS, 1)
       if (!all_ok) break;
       const bool whole = (kb0 == 0 && kb1 == p.kblocks);
       uint8_t* qbuf = reinterpret_cast<uint8_t*>(bars.ybuf);   // NVFP4 staging
-      if (whole) {
-        const float gs = FP4 ? __ldg(p.gscale) : 0.f;
+      if (whole && OUT == kOutPartial) {
+        // the tile's fp32 accumulators and (tile 0) the sums of squares, not post-scaled
+#pragma unroll
+        for (int j = 0; j < RPS; ++j) {
+          const int m = m0 + j;
+          if (m >= p.M) break;
+          p.part_out[static_cast<int64_t>(m) * p.ncols + tile * 128 + n] =
+              (j & 1) ? f2_hi(acc[0][j / 2]) : f2_lo(acc[0][j / 2]);
+        }
+        if (tile == 0 && st < p.M) p.part_out[static_cast<int64_t>(p.M) * p.ncols + st] = bars.ssq[b][st];
+      } else if (whole) {
+        const float gs = OUT == kOutNvfp4 ? __ldg(p.gscale) : 0.f;
 #pragma unroll
         for (int j = 0; j < RPS; ++j) {
           const int m = m0 + j;
@@ -544,7 +555,7 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES, PRESPLIT>::THREADS, 1)
           const float a0 = (j & 1) ? f2_hi(acc[0][j / 2]) : f2_lo(acc[0][j / 2]);
           float v = a0 * r;
           if (HALVES == 2) v = silu_f32(v) * (((j & 1) ? f2_hi(acc[1][j / 2]) : f2_lo(acc[1][j / 2])) * r);
-          if constexpr (FP4) dec::stage_fp4(qbuf, MPAD, m, n, v, gs);
+          if constexpr (OUT == kOutNvfp4) dec::stage_fp4(qbuf, MPAD, m, n, v, gs);
           else bars.ybuf[m * 128 + n] = __float2bfloat16_rn(v);
         }
       } else {
@@ -568,8 +579,8 @@ __global__ void __launch_bounds__(Cfg<MPAD, HALVES, PRESPLIT>::THREADS, 1)
       named_bar_sync(1, C::SCALE_THREADS);   // sums of squares read, staging complete
       if (st == 0) mbar_arrive(&bars.ssq_empty[b]);
       if (whole) {
-        if constexpr (FP4) dec::store_tile_fp4(qbuf, MPAD, p, tile, st, C::SCALE_THREADS);
-        else dec::store_tile_rows(bars.ybuf, p, tile, st, C::SCALE_THREADS);
+        if constexpr (OUT == kOutNvfp4) dec::store_tile_fp4(qbuf, MPAD, p, tile, st, C::SCALE_THREADS);
+        else if constexpr (OUT == kOutBf16) dec::store_tile_rows(bars.ybuf, p, tile, st, C::SCALE_THREADS);
       }
     }
   }
@@ -598,7 +609,7 @@ static_assert(Cfg<16, 1>::TMEM_COLS == 64 && Cfg<64, 2>::TMEM_COLS == 512, "TMEM
 template <int MPAD>
 constexpr bool presplit() { return MPAD >= 32; }
 
-template <int MPAD, int HALVES, bool FP4 = false>
+template <int MPAD, int HALVES, int OUT = kOutBf16>
 cudaError_t launch_impl(const CallArgs& a) {
   constexpr bool PRE = presplit<MPAD>();
   using C = Cfg<MPAD, HALVES, PRE>;
@@ -637,6 +648,7 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.yq = static_cast<uint8_t*>(a.yq);
   p.ysf = static_cast<uint8_t*>(a.ysf);
   p.gscale = a.gscale;
+  p.part_out = a.part_out;
   tq = tw;   // unused unless x is split once per call
   if (PRE) {
     // after the partial slots: x_hi / x_lo slabs, then the scale factors
@@ -647,17 +659,17 @@ cudaError_t launch_impl(const CallArgs& a) {
       return cudaErrorInvalidValue;
   }
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES, PRE>();
-  cudaError_t e = ensure_smem_limit<decode_fp8_kernel<MPAD, HALVES, PRE, FP4>>(static_cast<int>(SMEM));
+  cudaError_t e = ensure_smem_limit<decode_fp8_kernel<MPAD, HALVES, PRE, OUT>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
   if (PRE) {
     const int warps = p.kblocks * MPAD;
     e = launch_pdl(xsplit_kernel<MPAD>, static_cast<unsigned>((warps + 7) / 8), 256, 0, a.stream, p);
     if (e != cudaSuccess) return e;
   }
-  e = launch_pdl(decode_fp8_kernel<MPAD, HALVES, PRE, FP4>, p.grid, C::THREADS, SMEM, a.stream, tx, tw, tq, p);
+  e = launch_pdl(decode_fp8_kernel<MPAD, HALVES, PRE, OUT>, p.grid, C::THREADS, SMEM, a.stream, tx, tw, tq, p);
   if (e != cudaSuccess) return e;
   if (!dec::any_split_tile(p.grid, p.total, p.kblocks)) return cudaSuccess;
-  return dec::launch_fixup<MPAD, HALVES, FP4>(p, a.stream);
+  return dec::launch_fixup<MPAD, HALVES, OUT>(p, a.stream);
 }
 
 }  // namespace dec8
@@ -670,10 +682,15 @@ size_t decode_fp8_presplit_bytes(int64_t M, int64_t d) {
 }
 
 cudaError_t launch_decode_fp8(const CallArgs& a, int mpad) {
+  if (a.part_out) {   // partial output: a plain projection of the stored columns
+    if (mpad == 16) return dec8::launch_impl<16, 1, kOutPartial>(a);
+    if (mpad == 32) return dec8::launch_impl<32, 1, kOutPartial>(a);
+    return dec8::launch_impl<64, 1, kOutPartial>(a);
+  }
   if (a.yq) {   // NVFP4 output (SwiGLU only)
-    if (mpad == 16) return dec8::launch_impl<16, 2, true>(a);
-    if (mpad == 32) return dec8::launch_impl<32, 2, true>(a);
-    return dec8::launch_impl<64, 2, true>(a);
+    if (mpad == 16) return dec8::launch_impl<16, 2, kOutNvfp4>(a);
+    if (mpad == 32) return dec8::launch_impl<32, 2, kOutNvfp4>(a);
+    return dec8::launch_impl<64, 2, kOutNvfp4>(a);
   }
   if (mpad == 16) return a.swiglu ? dec8::launch_impl<16, 2>(a) : dec8::launch_impl<16, 1>(a);
   if (mpad == 32) return a.swiglu ? dec8::launch_impl<32, 2>(a) : dec8::launch_impl<32, 1>(a);

@@ -17,6 +17,11 @@ constexpr size_t kWsHeaderBytes = 256;
 // workspace (bf16) instead of converting every weight tile once per row tile.
 constexpr int64_t kFp8DequantOnceM = 1024;
 
+// What a fused call writes: bf16 y; NVFP4 codes and scale bytes (SwiGLU
+// only); or, for one rank of a row-parallel split of d, the fp32 accumulators
+// and sums of squares before the post-scale.
+enum OutKind : int { kOutBf16 = 0, kOutNvfp4 = 1, kOutPartial = 2 };
+
 // One fused norm+projection call, validated by the ABI layer.
 struct CallArgs {
   const void* x;          // bf16 [M, d]
@@ -32,6 +37,7 @@ struct CallArgs {
   void* yq;               // NVFP4 output, SwiGLU only: e2m1 codes [M, N/2] bytes, or null
   void* ysf;              //   e4m3 scale codes [M, N/16]
   const float* gscale;    //   global scale, one fp32 value in device memory
+  float* part_out;        // kOutPartial: fp32 [M, ncols] accumulators, then [M] sums of squares
   void* ws;               // workspace (status word + decode scratch)
   size_t ws_bytes;
   cudaStream_t stream;
@@ -73,6 +79,9 @@ cudaError_t launch_fold_fp8(const void* W0, const void* W1, const float* g, int6
                             float* scales, cudaStream_t s);
 cudaError_t launch_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, float eps, void* h,
                            cudaStream_t s);
+// Row-parallel split of d: the post-scale after the partials were summed (post_scale.cu).
+cudaError_t launch_post_scale(const float* part, int64_t M, int64_t N, bool swiglu, int64_t d_total, float eps,
+                              void* y, cudaStream_t s);
 cudaError_t launch_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t ncols, void* W,
                                cudaStream_t s);
 

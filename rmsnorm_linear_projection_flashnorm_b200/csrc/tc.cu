@@ -69,6 +69,7 @@ struct Params {
   uint8_t* yq;           // NVFP4 output (SwiGLU only; y is null then): codes [M][nout / 2]
   uint8_t* ysf;          //   and e4m3 scale codes [M][nout / 16]
   const float* gscale;   //   global scale (one fp32 value in device memory)
+  float* part_out;       // partial output: fp32 [M][ncols] accumulators, then [M] sums of squares
 };
 
 template <int STAGES>
@@ -108,12 +109,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
   }
 }
 
-// FP4: write the SwiGLU output in NVFP4 (yq, ysf) instead of bf16 y.
-template <bool SWIGLU, bool FP8, bool FP4 = false>
+// OUT: bf16 y, NVFP4 codes and scales (SwiGLU only), or fp32 partials (OutKind).
+template <bool SWIGLU, bool FP8, int OUT = kOutBf16>
 __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
               const Params p) {
-  static_assert(!FP4 || SWIGLU, "NVFP4 output is a SwiGLU epilogue");
+  static_assert(OUT != kOutNvfp4 || SWIGLU, "NVFP4 output is a SwiGLU epilogue");
   constexpr int STAGES = Cfg<FP8>::STAGES;
   constexpr int STAGE_BYTES = Cfg<FP8>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
@@ -304,12 +305,31 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
       ok = ok && mbar_wait(&bars.ssq_full[b], aph, ctl, kSiteEpiSsqFull);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const float r = inv_rms(bars.ssq[b][row], p.inv_d, p.eps);
+      const float ssq_row = bars.ssq[b][row];
+      const float r = inv_rms(ssq_row, p.inv_d, p.eps);
       mbar_arrive(&bars.ssq_empty[b]);
       const int grow = mb * BM + row;
       const bool row_ok = grow < p.M;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
-      if constexpr (FP4) {
+      if constexpr (OUT == kOutPartial) {
+        // One rank of a row-parallel split of d: the fp32 accumulators of the
+        // stored columns and the row's sum of squares, before any post-scale.
+        float* prow = p.part_out + static_cast<int64_t>(grow) * p.ncols + nb * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_ld_wait();
+          if (row_ok && nb * BN + c < p.ncols) {
+            float4* dst = reinterpret_cast<float4*>(prow + c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          }
+        }
+        if (row_ok && nb == 0) p.part_out[static_cast<int64_t>(p.M) * p.ncols + grow] = ssq_row;
+      } else if constexpr (OUT == kOutNvfp4) {
         // NVFP4 output: this thread's row holds whole 16-column blocks
         const float gs = __ldg(p.gscale);
         uint8_t* qrow = p.yq + static_cast<int64_t>(grow) * (p.nout / 2) + nb * (BN / 4);
@@ -393,7 +413,7 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
   }
 }
 
-template <bool SWIGLU, bool FP8, bool FP4 = false>
+template <bool SWIGLU, bool FP8, int OUT = kOutBf16>
 cudaError_t launch_impl(const CallArgs& a) {
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, BM, BK)) return cudaErrorInvalidValue;
@@ -422,17 +442,21 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.yq = static_cast<uint8_t*>(a.yq);
   p.ysf = static_cast<uint8_t*>(a.ysf);
   p.gscale = a.gscale;
+  p.part_out = a.part_out;
   constexpr size_t SMEM_BYTES = smem_bytes<FP8>();
-  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU, FP8, FP4>>(static_cast<int>(SMEM_BYTES));
+  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU, FP8, OUT>>(static_cast<int>(SMEM_BYTES));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
-  return launch_pdl(tc_kernel<SWIGLU, FP8, FP4>, grid, Cfg<FP8>::NUM_THREADS, SMEM_BYTES, a.stream, tx, tw, p);
+  return launch_pdl(tc_kernel<SWIGLU, FP8, OUT>, grid, Cfg<FP8>::NUM_THREADS, SMEM_BYTES, a.stream, tx, tw, p);
 }
 
 }  // namespace tc
 
 cudaError_t launch_tc(const CallArgs& a) {
-  if (a.yq) return a.wtype == 1 ? tc::launch_impl<true, true, true>(a) : tc::launch_impl<true, false, true>(a);
+  if (a.yq) return a.wtype == 1 ? tc::launch_impl<true, true, kOutNvfp4>(a) : tc::launch_impl<true, false, kOutNvfp4>(a);
+  // partial output: no activation, so every weight is a plain projection of its stored columns
+  if (a.part_out)
+    return a.wtype == 1 ? tc::launch_impl<false, true, kOutPartial>(a) : tc::launch_impl<false, false, kOutPartial>(a);
   if (a.wtype == 1) return a.swiglu ? tc::launch_impl<true, true>(a) : tc::launch_impl<false, true>(a);
   return a.swiglu ? tc::launch_impl<true, false>(a) : tc::launch_impl<false, false>(a);
 }

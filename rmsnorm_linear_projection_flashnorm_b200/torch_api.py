@@ -8,7 +8,8 @@ from typing import Optional, Tuple
 import torch
 
 from . import (FN_W_BF16, FN_W_FP8_E4M3_B128, check, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
-               fn_norm_proj_swiglu_nvfp4, fn_query_device_status, fn_workspace_size)
+               fn_norm_proj_partial, fn_norm_proj_swiglu_nvfp4, fn_post_scale, fn_query_device_status,
+               fn_workspace_size)
 
 
 def fold(W0: torch.Tensor, g: torch.Tensor, W1: Optional[torch.Tensor] = None, wtype: int = FN_W_BF16,
@@ -78,3 +79,28 @@ def norm_proj_swiglu_nvfp4(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float
     check(fn_norm_proj_swiglu_nvfp4(x, M, d, Wp, scales, wt, N, eps, global_scale, q, sf, buf, buf.numel(), stream),
           "fn_norm_proj_swiglu_nvfp4")
     return q, sf
+
+
+def norm_proj_partial(x: torch.Tensor, Wp: torch.Tensor, ncols: int, scales: Optional[torch.Tensor] = None,
+                      ws: Optional[Workspace] = None, out: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """One rank's share of a row-parallel projection: fp32 [M * ncols + M]
+    (unscaled x @ Wp in stored column order, then the rows' sums of squares)."""
+    M, d = x.shape
+    wt = FN_W_BF16 if Wp.dtype == torch.bfloat16 else FN_W_FP8_E4M3_B128
+    if ws is None:
+        ws = Workspace(x.device)
+    buf = ws.get(M, d, ncols, wt, False)
+    if out is None:
+        out = torch.empty(M * ncols + M, dtype=torch.float32, device=x.device)
+    check(fn_norm_proj_partial(x, M, d, Wp, scales, wt, ncols, out, buf, buf.numel(), stream), "fn_norm_proj_partial")
+    return out
+
+
+def post_scale(partial: torch.Tensor, M: int, N: int, d_total: int, eps: float, swiglu: bool = False,
+               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bf16 [M, N] from a summed partial buffer (see fn_post_scale)."""
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=partial.device)
+    check(fn_post_scale(partial, M, N, int(swiglu), d_total, eps, out, stream), "fn_post_scale")
+    return out

@@ -164,3 +164,50 @@ def test_no_device_means_no_launch(L):
         pytest.skip("a GPU is present")
     st = np_()
     assert st in (fnb.FN_ERR_CUDA, fnb.FN_ERR_UNSUPPORTED_DEVICE)
+
+
+P = 1 << 40           # partial buffer
+
+
+def partial_(x=A, M=4, d=256, Wp=B, scales=None, wt=0, ncols=512, part=P, ws=WS, ws_bytes=1 << 30):
+    return fnb.fn_norm_proj_partial(x, M, d, Wp, scales, wt, ncols, part, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(M=-1), fnb.FN_ERR_INVALID_ARG),
+    (dict(part=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(x=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(ncols=500), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(d=96), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(wt=1, d=192, scales=A + (1 << 18)), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(part=P + 8), fnb.FN_ERR_ALIGNMENT),
+    (dict(part=A + 512), fnb.FN_ERR_ALIAS),      # overlaps x
+    (dict(part=WS + 1024), fnb.FN_ERR_ALIAS),    # inside the workspace
+    (dict(ws=P + 4096), fnb.FN_ERR_ALIAS),       # partial is (4*512 + 4) floats
+])
+def test_partial_rejects_bad_arguments(L, kw, code):
+    assert partial_(**kw) == code
+
+
+def post_(part=P, M=4, N=256, swiglu=0, d_total=1024, eps=1e-6, y=C):
+    return fnb.fn_post_scale(part, M, N, swiglu, d_total, eps, y, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(M=-1), fnb.FN_ERR_INVALID_ARG),
+    (dict(d_total=0), fnb.FN_ERR_INVALID_ARG),
+    (dict(eps=-1.0), fnb.FN_ERR_INVALID_ARG),
+    (dict(N=200), fnb.FN_ERR_UNSUPPORTED_SHAPE),
+    (dict(part=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(y=None), fnb.FN_ERR_INVALID_ARG),
+    (dict(y=C + 4), fnb.FN_ERR_ALIGNMENT),
+    (dict(y=P + 1024), fnb.FN_ERR_ALIAS),
+    (dict(swiglu=1, y=P + 8192), fnb.FN_ERR_ALIAS),   # SwiGLU partial: 4 x 512 + 4 floats
+])
+def test_post_scale_rejects_bad_arguments(L, kw, code):
+    assert post_(**kw) == code
+
+
+def test_partial_and_post_scale_empty_batch(L):
+    assert partial_(M=0, x=None, part=None, ws=None) == fnb.FN_OK
+    assert post_(M=0, part=None, y=None) == fnb.FN_OK
