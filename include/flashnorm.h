@@ -185,7 +185,8 @@ fn_status fn_norm_proj_partial(const void* x, int64_t M, int64_t d, const void* 
  *   r[m] = 1/sqrt(ssq[m] / d_total + eps), d_total the full input width;
  *   y = r * acc (plain), or silu(r * gate) * (r * up) for swiglu != 0, with
  *   the gate and up columns read from the interleaved stored order;
- *   one round to bf16 into y [M, N], 16-byte aligned, not overlapping partial.
+ *   one round to bf16 into y [M, N], 16-byte aligned, not overlapping partial;
+ *   M * N < 2^42 (one thread per 8 outputs), else FN_ERR_UNSUPPORTED_SHAPE.
  * With one rank (d_total = d) the result equals fn_norm_proj on the same
  * inputs up to the rounding order of the sums: bit for bit for M > 64 (every
  * column tile reduces a row's sum of squares in the same k order), while for

@@ -299,6 +299,7 @@ fn_status fn_post_scale(const float* partial, int64_t M, int64_t N, int swiglu, 
   if (N % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
   const int64_t ncols = swiglu ? 2 * N : N;
   if (M > kMaxDim || ncols > kMaxDim || d_total > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (M * (N / 8) / 256 > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;   // one thread per 8 outputs, 256 per block
   if (M == 0) return FN_OK;
   if (!partial || !y) return FN_ERR_INVALID_ARG;
   if (!aligned16(partial) || !aligned16(y)) return FN_ERR_ALIGNMENT;

@@ -211,3 +211,8 @@ def test_post_scale_rejects_bad_arguments(L, kw, code):
 def test_partial_and_post_scale_empty_batch(L):
     assert partial_(M=0, x=None, part=None, ws=None) == fnb.FN_OK
     assert post_(M=0, part=None, y=None) == fnb.FN_OK
+
+
+def test_post_scale_rejects_a_grid_too_large(L):
+    # (2^31 - 1) rows x 2^21 columns: more than 2^31 blocks of 256 threads
+    assert post_(M=(1 << 31) - 1, N=1 << 21) == fnb.FN_ERR_UNSUPPORTED_SHAPE
