@@ -646,7 +646,9 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": job_ms / K, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if wl.wtype == "bf16" else "bf16 (e4m3 weights)",
+            "vs_baseline": None,
+            "dtype": ("bf16" if wl.wtype == "bf16" else "bf16 (e4m3 weights)")
+                     + (", NVFP4 output" if args.out == "nvfp4" else ""),
             "data": "synthetic (seeded workloads recipe; random-init weights)",
             "config": {"workload": wl.name, "M": Ms, "d": wl.d, "N": wl.N, "swiglu": wl.swiglu, "output": args.out,
                        "weights": wl.wtype, "parallelism": f"replicas x{world} (rows shard, no collective)",
