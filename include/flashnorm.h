@@ -13,6 +13,10 @@
  *     matmul and the reduction.
  * SwiGLU epilogue: the fused FC1 + SwiGLU of the FlashInfer PR #5521 analysis
  * ("Register-level SwiGLU" design item): out = silu(gate) * up.
+ * Further forms of the same call: the SwiGLU output quantised to NVFP4 in the
+ * epilogue (FlashInfer PR #4040 analysis), and a row-parallel split of d for
+ * tensor parallelism (per-rank partial products and sums of squares, one
+ * all-reduce, a post-scale), which Proposal 2 makes a single exchange.
  *
  * Definitions (the pages print no formula; these are the plain readings):
  *   r[m]  = 1 / sqrt( (1/d) sum_k x[m,k]^2 + eps )
