@@ -14,7 +14,7 @@ exchange is one ``torch.distributed.all_reduce`` (NCCL on GPUs).
 """
 from __future__ import annotations
 
-from typing import Callable, List, Optional, Tuple
+from typing import List, Optional, Tuple
 
 import torch
 import torch.distributed as dist
@@ -39,24 +39,17 @@ def rowparallel_slices(d: int, world: int, align: int = 64) -> List[Tuple[int, i
 
 
 def row_parallel_norm_proj(x_local: torch.Tensor, Wp_local: torch.Tensor, N: int, eps: float, d_total: int,
-                           swiglu: bool = False, scales: Optional[torch.Tensor] = None, group=None, ws=None,
-                           partial_fn: Optional[Callable] = None,
-                           post_fn: Optional[Callable] = None) -> torch.Tensor:
+                           swiglu: bool = False, scales: Optional[torch.Tensor] = None, group=None,
+                           ws=None) -> torch.Tensor:
     """y [M, N] (bf16) of RMSNorm(x) @ W with d split across the ranks of
     `group`: this rank passes its columns x_local [M, d_local] and its rows of
     the folded weight (and of the fp8 block scales).  Every rank returns the
-    full y.  `partial_fn` / `post_fn` replace the two library calls (tests
-    drive the exchange on CPU ranks with them)."""
+    full y."""
     from . import torch_api as T
     M = x_local.shape[0]
     ncols = 2 * N if swiglu else N
-    if partial_fn is None:
-        part = T.norm_proj_partial(x_local, Wp_local, ncols, scales=scales, ws=ws)
-    else:
-        part = partial_fn(x_local, Wp_local, ncols)
+    part = T.norm_proj_partial(x_local, Wp_local, ncols, scales=scales, ws=ws)
     world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
     if world > 1:
         dist.all_reduce(part, op=dist.ReduceOp.SUM, group=group)
-    if post_fn is None:
-        return T.post_scale(part, M, N, d_total, eps, swiglu=swiglu)
-    return post_fn(part, M, N, d_total, eps, swiglu)
+    return T.post_scale(part, M, N, d_total, eps, swiglu=swiglu)

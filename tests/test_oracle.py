@@ -16,26 +16,17 @@ import pytest
 import torch
 
 import oracle as O
+from tests._golden import read_golden
 import workloads as WL
 
 
 # ---------------------------------------------------------------------------
 # number formats
 # ---------------------------------------------------------------------------
-def _read_golden(path):
-    rows = []
-    with open(path) as f:
-        for line in f:
-            line = line.strip()
-            if not line or line.startswith("#"):
-                continue
-            parts = line.split()
-            rows.append((float(parts[0]), int(parts[1], 16)))
-    return rows
 
 
 def test_e4m3_golden_points(golden_dir):
-    rows = _read_golden(os.path.join(golden_dir, "e4m3_points.txt"))
+    rows = read_golden(os.path.join(golden_dir, "e4m3_points.txt"))
     vals = np.array([v for v, _ in rows])
     want = np.array([c for _, c in rows], dtype=np.uint8)
     got = O.e4m3_encode(vals)
@@ -43,7 +34,7 @@ def test_e4m3_golden_points(golden_dir):
 
 
 def test_bf16_golden_points(golden_dir):
-    rows = _read_golden(os.path.join(golden_dir, "bf16_points.txt"))
+    rows = read_golden(os.path.join(golden_dir, "bf16_points.txt"))
     vals = np.array([v for v, _ in rows])
     want = np.array([c for _, c in rows], dtype=np.uint16)
     got = O.bf16_bits(vals)

@@ -17,6 +17,7 @@ import pytest
 import torch
 
 import oracle as O
+from tests._golden import read_golden
 import oracle.flashnorm_oracle as OF
 
 # The eight e2m1 magnitudes in code order (OCP Microscaling formats
@@ -24,20 +25,10 @@ import oracle.flashnorm_oracle as OF
 E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
 
 
-def _read_golden(path):
-    rows = []
-    with open(path) as f:
-        for line in f:
-            line = line.strip()
-            if not line or line.startswith("#"):
-                continue
-            parts = line.split()
-            rows.append((float(parts[0]), int(parts[1], 16)))
-    return rows
 
 
 def test_e2m1_golden_points(golden_dir):
-    rows = _read_golden(os.path.join(golden_dir, "e2m1_points.txt"))
+    rows = read_golden(os.path.join(golden_dir, "e2m1_points.txt"))
     vals = np.array([v for v, _ in rows])
     want = np.array([c for _, c in rows], dtype=np.uint8)
     got = O.e2m1_encode(vals)

@@ -4,7 +4,8 @@
 Each rank takes its slice of the input width from ``rowparallel_slices``,
 computes its share, and ``row_parallel_norm_proj`` sums the shares with one
 all-reduce and post-scales.  On CPU ranks the two library calls are replaced
-by the oracle's statement of them, so what is checked here is the plumbing:
+(patched in each worker) by the oracle's statement of them, so what is
+checked here is the plumbing:
 slicing, the buffer layout ([M, ncols] products then [M] sums of squares),
 the collective, and that every rank ends with the single-device result.
 """
@@ -41,24 +42,26 @@ def _worker(rank, world, port, swiglu, q):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     sys.path.insert(0, ROOT)
     import oracle as O
+    from rmsnorm_linear_projection_flashnorm_b200 import torch_api as T
     from rmsnorm_linear_projection_flashnorm_b200 import tp
     M, d, N = 4, 384, 256
     x, Wg, Wu = _inputs(M, d, N, swiglu)
     W = O.interleave128(Wg, Wu) if swiglu else Wg
     k0, k1 = tp.rowparallel_slices(d, world, align=64)[rank]
 
-    def partial_fn(xl, Wl, ncols):
+    def partial_cpu(xl, Wl, ncols, scales=None, ws=None):
         acc, ssq = O.rowparallel_partial(xl.numpy(), Wl.numpy())
         assert acc.shape == (M, ncols)
         return torch.from_numpy(np.concatenate([acc.reshape(-1), ssq]))
 
-    def post_fn(part, M_, N_, d_total, eps, sw):
+    def post_cpu(part, M_, N_, d_total, eps, swiglu=False):
         p = part.numpy()
-        ncols = 2 * N_ if sw else N_
-        return O.rowparallel_finish(p[:M_ * ncols].reshape(M_, ncols), p[M_ * ncols:], d_total, eps, sw)
+        ncols = 2 * N_ if swiglu else N_
+        return O.rowparallel_finish(p[:M_ * ncols].reshape(M_, ncols), p[M_ * ncols:], d_total, eps, swiglu)
 
+    T.norm_proj_partial, T.post_scale = partial_cpu, post_cpu   # this worker process only
     y = tp.row_parallel_norm_proj(torch.from_numpy(x[:, k0:k1].copy()), torch.from_numpy(W[k0:k1].copy()), N, 1e-6,
-                                  d, swiglu=swiglu, partial_fn=partial_fn, post_fn=post_fn)
+                                  d, swiglu=swiglu)
     q.put((rank, (k0, k1), y))
     dist.destroy_process_group()
 
