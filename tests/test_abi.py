@@ -216,3 +216,23 @@ def test_partial_and_post_scale_empty_batch(L):
 def test_post_scale_rejects_a_grid_too_large(L):
     # (2^31 - 1) rows x 2^21 columns: more than 2^31 blocks of 256 threads
     assert post_(M=(1 << 31) - 1, N=1 << 21) == fnb.FN_ERR_UNSUPPORTED_SHAPE
+
+
+def test_abi_is_usable_from_plain_c(L, tmp_path):
+    """Compile a C11 program against the header with gcc (no C++, no CUDA
+    headers), link it to the library, and run it: the declarations are valid
+    C, every symbol links, and argument errors come back as status codes."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(fnb.LIB_PATH)
+    exe = str(tmp_path / "abi_from_c")
+    src = os.path.join(ROOT, "tests", "c", "abi_from_c.c")
+    r = subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), src, "-o", exe,
+                        "-L", lib_dir, "-lflashnorm", f"-Wl,-rpath,{lib_dir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")   # validation only: no device is touched
+    r = subprocess.run([exe], capture_output=True, text=True, env=env, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
