@@ -236,3 +236,36 @@ def test_abi_is_usable_from_plain_c(L, tmp_path):
     env = dict(os.environ, CUDA_VISIBLE_DEVICES="")   # validation only: no device is touched
     r = subprocess.run([exe], capture_output=True, text=True, env=env, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
+
+
+def test_validation_never_crashes_and_returns_a_status(L):
+    """Random argument combinations (sizes, alignments, overlaps, null
+    pointers) on a host without a GPU: every call returns one of the declared
+    status codes, and with no device none can succeed (M > 0).  Skipped where
+    a GPU is visible: random addresses must never reach a launch."""
+    import torch
+    from hypothesis import given, settings, strategies as st
+    if torch.cuda.is_available():
+        pytest.skip("random device addresses are only safe without a GPU")
+
+    codes = {fnb.FN_OK, fnb.FN_ERR_INVALID_ARG, fnb.FN_ERR_UNSUPPORTED_SHAPE, fnb.FN_ERR_ALIGNMENT,
+             fnb.FN_ERR_ALIAS, fnb.FN_ERR_WORKSPACE, fnb.FN_ERR_CUDA, fnb.FN_ERR_UNSUPPORTED_DEVICE}
+    ptr = st.one_of(st.none(), st.integers(1, 1 << 44))
+    size = st.integers(-2, 1 << 33)
+
+    @settings(max_examples=300, deadline=None, database=None)
+    @given(M=size, d=size, N=size, wt=st.integers(-1, 2), eps=st.floats(allow_nan=True, allow_infinity=True),
+           x=ptr, w=ptr, y=ptr, ws=ptr, ws_bytes=st.integers(0, 1 << 34), swiglu=st.booleans(),
+           fp4=st.booleans(), part=st.booleans())
+    def run(M, d, N, wt, eps, x, w, y, ws, ws_bytes, swiglu, fp4, part):
+        if fp4:
+            st_ = fnb.fn_norm_proj_swiglu_nvfp4(x, M, d, w, None, wt, N, eps, ws, y, x, ws, ws_bytes, None)
+        elif part:
+            st_ = fnb.fn_norm_proj_partial(x, M, d, w, None, wt, N, y, ws, ws_bytes, None)
+        else:
+            f = fnb.fn_norm_proj_swiglu if swiglu else fnb.fn_norm_proj
+            st_ = f(x, M, d, w, None, wt, N, eps, y, ws, ws_bytes, None)
+        assert st_ in codes
+        assert st_ != fnb.FN_OK or M == 0
+
+    run()
