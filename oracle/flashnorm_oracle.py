@@ -65,6 +65,7 @@ __all__ = [
     "E2M1", "E2M1_MAX", "NVFP4_BLOCK", "e2m1_round", "e2m1_encode", "e2m1_decode",
     "nvfp4_quantize", "nvfp4_pack", "nvfp4_unpack", "nvfp4_dequantize",
     "rowparallel_partial", "rowparallel_finish",
+    "MX_BLOCK", "fold_mxfp8", "dequant_mxfp8",
 ]
 
 FP8_BLOCK = 128
@@ -411,3 +412,40 @@ def rowparallel_finish(acc, ssq, d_total: int, eps: float, swiglu: bool = False)
         return acc * r[:, None]
     gate, up = deinterleave128(acc)
     return silu(gate * r[:, None]) * (up * r[:, None])
+
+
+# ---------------------------------------------------------------------------
+# MXFP8 weights: e4m3 codes with one power-of-two (ue8m0) scale per 32 k values
+# ---------------------------------------------------------------------------
+MX_BLOCK = 32
+
+
+def fold_mxfp8(W, g) -> Tuple[np.ndarray, np.ndarray]:
+    """Folded weight P = fp32(g[k]) * fp32(W[k,n]) in the block-scaled form the
+    tensor cores' kind::mxf8f6f4 MMAs read: per column n and block b of 32
+    consecutive k, a shared exponent E (stored as the ue8m0 byte E + 127) with
+        E = ceil(log2(amax_b / 448))      the smallest power of two that keeps
+                                          every |P| / 2^E <= 448 (no saturation)
+        q = RN_e4m3(P / 2^E)              (exact division by a power of two)
+    An all-zero block stores E = -127 (byte 0) and zero codes.  Reading: the
+    OCP MX rule floor(log2 amax) - 8 lets a block maximum land in [448, 512)
+    and clamps it; the round-up rule loses no accuracy against the 128x128
+    fp32-scaled format (the format study in the tests), so it is used here.
+    Returns codes [d, N] and scale bytes [d/32, N]."""
+    P = _gain_product_f32(W, g).astype(np.float64)
+    d, N = P.shape
+    assert d % MX_BLOCK == 0
+    Pb = P.reshape(d // MX_BLOCK, MX_BLOCK, N)
+    amax = np.max(np.abs(Pb), axis=1)                                   # [d/32, N]
+    _, ex = np.frexp(np.where(amax > 0, amax / E4M3_MAX, 1.0))          # amax/448 = m * 2^ex, m in [0.5, 1)
+    m = np.ldexp(np.where(amax > 0, amax / E4M3_MAX, 1.0), -ex)
+    E = np.where(m == 0.5, ex - 1, ex)                                  # ceil(log2(amax/448))
+    E = np.where(amax > 0, np.clip(E, -127, 127), -127).astype(np.int64)
+    q = e4m3_encode(Pb / np.ldexp(1.0, E)[:, None, :])
+    return q.reshape(d, N), (E + 127).astype(np.uint8)
+
+
+def dequant_mxfp8(q: np.ndarray, sbytes: np.ndarray) -> np.ndarray:
+    """float64 e4m3(q[k,n]) * 2^(s[k/32, n] - 127) (exact in fp64)."""
+    scale = np.ldexp(1.0, np.asarray(sbytes, dtype=np.int64) - 127)
+    return e4m3_decode(q) * np.repeat(scale, MX_BLOCK, axis=0)
