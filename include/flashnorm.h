@@ -208,21 +208,35 @@ fn_status fn_post_scale(const float* partial, int64_t M, int64_t N, int swiglu, 
  * because it can synchronise the device.  The pages have no counterpart of
  * this entry point; it only moves the scratch memory.
  *   Arguments, layout and results as fn_norm_proj, minus the workspace.  The
- *   call's scratch (status word and split-K partials) lives in a fixed
- *   8 MiB array inside the library that every GPU loading the library holds
- *   until the process exits.  Sizes whose scratch exceeds it (as computed by
- *   fn_workspace_size) are rejected with FN_ERR_WORKSPACE before any launch:
- *   on a 148-SM B200 every shape with M <= 32 or M > 64 fits, and M in 33..64
- *   fits only while the split-K partials stay under 8 MiB.
- *   The first call on a device fetches the array's device address and zeroes
- *   its status word (a synchronous set-up step): make that first call before
- *   any stream capture.  All calls on a device share the array and it keeps
- *   the last call's contents; calls that may overlap on the GPU race on it.
- *   Device-side wait timeouts are recorded in the array, not reported.  The
- *   call allocates nothing.
+ *   call's scratch (status word, split-K partials, and for fp8 weights at
+ *   17..64 rows the activations split once per call) lives in a fixed 8 MiB
+ *   array inside the library that every GPU loading the library holds until
+ *   the process exits.  A shape is served exactly when
+ *   fn_workspace_size(M, d, N, wt, 0) <= 8 MiB; larger ones are rejected with
+ *   FN_ERR_WORKSPACE before any launch.  On a 148-SM B200 that admits bf16
+ *   weights at every M > 64 and at M <= 32, M in 33..64 while the split-K
+ *   partials stay under 8 MiB, and fp8 weights at M <= 64 and 65..1023 under
+ *   the same rule; fp8 weights at M >= 1024 need a bf16 copy of the weight
+ *   (2 d N bytes) in the scratch and are rejected for any weight over 4 Mi
+ *   elements.
+ *   The array is zero when the library loads, so no set-up copy is made; the
+ *   first call on a device only fetches the array's device address (a host
+ *   query): make that first call before any stream capture.  All calls on a
+ *   device share the array and it keeps the last call's contents; calls that
+ *   may overlap on the GPU race on it.  A device-side wait that ran out of
+ *   time is recorded in the array's status word: fn_query_static_status
+ *   reports and clears it.  The call allocates nothing.
  */
 fn_status fn_norm_proj_static(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
                               fn_wtype wt, int64_t N, float eps, void* y, fn_stream_t stream);
+
+/*
+ * fn_query_static_status — fn_query_device_status for the scratch array of
+ * fn_norm_proj_static on the current device: synchronises `stream`, reads and
+ * clears the status word.  Returns FN_OK or FN_ERR_TIMEOUT; *detail (if not
+ * NULL) receives the raw word.  Allocates nothing.
+ */
+fn_status fn_query_static_status(unsigned int* detail, fn_stream_t stream);
 
 /*
  * fn_query_device_status — synchronises `stream`, reads and clears the status

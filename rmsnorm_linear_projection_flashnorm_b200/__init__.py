@@ -48,6 +48,7 @@ _SIGNATURES = {
     "fn_post_scale": (_int, [_vp, _i64, _i64, _int, _i64, _f32, _vp, _vp]),
     "fn_norm_proj_static": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp]),
     "fn_query_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_uint), _vp]),
+    "fn_query_static_status": (_int, [ctypes.POINTER(ctypes.c_uint), _vp]),
     "fn_rmsnorm": (_int, [_vp, _i64, _i64, _vp, _f32, _vp, _vp]),
     "fn_dequant_fp8": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "fn_status_string": (ctypes.c_char_p, [_int]),
@@ -167,6 +168,14 @@ def fn_query_device_status(workspace, stream=None):
     """Returns (status, raw status word)."""
     word = ctypes.c_uint(0)
     st = lib().fn_query_device_status(_ptr(workspace), ctypes.byref(word), _stream(stream))
+    return st, word.value
+
+
+def fn_query_static_status(stream=None):
+    """Status of fn_norm_proj_static's scratch on the current device:
+    (status, raw status word); the word is cleared."""
+    word = ctypes.c_uint(0)
+    st = lib().fn_query_static_status(ctypes.byref(word), _stream(stream))
     return st, word.value
 
 

@@ -7,19 +7,23 @@
 // owns every device allocation, and latency-critical loops that must never
 // call cudaMalloc because it can synchronise the device.  For them the
 // scratch memory of the call (the status word and the per-CTA split-K
-// partial sums of the decode path) lives in a fixed-size array inside this
-// library instead of a caller-provided workspace.
+// partial sums of the decode path, the activations split once per call of the
+// fp8 decode path) lives in a fixed-size array inside this library instead of
+// a caller-provided workspace.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the
-// library holds kStaticScratchBytes of it until the process exits.  In host
-// code its name is only a host-side stand-in, so its device address is
+// library holds kStaticScratchBytes of it until the process exits.  Global
+// device variables without an initialiser are zero when the module loads, so
+// the status word starts at zero without any set-up copy.  In host code the
+// array's name is only a host-side stand-in, so its device address is
 // fetched with cudaGetSymbolAddress once per device, with that device
-// current, on the first call made on that device; that first call also zeroes
-// the status word.  That first call must therefore come before any stream
-// capture.  All calls on a device share the array and it keeps the last
-// call's contents (every call overwrites the partials it reads, so nothing
-// else has to start at zero); calls that may overlap on the GPU, on any
-// streams, race on it.
+// current, on the first call made on that device; that first call must
+// therefore come before any stream capture.  All calls on a device share the
+// array and it keeps the last call's contents (every call overwrites the
+// partials it reads, so nothing else has to start at zero); calls that may
+// overlap on the GPU, on any streams, race on it.  A device-side wait that
+// runs out of time records itself in the array's status word, which
+// fn_query_static_status reads and clears.
 #include <cstdint>
 #include <mutex>
 
@@ -38,7 +42,8 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (set-up on first use).
+// Device address of the scratch array on the current device (fetched on
+// first use; no memory is allocated or written).
 fn_status static_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -49,10 +54,6 @@ fn_status static_scratch(void** out) {
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return FN_ERR_CUDA;
-    }
-    if (cudaMemset(p, 0, fn::kWsHeaderBytes) != cudaSuccess) {   // the status word starts at zero
       cudaGetLastError();
       return FN_ERR_CUDA;
     }
@@ -76,4 +77,11 @@ extern "C" fn_status fn_norm_proj_static(const void* x, int64_t M, int64_t d, co
     if (st != FN_OK) return st;
   }
   return fn_norm_proj(x, M, d, Wp, scales, wt, N, eps, y, scratch, kStaticScratchBytes, stream);
+}
+
+extern "C" fn_status fn_query_static_status(unsigned int* detail, fn_stream_t stream) {
+  void* scratch = nullptr;
+  const fn_status st = static_scratch(&scratch);
+  if (st != FN_OK) return st;
+  return fn_query_device_status(scratch, detail, stream);
 }
