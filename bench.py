@@ -208,18 +208,31 @@ def profile_traffic(profile_name: str, src_hash: str):
 
 
 class Setup:
-    def __init__(self, wl: WL.Workload, Ms, device, out: str = "bf16"):
+    """Operands of one workload on the device: folded weight copies (rotated so
+    that consecutive calls never find their weight in L2), activations for each
+    M, outputs, the workspace.  gen="host" draws the inputs with the seeded
+    host recipe (and keeps pinned host copies for the end-to-end timing);
+    gen="device" draws the same distributions on the device (large prefill
+    shapes, where host generation would dominate the run)."""
+
+    def __init__(self, wl: WL.Workload, Ms, device, out: str = "bf16", gen: str = "host"):
         import rmsnorm_linear_projection_flashnorm_b200 as fnb
         from rmsnorm_linear_projection_flashnorm_b200 import torch_api as T
         self.fnb, self.T = fnb, T
         self.wl, self.Ms, self.dev = wl, list(Ms), device
         d, N, sw = wl.d, wl.N, wl.swiglu
         self.wtype = fnb.FN_W_BF16 if wl.wtype == "bf16" else fnb.FN_W_FP8_E4M3_B128
-        g = WL.gain(d, wl.seed).to(device)
-        if sw:
-            W0, W1 = (w.to(device) for w in WL.weights(d, N, wl.seed, halves=2))
+        Mmax = max(self.Ms)
+        if gen == "device":
+            x_all, g, W = WL.device_inputs(wl, Mmax, device)
+            W0, W1 = (W if sw else (W, None))
         else:
-            W0, W1 = WL.weights(d, N, wl.seed).to(device), None
+            g = WL.gain(d, wl.seed).to(device)
+            if sw:
+                W0, W1 = (w.to(device) for w in WL.weights(d, N, wl.seed, halves=2))
+            else:
+                W0, W1 = WL.weights(d, N, wl.seed).to(device), None
+            x_all = WL.activations(Mmax, d, wl.seed, wl.outliers)
         Wp, scales = T.fold(W0, g, W1, wtype=self.wtype)
         wp_bytes = Wp.numel() * Wp.element_size()
         self.copies = max(2, math.ceil(2 * L2_BYTES / wp_bytes) + 1)
@@ -230,22 +243,26 @@ class Setup:
         self.g = g
         self._W_src = (W0, W1)
         self.W_unf = None
-        Mmax = max(self.Ms)
-        x_all = WL.activations(Mmax, d, wl.seed, wl.outliers)
-        self.x_host = {M: x_all[:M].contiguous().pin_memory() for M in self.Ms}
-        self.x = {M: self.x_host[M].to(device) for M in self.Ms}
+        if gen == "device":
+            self.x_host = None
+            self.x = {M: x_all[:M].contiguous() for M in self.Ms}
+        else:
+            self.x_host = {M: x_all[:M].contiguous().pin_memory() for M in self.Ms}
+            self.x = {M: self.x_host[M].to(device) for M in self.Ms}
         self.out = out
         if out == "nvfp4":
             # codes [M, N/2] and scale bytes [M, N/16], copied to one host buffer
             # per M; a fixed global scale (its value does not change the work)
             self.y = {M: torch.empty((M, N // 2 + N // 16), dtype=torch.uint8, device=device) for M in self.Ms}
-            self.y_host = {M: torch.empty((M, N // 2 + N // 16), dtype=torch.uint8).pin_memory() for M in self.Ms}
+            self.y_host = {M: torch.empty((M, N // 2 + N // 16), dtype=torch.uint8).pin_memory() for M in self.Ms} \
+                if gen == "host" else None
             self.yq = {M: torch.empty((M, N // 2), dtype=torch.uint8, device=device) for M in self.Ms}
             self.ysf = {M: torch.empty((M, N // 16), dtype=torch.uint8, device=device) for M in self.Ms}
             self.gscale = torch.tensor([448.0 * 6.0 / 8.0], dtype=torch.float32, device=device)
         else:
             self.y = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in self.Ms}
-            self.y_host = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in self.Ms}
+            self.y_host = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in self.Ms} \
+                if gen == "host" else None
         self.ws = T.Workspace(device)
         for M in self.Ms:
             self.ws.get(M, d, N, self.wtype, sw)
@@ -412,17 +429,127 @@ def _stage(msg: str) -> None:
         print(f"[bench] {msg}", file=sys.stderr, flush=True)
 
 
+def roofline_entry(units_per_call: float, us_per_call: float, hbm_bound: bool, peaks, peaks_kind, clocks_summary,
+                   kernel: str, traffic):
+    """Roofline record of one call: algorithmic bytes (decode) or flops (prefill)
+    of a call over its in-stream duration, against the measured peak.  A
+    tensor-bound run that saw the power cap (or ran well below the maximum SM
+    clock) is compared with the sustained GEMM peak, otherwise with the burst
+    peak."""
+    if hbm_bound:
+        peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+        achieved = units_per_call / (us_per_call / 1e6) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic, "kernel": kernel, "peak_source": f"hbm_gbs ({peaks_kind})",
+                "bytes_per_launch": units_per_call, "avg_launch_us": us_per_call}
+    ck = clocks_summary
+    capped = "sw_power_cap" in ck.get("reasons", []) or bool(
+        ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] < 0.9 * ck["sm_max_mhz"])
+    burst = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    peak = sustained if capped else burst
+    achieved = units_per_call / (us_per_call / 1e6) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic, "kernel": kernel,
+            "peak_source": f"bf16_tflops{'_sustained' if capped else ''} ({peaks_kind})",
+            "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
+            "flops_per_launch": units_per_call, "avg_launch_us": us_per_call}
+
+
+def kernel_for(wl: WL.Workload, M: int, out: str):
+    """Name of the dominant kernel of a call, its sources and its ncu summary file."""
+    if M <= 64:
+        kname = "decode_kernel" if wl.wtype == "bf16" else "decode_fp8_kernel"
+        sources = ["decode.cu" if wl.wtype == "bf16" else "decode_fp8.cu", "decode_common.cuh", "ptx.cuh",
+                   "nvfp4.cuh"]
+        label = f"{kname} (+ decode_fixup_kernel where a tile's k range is split)"
+    else:
+        kname, sources = "tc_kernel", ["tc.cu", "ptx.cuh", "nvfp4.cuh"]
+        label = "tc_kernel" + (" (after the dequantise-once kernel)" if wl.wtype != "bf16" and M >= 1024 else "")
+    src_hash = kernel_source_hash(sources)
+    prof = f"{kname}_{wl.name}{'_nvfp4' if out == 'nvfp4' else ''}.md"
+    return kname, label, src_hash, profile_traffic(prof, src_hash)
+
+
+# Same-run records for the rest of the metric: the prefill half (tensor-bound
+# shapes) and the other decode workloads, each with its own roofline, clocks
+# and unfused chain.
+SUB_RECORDS = (
+    ("ffn_swiglu", 4096), ("prefill_swiglu_large", 16384), ("fp8_swiglu", 8192), ("fp8_swiglu", 256),
+    ("ffn_swiglu", 16), ("fp8_swiglu", 1), ("fp8_swiglu", 64),
+)
+
+
+def run_sub_record(name: str, M: int, dev, peaks, peaks_kind, world: int, target_s: float = 0.25):
+    """One call shape timed on its own: direct calls on the launching stream
+    (inputs drawn on the device; weights rotated over copies that together
+    exceed twice the L2), CUDA events around n calls, NVML clocks during them,
+    then the unfused chain over the same rotation."""
+    wl = WL.WORKLOADS[name]
+    S = Setup(wl, [M], dev, "bf16", gen="device")
+    stream = torch.cuda.current_stream()
+    wbyte = 2 if wl.wtype == "bf16" else 1
+    by, fl = algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte)
+    if wl.wtype != "bf16":
+        by += (wl.d // 128) * (wl.ncols // 128) * 4       # fp32 block scales
+    hbm_bound = M <= 64
+
+    def timed(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / n * 1e3          # us per call
+
+    for _ in range(3):
+        S.call(M)
+    est = timed(lambda: S.call(M), 3)
+    n = int(min(2000, max(10, math.ceil(target_s / (est * 1e-6)))))
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        us = timed(lambda: S.call(M), n)
+    units, ms = aggregate((by if hbm_bound else fl) * n, us * n / 1e3, world, dev)
+    ck = clocks.summary()
+    _, label, src_hash, traffic = kernel_for(wl, M, "bf16")
+    rec = {"workload": name, "M": M, "d": wl.d, "N": wl.N, "swiglu": wl.swiglu, "weights": wl.wtype,
+           "calls": n, "us_per_call": ms * 1e3 / n,
+           "value": units / (ms / 1e3) / (1e9 if hbm_bound else 1e12), "unit": "GB/s" if hbm_bound else "TFLOP/s",
+           "roofline": roofline_entry(by if hbm_bound else fl, ms * 1e3 / n, hbm_bound, peaks, peaks_kind, ck,
+                                      label, traffic),
+           "clocks": ck, "l2": f"{S.copies} rotating W' copies", "kernel_source_sha256": src_hash}
+    for _ in range(2):
+        S.chain(M)
+    n_c = int(min(n, max(5, math.ceil(target_s / (timed(lambda: S.chain(M), 2) * 1e-6)))))
+    with ClockSampler(dev.index if dev.index is not None else 0) as cclk:
+        chain_us = timed(lambda: S.chain(M), n_c)
+    chain_us = max_over_ranks(chain_us, world, dev)
+    rec["unfused_chain"] = {"us_per_call": chain_us, "fused_speedup": chain_us / rec["us_per_call"],
+                            "clocks": cclk.summary(),
+                            "what": ("fn_dequant_fp8 (e4m3 W' -> bf16) -> fn_rmsnorm (no gain) -> torch.matmul "
+                                     "(cuBLAS)" if wl.wtype != "bf16" else
+                                     "fn_rmsnorm -> torch.matmul (cuBLAS) with unfolded W")
+                                    + (" -> silu(gate)*up" if wl.swiglu else "")}
+    del S
+    torch.cuda.empty_cache()
+    return rec
+
+
 def main():
     faulthandler.enable()
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="fused", choices=["fused", "reference"])
     ap.add_argument("--workload", default="decode_qkv", choices=list(WL.WORKLOAD_ORDER))
     ap.add_argument("--m", type=int, default=0, help="run a single batch size of the workload")
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU oracle baseline")
     ap.add_argument("--skip-chain", action="store_true", help="omit the unfused-chain baseline")
+    ap.add_argument("--sub", default="all", choices=["all", "none"],
+                    help="same-run records of the prefill and other decode shapes")
     ap.add_argument("--out", default="bf16", choices=["bf16", "nvfp4"],
                     help="output format; nvfp4 (SwiGLU workloads) runs the quantising epilogue")
     args = ap.parse_args()
@@ -465,64 +592,46 @@ def main():
     torch.cuda.synchronize()
     _stage("warm-up done")
 
-    # Timed region: K steps, each replaying a CUDA graph of one step (the way a
-    # decode loop issues work).  Graph p holds calls p*len(Ms) .. of the
-    # weight-copy rotation, so consecutive calls always read different copies.
-    # Event records between kernels would break the programmatic launch
-    # overlap between consecutive calls, so the graphs that carry the per-call
-    # event pairs are separate copies, replayed in every 8th step of the timed
-    # region; they give the calls' own durations on the launching stream.
+    # Timed region: K steps, each a replay of a CUDA graph of G steps (the way a
+    # decode loop issues many layers' projections per graph), so consecutive
+    # calls overlap through programmatic dependent launch exactly as they do in
+    # such a loop.  Graph p holds calls p*G*len(Ms) .. of the weight-copy
+    # rotation, so consecutive calls always read different copies.  The
+    # per-call time is the timed region over the calls it holds: in-stream,
+    # kernel boundaries included, and consistent with ms_per_step.
     K = args.steps
     n_calls = len(Ms)
-    # G steps per graph (at least 16 calls, as a decode loop captures many
-    # layers per graph); a tail of K mod G steps uses one-step graphs.
     G = max(1, min(K, math.ceil(16 / n_calls)))
     per_graph = G * n_calls
     n_graphs = S.copies // math.gcd(per_graph, S.copies)
-    n_graphs = n_graphs * max(1, math.ceil(8 / n_graphs))
     cap_stream = torch.cuda.Stream()
 
-    def capture(start_call, steps, with_events):
+    def capture(start_call, steps, Ms_):
         S.i = start_call % S.copies
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * steps * n_calls)] \
-            if with_events else []
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=cap_stream):
-            for st in range(steps):
-                for j, M in enumerate(Ms):
-                    if with_events:
-                        evs[2 * (st * n_calls + j)].record()
+            for _ in range(steps):
+                for M in Ms_:
                     S.call(M)
-                    if with_events:
-                        evs[2 * (st * n_calls + j) + 1].record()
-        return gr, evs
+        return gr
 
     launches0 = fnb.fn_kernel_launches()
-    clean = [capture(gi * per_graph, G, False)[0] for gi in range(n_graphs)]
+    graphs = [capture(gi * per_graph, G, Ms) for gi in range(n_graphs)]
     kernels_per_step = (fnb.fn_kernel_launches() - launches0) // (n_graphs * G)
-    timed = [capture(gi * per_graph, G, True) for gi in range(n_graphs)]
-    tail = [capture(j * n_calls, 1, False)[0] for j in range(K % G)]
-    _stage(f"{2 * n_graphs} graphs of {G} steps captured, {kernels_per_step} kernels per step")
+    tail = [capture(j * n_calls, 1, Ms) for j in range(K % G)]
+    _stage(f"{n_graphs} graphs of {G} steps captured, {kernels_per_step} kernels per step")
     for gi in range(max(args.warmup, n_graphs)):
-        clean[gi % n_graphs].replay()
-        timed[gi % n_graphs][0].replay()
+        graphs[gi % n_graphs].replay()
     for gr in tail:
         gr.replay()
     torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    instrumented = set()
-    n_full = K // G
     with ClockSampler(local) as clocks:
         t_start.record(stream)
-        for k in range(n_full):
-            gi = k % n_graphs
-            if k % 8 == 7:
-                timed[gi][0].replay()
-                instrumented.add(gi)
-            else:
-                clean[gi].replay()
+        for k in range(K // G):
+            graphs[k % n_graphs].replay()
         for gr in tail:
             gr.replay()
         t_end.record(stream)
@@ -533,59 +642,38 @@ def main():
     job_units, job_ms = aggregate(float(bytes_per_step if hbm_bound else flops_per_step) * K, elapsed_ms,
                                   world, dev)
     gpu_launches = K * kernels_per_step
-    # per-call durations: the last replay of each instrumented graph in the timed region
-    kernel_ms, kernel_n = 0.0, 0
-    if not instrumented:   # too few steps for an instrumented replay inside the timed region
-        for gi in range(n_graphs):
-            timed[gi][0].replay()
-            instrumented.add(gi)
-        torch.cuda.synchronize()
-    for gi in sorted(instrumented):
-        evs = timed[gi][1]
-        for c in range(G * n_calls):
-            kernel_ms += evs[2 * c].elapsed_time(evs[2 * c + 1])
-            kernel_n += 1
+    us_per_call = max_over_ranks(elapsed_ms, world, dev) / (K * n_calls) * 1e3
+    kname, label, src_hash, traffic = kernel_for(wl, max(Ms), args.out)
+    ck = clocks.summary()
+    units_per_call = (bytes_per_step if hbm_bound else flops_per_step) / n_calls
+    roofline = roofline_entry(units_per_call, us_per_call, hbm_bound, peaks, peaks_kind, ck,
+                              f"{label}: one fn_norm_proj call, averaged over M={Ms}", traffic)
+    roofline["timing"] = "timed region / calls (in-stream, graph replays, kernel boundaries included)"
+    value = job_units / (job_ms / 1e3) / (1e9 if hbm_bound else 1e12)
+    unit = "GB/s" if hbm_bound else "TFLOP/s"
 
-    value_bytes = job_units / (job_ms / 1e3) if hbm_bound else 0.0
-    value_flops = job_units / (job_ms / 1e3) if not hbm_bound else 0.0
-    kernel_avg_ms = kernel_ms / max(kernel_n, 1)
-    per_launch_bytes = bytes_per_step / len(Ms)
-    per_launch_flops = flops_per_step / len(Ms)
-    if hbm_bound:
-        kname = "decode_kernel" if wl.wtype == "bf16" else "decode_fp8_kernel"
-        sources = ["decode.cu" if wl.wtype == "bf16" else "decode_fp8.cu", "decode_common.cuh", "ptx.cuh",
-                   "nvfp4.cuh"]
-    else:
-        kname, sources = "tc_kernel", ["tc.cu", "ptx.cuh", "nvfp4.cuh"]
-    src_hash = kernel_source_hash(sources)
-    traffic = profile_traffic(f"{kname}_{wl.name}{'_nvfp4' if args.out == 'nvfp4' else ''}.md", src_hash)
-    if hbm_bound:
-        peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
-        achieved = per_launch_bytes / (kernel_avg_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": traffic, "kernel": f"{kname} (+ decode_fixup_kernel): one fn_norm_proj call",
-                    "peak_source": f"hbm_gbs ({peaks_kind})",
-                    "bytes_per_launch": per_launch_bytes, "avg_launch_us": kernel_avg_ms * 1e3,
-                    "stream_us_per_call": job_ms / K / n_calls * 1e3,
-                    "frac_stream": per_launch_bytes / (job_ms / K / n_calls / 1e3) / 1e9 / peak}
-        value, unit = value_bytes / 1e9, "GB/s"
-    else:
-        # burst peak for a kernel that ran at full clock, sustained when the
-        # timed region was power-capped or clocked down
-        ck = clocks.summary()
-        capped = "sw_power_cap" in ck.get("reasons", []) or (
-            ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] < 0.9 * ck["sm_max_mhz"])
-        burst = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
-        sustained = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
-        peak = sustained if capped else burst
-        achieved = per_launch_flops / (kernel_avg_ms / 1e3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": traffic, "kernel": "tc_kernel: one fn_norm_proj call",
-                    "peak_source": f"bf16_tflops{'_sustained' if capped else ''} ({peaks_kind})",
-                    "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
-                    "flops_per_launch": per_launch_flops, "avg_launch_us": kernel_avg_ms * 1e3,
-                    "stream_us_per_call": job_ms / K / n_calls * 1e3}
-        value, unit = value_flops / 1e12, "TFLOP/s"
+    # the same timing per batch size (one M per graph), for the breakdown
+    per_m = None
+    if len(Ms) > 1:
+        per_m = {}
+        reps = max(1, min(K // G, 50))
+        for M in Ms:
+            gs = [capture(gi * 16, 1, [M] * 16) for gi in range(max(1, S.copies // math.gcd(16, S.copies)))]
+            for gr in gs:
+                gr.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for r in range(reps):
+                gs[r % len(gs)].replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            us_m = max_over_ranks(e0.elapsed_time(e1), world, dev) / (reps * 16) * 1e3
+            by_m = algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte, args.out)[0]
+            per_m[str(M)] = {"us_per_call": us_m, "GB/s": by_m / (us_m / 1e6) / 1e9,
+                             "frac": by_m / (us_m / 1e6) / 1e9 / roofline["peak"]} if hbm_bound else \
+                {"us_per_call": us_m}
+            del gs
 
     # end to end through the public API: pinned host x -> device -> call -> host y
     e2e_steps = max(1, min(K, 2000))
@@ -630,14 +718,25 @@ def main():
                 S.chain(M)
         c1.record(stream)
         torch.cuda.synchronize()
-        chain_ms = c0.elapsed_time(c1) / c_steps
-        chain = {"ms_per_step": chain_ms, "fused_speedup": chain_ms / (elapsed_ms / K),
+        chain_ms = max_over_ranks(c0.elapsed_time(c1) / c_steps, world, dev)
+        chain = {"ms_per_step": chain_ms, "fused_speedup": chain_ms / (job_ms / K),
                  "what": ("fn_dequant_fp8 kernel (e4m3 W' -> bf16) -> fn_rmsnorm kernel (no gain) -> "
                           "torch.matmul (cuBLAS)" if wl.wtype != "bf16" else
                           "fn_rmsnorm kernel -> torch.matmul (cuBLAS) with unfolded W")
                          + (" -> silu(gate)*up" if wl.swiglu else "")}
-
     _stage("chain done")
+    l2_desc = (f"{S.copies} rotating W' copies "
+               f"({S.copies * S.Wp[0].numel() * S.Wp[0].element_size() / 1e6:.0f} MB > L2)")
+    del S, xs
+    torch.cuda.empty_cache()
+
+    subs = None
+    if args.sub == "all" and not args.m and args.workload == "decode_qkv" and args.out == "bf16":
+        subs = {}
+        for name, M in SUB_RECORDS:
+            _stage(f"sub-record {name} M={M}")
+            subs[f"{name}_M{M}"] = run_sub_record(name, M, dev, peaks, peaks_kind, world)
+
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         cpu = run_cpu_baseline(wl, Ms)
@@ -652,14 +751,12 @@ def main():
             "data": "synthetic (seeded workloads recipe; random-init weights)",
             "config": {"workload": wl.name, "M": Ms, "d": wl.d, "N": wl.N, "swiglu": wl.swiglu, "output": args.out,
                        "weights": wl.wtype, "parallelism": f"replicas x{world} (rows shard, no collective)",
-                       "l2": f"{S.copies} rotating W' copies ({S.copies * S.Wp[0].numel() * S.Wp[0].element_size() / 1e6:.0f} MB > L2)",
+                       "l2": l2_desc,
                        "step": f"{len(Ms)} fused calls, one per M; CUDA graphs of {G} steps",
-                       "kernel_timing": "event pairs around each call in the instrumented graphs "
-                                        "(every 8th step of the timed region)",
                        "kernels_per_step": kernels_per_step},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks.summary(),
+            "roofline": roofline, "per_m": per_m, "cpu_baseline": cpu, "e2e": e2e, "clocks": ck,
             "gpu_launches": gpu_launches, "unfused_chain": chain,
-            "kernel_source_sha256": src_hash,
+            "kernel_source_sha256": src_hash, "sub_records": subs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -164,3 +164,29 @@ def sample_rows(M: int, seed: int, per_tile: int = 2, tile: int = 128) -> np.nda
     s = row_scales(M, seed)
     rows.extend([int(np.argmin(s)), int(np.argmax(s))])
     return np.unique(np.asarray(rows, dtype=np.int64))
+
+
+def device_inputs(w: Workload, M: int, device, seed_offset: int = 0):
+    """The same distributions as the host recipe above, drawn on the device with
+    torch's generator (seeded), for benchmark workloads whose host generation
+    would take longer than the measurement: returns x [M, d] bf16, g [d] fp32
+    (bf16-representable), and W [d, N] bf16 (or the pair W_gate, W_up).  The
+    values differ from the host recipe's; only shapes and distributions match."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1_000_003 * (w.seed + 1) + seed_offset)
+    d, N = w.d, w.N
+    g = (1.0 + 0.1 * torch.randn(d, generator=gen, device=device)).to(torch.bfloat16).to(torch.float32)
+    std = 1.0 / math.sqrt(d)
+    Ws = tuple((torch.randn((d, N), generator=gen, device=device) * std).to(torch.bfloat16)
+               for _ in range(2 if w.swiglu else 1))
+    u = torch.rand((M, 1), generator=gen, device=device, dtype=torch.float64)
+    scale = torch.exp(math.log(0.1) + u * (math.log(10.0) - math.log(0.1))).to(torch.float32)
+    colmul = torch.ones((1, d), dtype=torch.float32, device=device)
+    if w.outliers:
+        colmul[0, torch.randperm(d, generator=gen, device=device)[: d // 100]] = 20.0
+    x = torch.empty((M, d), dtype=torch.bfloat16, device=device)
+    step = max(1, (1 << 26) // d)
+    for r0 in range(0, M, step):
+        r1 = min(M, r0 + step)
+        x[r0:r1] = (torch.randn((r1 - r0, d), generator=gen, device=device) * scale[r0:r1] * colmul).to(torch.bfloat16)
+    return x, g, (Ws[0] if len(Ws) == 1 else Ws)
