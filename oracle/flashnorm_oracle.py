@@ -66,6 +66,7 @@ __all__ = [
     "nvfp4_quantize", "nvfp4_pack", "nvfp4_unpack", "nvfp4_dequantize",
     "rowparallel_partial", "rowparallel_finish",
     "MX_BLOCK", "fold_mxfp8", "dequant_mxfp8",
+    "sf_chunk_layout", "sf_chunk_unlayout", "fold_mxfp8_stored",
 ]
 
 FP8_BLOCK = 128
@@ -449,3 +450,48 @@ def dequant_mxfp8(q: np.ndarray, sbytes: np.ndarray) -> np.ndarray:
     """float64 e4m3(q[k,n]) * 2^(s[k/32, n] - 127) (exact in fp64)."""
     scale = np.ldexp(1.0, np.asarray(sbytes, dtype=np.int64) - 127)
     return e4m3_decode(q) * np.repeat(scale, MX_BLOCK, axis=0)
+
+
+# ---------------------------------------------------------------------------
+# Scale bytes in the chunked layout that block-scaled tensor-core MMAs read
+# ---------------------------------------------------------------------------
+def sf_chunk_layout(S) -> np.ndarray:
+    """Scale bytes S [R, C] (R rows along the M or N side of a block-scaled
+    MMA, C scale columns along its K side) in the chunked layout the tensor
+    cores read: the matrix is cut into chunks of 128 rows x 4 scale columns
+    (512 bytes each, rows padded to a multiple of 128 and columns to a
+    multiple of 4 with zero bytes), chunk (rb, cg) stored at byte
+    512 * (rb * ceil(C/4) + cg), and inside a chunk the byte of row r, column c
+    sits at 16 * (r mod 32) + 4 * ((r mod 128) div 32) + (c mod 4): 32
+    sixteen-byte lines, line i holding rows i, i+32, i+64, i+96 of the chunk.
+    This is the layout the FlashInfer PR #4040 analysis calls swizzled scale
+    factors (is_swizzled), which a block-scaled GEMM consumes directly.
+    Returns a flat uint8 array."""
+    S = np.asarray(S, dtype=np.uint8)
+    R, C = S.shape
+    Rp, Cp = -(-R // 128) * 128, -(-C // 4) * 4
+    r, c = np.indices((R, C))
+    dest = 512 * ((r // 128) * (Cp // 4) + c // 4) + 16 * (r % 32) + 4 * ((r % 128) // 32) + (c % 4)
+    out = np.zeros(Rp * Cp, dtype=np.uint8)
+    out[dest.ravel()] = S.ravel()
+    return out
+
+
+def sf_chunk_unlayout(flat, R: int, C: int) -> np.ndarray:
+    """Inverse of sf_chunk_layout: the [R, C] scale bytes back from the flat
+    chunked array."""
+    flat = np.asarray(flat, dtype=np.uint8)
+    Cp = -(-C // 4) * 4
+    r, c = np.indices((R, C))
+    src = 512 * ((r // 128) * (Cp // 4) + c // 4) + 16 * (r % 32) + 4 * ((r % 128) // 32) + (c % 4)
+    return flat[src]
+
+
+def fold_mxfp8_stored(W, g) -> Tuple[np.ndarray, np.ndarray]:
+    """The MXFP8 fold as the library stores it: the e4m3 codes [d, N] of
+    fold_mxfp8, and its scale bytes [d/32, N] transposed to the weight's MMA
+    orientation (rows = output columns n, scale columns = 32-deep k blocks)
+    and laid out by sf_chunk_layout: one 512-byte chunk per 128 output
+    columns and 128 k rows, the k groups of a column block consecutive."""
+    q, sb = fold_mxfp8(W, g)
+    return q, sf_chunk_layout(sb.T)

@@ -6,6 +6,8 @@ exponent, the defining property of the round-up exponent rule, closed forms
 and the format's rounding bound.  The kernel for this format is not built
 yet; the oracle comes first.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -83,3 +85,78 @@ def test_exact_blocks_round_trip(k):
     q, s = O.fold_mxfp8(W, np.ones(64))
     assert np.all(s == k + 127)
     assert np.array_equal(O.dequant_mxfp8(q, s), W)
+
+
+# ---------------------------------------------------------------------------
+# the chunked scale layout (block-scaled tensor-core MMAs; NVFP4 swizzled scales)
+# ---------------------------------------------------------------------------
+def _golden_positions(golden_dir):
+    rows = []
+    with open(os.path.join(golden_dir, "sf_chunk_points.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                r, c, off = line.split()[:3]
+                rows.append((int(r), int(c), int(off)))
+    return rows
+
+
+def test_sf_chunk_golden_positions(golden_dir):
+    S = np.zeros((256, 8), dtype=np.uint8)
+    pts = _golden_positions(golden_dir)
+    for i, (r, c, _) in enumerate(pts):
+        S[r, c] = i + 1
+    flat = O.sf_chunk_layout(S)
+    assert flat.size == 256 * 8
+    for i, (_, _, off) in enumerate(pts):
+        assert flat[off] == i + 1, (pts[i], int(np.argmax(flat == i + 1)))
+
+
+def test_sf_chunk_reshape_form():
+    """The same layout written as a reshape and a transposition: rows split
+    into (block, group of 32, lane), columns into (chunk, slot); the chunk
+    is [lane][group][slot]."""
+    rng = np.random.default_rng(3)
+    R, C = 384, 12
+    S = rng.integers(0, 256, (R, C)).astype(np.uint8)
+    t = S.reshape(R // 128, 4, 32, C // 4, 4)             # [block][group][lane][chunk][slot]
+    want = t.transpose(0, 3, 2, 1, 4).reshape(-1)         # [block][chunk][lane][group][slot]
+    assert np.array_equal(O.sf_chunk_layout(S), want)
+
+
+def test_sf_chunk_padding_and_inverse():
+    rng = np.random.default_rng(4)
+    R, C = 200, 6                                          # ragged: padded to 256 x 8
+    S = rng.integers(1, 256, (R, C)).astype(np.uint8)
+    flat = O.sf_chunk_layout(S)
+    assert flat.size == 256 * 8
+    assert np.count_nonzero(flat) == R * C                 # padding bytes are zero
+    assert np.array_equal(O.sf_chunk_unlayout(flat, R, C), S)
+    assert sorted(flat[flat > 0].tolist()) == sorted(S.ravel().tolist())
+
+
+def test_sf_chunk_planted_mistake_is_caught(golden_dir, monkeypatch):
+    """A layout with the lane and row-group roles swapped fails the golden positions."""
+    def wrong(S):
+        S = np.asarray(S, dtype=np.uint8)
+        R, C = S.shape
+        r, c = np.indices((R, C))
+        dest = 512 * ((r // 128) * (C // 4) + c // 4) + 4 * (r % 32) + 128 * ((r % 128) // 32) + (c % 4)
+        out = np.zeros(R * C, dtype=np.uint8)
+        out[dest.ravel()] = S.ravel()
+        return out
+    monkeypatch.setattr(O, "sf_chunk_layout", wrong)
+    with pytest.raises(AssertionError):
+        test_sf_chunk_golden_positions(golden_dir)
+
+
+def test_stored_mxfp8_fold_is_the_fold_in_chunks():
+    inp = WL.case(4, 256, 384, False, seed=22)
+    q, sb = O.fold_mxfp8(inp["W"], inp["g"])
+    q2, flat = O.fold_mxfp8_stored(inp["W"], inp["g"])
+    assert np.array_equal(q, q2)
+    # column n, k block j of the stored scales: chunk (n div 128, j div 4)
+    for n in (0, 31, 32, 127, 128, 300, 383):
+        for j in (0, 3, 4, 7):
+            off = 512 * ((n // 128) * 2 + j // 4) + 16 * (n % 32) + 4 * ((n % 128) // 32) + j % 4
+            assert flat[off] == sb[j, n]
