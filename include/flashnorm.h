@@ -64,8 +64,27 @@ typedef enum {
 
 typedef enum {
   FN_W_BF16 = 0,            /* W' stored as bf16 [d, ncols] */
-  FN_W_FP8_E4M3_B128 = 1    /* W' stored as e4m3 [d, ncols] + fp32 scales [d/128, ncols/128] */
+  FN_W_FP8_E4M3_B128 = 1,   /* W' stored as e4m3 [d, ncols] + fp32 scales [d/128, ncols/128] */
+  FN_W_MXFP8_E4M3 = 2       /* W' stored as e4m3 [d, ncols] + ue8m0 scale bytes, one per 32 k values
+                               of each column, in the chunked layout below */
 } fn_wtype;
+
+/*
+ * MXFP8 weights (FN_W_MXFP8_E4M3): the block-scaled format the tensor cores'
+ * kind::mxf8f6f4 MMAs read (the FlashInfer PR #5521 analysis, design item 4,
+ * runs its low-precision FC1 on the block-scaled MMA family).  Per stored
+ * column n and block j of 32 consecutive k (rows 32j .. 32j+31) a shared
+ * exponent E = ceil(log2(amax / 448)), the smallest E with amax <= 448 * 2^E
+ * (clamped to [-127, 127]; -127 for an all-zero block), stored as the byte
+ * E + 127; codes q = RN_e4m3(g*W / 2^E); value e4m3(q) * 2^E.  The d*ncols/32
+ * scale bytes are grouped by 128-deep k groups (4 blocks); in each group one
+ * 512-byte chunk per 128 columns; inside a chunk the byte of column n, block
+ * j sits at 16*(n mod 32) + 4*((n mod 128) div 32) + (j mod 4).  So the byte
+ * of (n, j) is at 512*((j div 4)*(ncols/128) + n div 128) + that offset, and
+ * a row slice of the weight on 128-row boundaries owns a contiguous range.
+ * Passed through the `scales` argument (its pointer type is nominal here);
+ * 16-byte aligned; needs d % 128 == 0.
+ */
 
 /*
  * fn_fold_weights — offline fold (Proposal 1, weightless normalisation).
@@ -78,6 +97,9 @@ typedef enum {
  *           [d/128, ncols/128]: per 128x128 block s = amax|g*W| / 448 (1 if the
  *           block is all zero), Wp = RN_e4m3_satfinite(fp32(g*W) / s); needs
  *           d % 128 == 0.
+ *           FN_W_MXFP8_E4M3: Wp = e4m3 bytes [d, ncols] and `scales` receives
+ *           the d*ncols/32 ue8m0 bytes described above (fp32 g*W, one exact
+ *           power-of-two scaling, one RN to e4m3); needs d % 128 == 0.
  *   ncols = N, or 2N with W1: then 128-column tiles alternate gate, up, gate,
  *           up (stored columns [256j, 256j+128) = gate columns [128j, 128j+128),
  *           [256j+128, 256j+256) = the same up columns).
@@ -96,7 +118,10 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
  * factors and per-block sums of squares; with fp8 weights and M >= 1024 one
  * bf16 copy of the weight, converted once per call with the same rounding the
  * on-chip conversion uses (bf16(fp32(q) * s)), because converting each weight
- * tile once per 128-row tile would repeat that work M/128 times.  Zero it once
+ * tile once per 128-row tile would repeat that work M/128 times; with MXFP8
+ * weights the same bf16 copy at every M > 64, and at M <= 64 the activations
+ * split once per call (2 x 64 x d bytes at most, their scale chunks and
+ * per-group sums of squares).  Zero it once
  * before its first use (the status word must start at zero); the calls keep
  * the status word at zero unless a device-side wait times out.  Depends on
  * the SM count of the current device (148 is assumed when no device is
@@ -108,14 +133,19 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
  * fn_norm_proj — y[M, N] = RMSNorm(x; g, eps) @ W, computed as
  *   r[m] * (x @ W')[m, :] with W' from fn_fold_weights (Proposal 2).
  *   x       bf16 [M, d] raw activations (never normalised in memory)
- *   Wp      folded weight [d, N] of type wt (scales: fp32 [d/128, N/128] for fp8)
+ *   Wp      folded weight [d, N] of type wt (scales: fp32 [d/128, N/128] for fp8,
+ *           the chunked ue8m0 bytes for MXFP8)
  *   eps     >= 0 and finite, added to the mean inside the square root
  *   y       bf16 [M, N] output; must not overlap x, Wp, scales or workspace
  *   workspace, ws_bytes  >= fn_workspace_size(M, d, N, wt, 0), zeroed before first use
  *   M == 0 is a no-op.  M <= 64 runs the split-K decode kernel (plus a small
  *   fix-up kernel for the column tiles whose k range it split), larger M the
  *   tensor-core tile kernel; both are deterministic (repeated calls with the
- *   same inputs give the same bits).
+ *   same inputs give the same bits).  MXFP8 weights: at M <= 64 the e4m3
+ *   codes and their scales go to block-scaled MMAs as stored (the bf16
+ *   activations split exactly into two e4m3 parts sharing one power-of-two
+ *   scale per 32 k values); at M > 64 the weight is converted to bf16 once per
+ *   call into the workspace (an exact conversion) for the tile kernel.
  */
 fn_status fn_norm_proj(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
                        int64_t N, float eps, void* y, void* workspace, size_t ws_bytes, fn_stream_t stream);
@@ -255,6 +285,10 @@ fn_status fn_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, float 
                      fn_stream_t stream);
 fn_status fn_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t ncols, void* W,
                          fn_stream_t stream);
+/* fn_dequant_mxfp8: W[d, ncols] = bf16(e4m3(q) * 2^(s - 127)), s the chunked
+ * MXFP8 scale bytes (exact for scales a fold produces). */
+fn_status fn_dequant_mxfp8(const void* q, const void* scales, int64_t d, int64_t ncols, void* W,
+                           fn_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* fn_status_string(fn_status s);

@@ -66,7 +66,7 @@ __all__ = [
     "nvfp4_quantize", "nvfp4_pack", "nvfp4_unpack", "nvfp4_dequantize",
     "rowparallel_partial", "rowparallel_finish",
     "MX_BLOCK", "fold_mxfp8", "dequant_mxfp8",
-    "sf_chunk_layout", "sf_chunk_unlayout", "fold_mxfp8_stored",
+    "sf_chunk_layout", "sf_chunk_unlayout", "mx_scale_store", "fold_mxfp8_stored",
 ]
 
 FP8_BLOCK = 128
@@ -487,11 +487,20 @@ def sf_chunk_unlayout(flat, R: int, C: int) -> np.ndarray:
     return flat[src]
 
 
+def mx_scale_store(sb) -> np.ndarray:
+    """MXFP8 scale bytes [d/32, ncols] (32-deep k blocks x stored columns) in
+    the order the library stores them: 128-deep k groups (4 blocks) one after
+    another; each group's [ncols, 4] slab, in the weight's MMA orientation
+    (rows = output columns), laid out by sf_chunk_layout (one 512-byte chunk
+    per 128 columns).  A row slice of the weight on 128-row boundaries
+    therefore owns one contiguous range of scale bytes."""
+    sb = np.asarray(sb, dtype=np.uint8)
+    assert sb.shape[0] % 4 == 0
+    return np.concatenate([sf_chunk_layout(sb[4 * kg: 4 * kg + 4, :].T) for kg in range(sb.shape[0] // 4)])
+
+
 def fold_mxfp8_stored(W, g) -> Tuple[np.ndarray, np.ndarray]:
     """The MXFP8 fold as the library stores it: the e4m3 codes [d, N] of
-    fold_mxfp8, and its scale bytes [d/32, N] transposed to the weight's MMA
-    orientation (rows = output columns n, scale columns = 32-deep k blocks)
-    and laid out by sf_chunk_layout: one 512-byte chunk per 128 output
-    columns and 128 k rows, the k groups of a column block consecutive."""
+    fold_mxfp8 and its scale bytes in the order of mx_scale_store."""
     q, sb = fold_mxfp8(W, g)
-    return q, sf_chunk_layout(sb.T)
+    return q, mx_scale_store(sb)

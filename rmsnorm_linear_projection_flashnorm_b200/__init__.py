@@ -28,6 +28,7 @@ FN_ERR_UNSUPPORTED_DEVICE = 8
 
 FN_W_BF16 = 0
 FN_W_FP8_E4M3_B128 = 1
+FN_W_MXFP8_E4M3 = 2
 
 FN_DEBUG_WAIT_BUDGET_NS = 1
 FN_DEBUG_WITHHOLD_ARRIVE = 2
@@ -51,6 +52,7 @@ _SIGNATURES = {
     "fn_query_static_status": (_int, [ctypes.POINTER(ctypes.c_uint), _vp]),
     "fn_rmsnorm": (_int, [_vp, _i64, _i64, _vp, _f32, _vp, _vp]),
     "fn_dequant_fp8": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
+    "fn_dequant_mxfp8": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "fn_status_string": (ctypes.c_char_p, [_int]),
     "fn_version": (_int, []),
     "fn_kernel_launches": (ctypes.c_uint64, []),
@@ -185,3 +187,7 @@ def fn_rmsnorm(x, M: int, d: int, g, eps: float, h, stream=None) -> int:
 
 def fn_dequant_fp8(q, scales, d: int, ncols: int, W, stream=None) -> int:
     return lib().fn_dequant_fp8(_ptr(q), _ptr(scales), d, ncols, _ptr(W), _stream(stream))
+
+
+def fn_dequant_mxfp8(q, scales, d: int, ncols: int, W, stream=None) -> int:
+    return lib().fn_dequant_mxfp8(_ptr(q), _ptr(scales), d, ncols, _ptr(W), _stream(stream))

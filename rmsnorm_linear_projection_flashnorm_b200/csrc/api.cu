@@ -125,10 +125,10 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   const bool fp4 = yq != nullptr || ysf != nullptr || gscale != nullptr;
   const bool partial = part_out != nullptr;
   if (M < 0 || d <= 0 || N <= 0) return FN_ERR_INVALID_ARG;
-  if (wt != FN_W_BF16 && wt != FN_W_FP8_E4M3_B128) return FN_ERR_INVALID_ARG;
+  if (wt != FN_W_BF16 && wt != FN_W_FP8_E4M3_B128 && wt != FN_W_MXFP8_E4M3) return FN_ERR_INVALID_ARG;
   if (!eps_ok(eps)) return FN_ERR_INVALID_ARG;
   if (d % 64 != 0 || N % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
-  if (wt == FN_W_FP8_E4M3_B128 && d % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (wt != FN_W_BF16 && d % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
   const int64_t ncols = swiglu ? 2 * N : N;
   if (M > kMaxDim || d > kMaxDim || ncols > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FN_OK;
@@ -136,19 +136,22 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   if (partial ? (y || fp4 || swiglu) : fp4 ? (!yq || !ysf || !gscale || y || !swiglu) : !y)
     return FN_ERR_INVALID_ARG;
   if (!ws) return FN_ERR_WORKSPACE;
-  if (wt == FN_W_FP8_E4M3_B128 && !scales) return FN_ERR_INVALID_ARG;
+  if (wt != FN_W_BF16 && !scales) return FN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wp) || !aligned16(ws)) return FN_ERR_ALIGNMENT;
   if (partial ? !aligned16(part_out)
               : fp4 ? (!aligned16(yq) || !aligned16(ysf) || (reinterpret_cast<uintptr_t>(gscale) & 3u))
                     : !aligned16(y))
     return FN_ERR_ALIGNMENT;
-  if (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return FN_ERR_ALIGNMENT;
+  if (scales && (reinterpret_cast<uintptr_t>(scales) & (wt == FN_W_MXFP8_E4M3 ? 15u : 3u))) return FN_ERR_ALIGNMENT;
 
   const size_t wbytes = static_cast<size_t>(d) * ncols * (wt == FN_W_BF16 ? 2 : 1);
   const size_t xbytes = static_cast<size_t>(M) * d * 2;
   const size_t ybytes = static_cast<size_t>(M) * N * 2;
-  const size_t sbytes = scales ? static_cast<size_t>(d / 128) * (ncols / 128) * 4 : 0;
-  if (overlaps(ws, ws_bytes, x, xbytes) || overlaps(ws, ws_bytes, Wp, wbytes)) return FN_ERR_ALIAS;
+  const size_t sbytes = !scales                  ? 0
+                        : wt == FN_W_MXFP8_E4M3 ? static_cast<size_t>(d / 32) * ncols
+                                                : static_cast<size_t>(d / 128) * (ncols / 128) * 4;
+  if (overlaps(ws, ws_bytes, x, xbytes) || overlaps(ws, ws_bytes, Wp, wbytes) || overlaps(ws, ws_bytes, scales, sbytes))
+    return FN_ERR_ALIAS;
   // every output region against every input region, the workspace and each other
   const size_t qbytes = static_cast<size_t>(M) * (N / 2), fbytes = static_cast<size_t>(M) * (N / 16);
   const size_t pbytes = partial ? (static_cast<size_t>(M) * ncols + M) * 4 : 0;
@@ -175,8 +178,11 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   int sms = 0;
   fn_status st = check_device(sms);
   if (st != FN_OK) return st;
-  const bool dequant_once = wt == FN_W_FP8_E4M3_B128 && !use_decode && M >= kFp8DequantOnceM;
-  const size_t need = use_decode     ? decode_workspace_bytes(M, d, ncols, swiglu, sms, wt == FN_W_FP8_E4M3_B128)
+  // fp8 weights at M >= kFp8DequantOnceM and MXFP8 weights on the tile path are
+  // converted to bf16 once per call into the workspace
+  const bool dequant_once =
+      !use_decode && ((wt == FN_W_FP8_E4M3_B128 && M >= kFp8DequantOnceM) || wt == FN_W_MXFP8_E4M3);
+  const size_t need = use_decode     ? decode_workspace_bytes(M, d, ncols, swiglu, sms, static_cast<int>(wt))
                       : dequant_once ? kWsHeaderBytes + wbytes * 2
                                      : kWsHeaderBytes;
   if (ws_bytes < need) return FN_ERR_WORKSPACE;
@@ -209,7 +215,9 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   if (dequant_once) {
     // the bf16 weight bf16(fp32(q) * s), the rounding the on-chip conversion uses
     void* wbf = static_cast<uint8_t*>(ws) + kWsHeaderBytes;
-    if (launch_dequant_fp8(Wp, scales, d, ncols, wbf, a.stream) != cudaSuccess) return FN_ERR_CUDA;
+    const cudaError_t de = wt == FN_W_MXFP8_E4M3 ? launch_dequant_mxfp8(Wp, scales, d, ncols, wbf, a.stream)
+                                                 : launch_dequant_fp8(Wp, scales, d, ncols, wbf, a.stream);
+    if (de != cudaSuccess) return FN_ERR_CUDA;
     a.Wp = wbf;
     a.wtype = FN_W_BF16;
     a.scales = nullptr;
@@ -228,19 +236,22 @@ extern "C" {
 fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, fn_wtype out_type,
                           void* Wp, float* scales, fn_stream_t stream) {
   if (d <= 0 || N <= 0) return FN_ERR_INVALID_ARG;
-  if (out_type != FN_W_BF16 && out_type != FN_W_FP8_E4M3_B128) return FN_ERR_INVALID_ARG;
+  if (out_type != FN_W_BF16 && out_type != FN_W_FP8_E4M3_B128 && out_type != FN_W_MXFP8_E4M3)
+    return FN_ERR_INVALID_ARG;
   if (!W0 || !g || !Wp) return FN_ERR_INVALID_ARG;
-  if (out_type == FN_W_FP8_E4M3_B128 && !scales) return FN_ERR_INVALID_ARG;
+  if (out_type != FN_W_BF16 && !scales) return FN_ERR_INVALID_ARG;
   if (d % 64 != 0 || N % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
-  if (out_type == FN_W_FP8_E4M3_B128 && d % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (out_type != FN_W_BF16 && d % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
   const int64_t ncols = W1 ? 2 * N : N;
   if (d > kMaxDim || ncols > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(W0) || (W1 && !aligned16(W1)) || !aligned16(Wp) || (reinterpret_cast<uintptr_t>(g) & 3u) ||
-      (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)))
+      (scales && (reinterpret_cast<uintptr_t>(scales) & (out_type == FN_W_MXFP8_E4M3 ? 15u : 3u))))
     return FN_ERR_ALIGNMENT;
   const size_t in_bytes = static_cast<size_t>(d) * N * 2;
   const size_t out_bytes = static_cast<size_t>(d) * ncols * (out_type == FN_W_BF16 ? 2 : 1);
-  const size_t s_bytes = scales ? static_cast<size_t>(d / 128) * (ncols / 128) * 4 : 0;
+  const size_t s_bytes = !scales                        ? 0
+                         : out_type == FN_W_MXFP8_E4M3 ? static_cast<size_t>(d / 32) * ncols
+                                                       : static_cast<size_t>(d / 128) * (ncols / 128) * 4;
   if (overlaps(Wp, out_bytes, W0, in_bytes) || overlaps(Wp, out_bytes, W1, in_bytes) ||
       overlaps(Wp, out_bytes, g, static_cast<size_t>(d) * 4) || overlaps(scales, s_bytes, Wp, out_bytes) ||
       overlaps(scales, s_bytes, W0, in_bytes) || overlaps(scales, s_bytes, W1, in_bytes))
@@ -249,8 +260,9 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
   fn_status st = check_device(sms);
   if (st != FN_OK) return st;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e = out_type == FN_W_BF16 ? launch_fold_bf16(W0, W1, g, d, N, Wp, s)
-                                              : launch_fold_fp8(W0, W1, g, d, N, Wp, scales, s);
+  const cudaError_t e = out_type == FN_W_BF16          ? launch_fold_bf16(W0, W1, g, d, N, Wp, s)
+                        : out_type == FN_W_MXFP8_E4M3 ? launch_fold_mxfp8(W0, W1, g, d, N, Wp, scales, s)
+                                                      : launch_fold_fp8(W0, W1, g, d, N, Wp, scales, s);
   return e == cudaSuccess ? FN_OK : FN_ERR_CUDA;
 }
 
@@ -258,11 +270,11 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
   if (M <= 0 || d <= 0 || N <= 0 || d % 64 != 0 || N % 128 != 0) return kWsHeaderBytes;
   const int64_t ncols = swiglu ? 2 * N : N;
   if (M > 64) {
-    if (wt == FN_W_FP8_E4M3_B128 && M >= kFp8DequantOnceM)
+    if ((wt == FN_W_FP8_E4M3_B128 && M >= kFp8DequantOnceM) || wt == FN_W_MXFP8_E4M3)
       return kWsHeaderBytes + static_cast<size_t>(d) * static_cast<size_t>(ncols) * 2;
     return kWsHeaderBytes;
   }
-  return decode_workspace_bytes(M, d, ncols, swiglu != 0, current_sms_or_default(), wt == FN_W_FP8_E4M3_B128);
+  return decode_workspace_bytes(M, d, ncols, swiglu != 0, current_sms_or_default(), static_cast<int>(wt));
 }
 
 fn_status fn_norm_proj(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
@@ -360,6 +372,22 @@ fn_status fn_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t 
   fn_status st = check_device(sms);
   if (st != FN_OK) return st;
   return launch_dequant_fp8(q, scales, d, ncols, W, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FN_OK
+             : FN_ERR_CUDA;
+}
+
+fn_status fn_dequant_mxfp8(const void* q, const void* scales, int64_t d, int64_t ncols, void* W,
+                           fn_stream_t stream) {
+  if (d <= 0 || ncols <= 0 || !q || !scales || !W) return FN_ERR_INVALID_ARG;
+  if (d % 128 != 0 || ncols % 128 != 0 || d > kMaxDim || ncols > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(W) || !aligned16(scales)) return FN_ERR_ALIGNMENT;
+  const size_t out = static_cast<size_t>(d) * ncols * 2;
+  if (overlaps(W, out, q, static_cast<size_t>(d) * ncols) || overlaps(W, out, scales, static_cast<size_t>(d / 32) * ncols))
+    return FN_ERR_ALIAS;
+  int sms = 0;
+  fn_status st = check_device(sms);
+  if (st != FN_OK) return st;
+  return launch_dequant_mxfp8(q, scales, d, ncols, W, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? FN_OK
              : FN_ERR_CUDA;
 }

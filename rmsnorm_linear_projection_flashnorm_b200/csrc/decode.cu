@@ -509,6 +509,8 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.ysf = static_cast<uint8_t*>(a.ysf);
   p.gscale = a.gscale;
   p.part_out = a.part_out;
+  p.wsf = nullptr;
+  p.xsf = nullptr;
   constexpr size_t SMEM = smem_bytes<MPAD, HALVES>();
   cudaError_t e = ensure_smem_limit<decode_kernel<MPAD, HALVES, OUT>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
@@ -540,9 +542,9 @@ cudaError_t launch_impl(const CallArgs& a) {
 
 int decode_mpad(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
-size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms, bool fp8) {
+size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms, int wtype) {
   const int mp = decode_mpad(M);
-  const size_t extra = fp8 ? decode_fp8_presplit_bytes(M, d) : 0;
+  const size_t extra = wtype == 1 ? decode_fp8_presplit_bytes(M, d) : wtype == 2 ? decode_mx_presplit_bytes(M, d) : 0;
   if (swiglu) {
     if (mp == 16) return dec::workspace_bytes<16, 2>(d, ncols, num_sms) + extra;
     if (mp == 32) return dec::workspace_bytes<32, 2>(d, ncols, num_sms) + extra;
@@ -556,6 +558,7 @@ size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, 
 cudaError_t launch_decode(const CallArgs& a) {
   const int mp = decode_mpad(a.M);
   if (a.wtype == 1) return launch_decode_fp8(a, mp);
+  if (a.wtype == 2) return launch_decode_mx(a, mp);
   if (a.part_out) {   // partial output: a plain projection of the stored columns
     if (mp == 16) return dec::launch_impl<16, 1, kOutPartial>(a);
     if (mp == 32) return dec::launch_impl<32, 1, kOutPartial>(a);

@@ -52,6 +52,8 @@ struct Params {
   uint8_t* ysf;              //   and e4m3 scale codes [M][nout / 16]
   const float* gscale;       //   global scale (one fp32 value in device memory)
   float* part_out;           // partial output: fp32 [M][ncols] accumulators, then [M] sums of squares
+  const uint8_t* wsf;        // MXFP8 weights: ue8m0 scale chunks (k groups, then 128-column blocks)
+  uint8_t* xsf;              // MXFP8 path, x split once per call: ue8m0 scale chunk per k group
 };
 
 // One partial-result slot: float4 groups [half][row / 4][column] for the

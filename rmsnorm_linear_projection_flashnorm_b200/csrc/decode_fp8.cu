@@ -649,6 +649,8 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.ysf = static_cast<uint8_t*>(a.ysf);
   p.gscale = a.gscale;
   p.part_out = a.part_out;
+  p.wsf = nullptr;
+  p.xsf = nullptr;
   tq = tw;   // unused unless x is split once per call
   if (PRE) {
     // after the partial slots: x_hi / x_lo slabs, then the scale factors

@@ -133,6 +133,102 @@ __global__ void __launch_bounds__(kFoldThreads) fold_fp8_kernel(const __nv_bfloa
   }
 }
 
+// MXFP8 fold: e4m3 codes with one power-of-two scale per 32 consecutive k
+// values of each stored column (the block-scaled format the tensor cores'
+// kind::mxf8f6f4 MMAs read).  Per block the shared exponent is the smallest
+// E with amax <= 448 * 2^E, i.e. E = ceil(log2(amax / 448)): with
+// amax = m * 2^e0 (m in [1, 2)) and 448 = 1.75 * 2^8 that is e0 - 8, plus one
+// when m > 1.75; clamped to [-127, 127]; an all-zero block stores E = -127.
+// Codes are RN_e4m3(P * 2^-E), an exact scaling.  The scale byte E + 127 is
+// stored in the chunked layout the block-scaled MMAs read (mx_sf_offset).
+//
+// Scale byte of stored column n, 32-deep k block kb32, for a weight of
+// `ncb` 128-column blocks: 128-deep k groups one after another, in each group
+// one 512-byte chunk per 128 columns, and in a chunk 32 lines of 16 bytes,
+// line (n mod 32) holding columns n, n+32, n+64, n+96 of the chunk, each with
+// its group's four k blocks.
+__device__ __forceinline__ int64_t mx_sf_offset(int64_t n, int64_t kb32, int64_t ncb) {
+  return 512 * ((kb32 >> 2) * ncb + (n >> 7)) + 16 * (n & 31) + 4 * ((n & 127) >> 5) + (kb32 & 3);
+}
+
+__device__ __forceinline__ float pow2f(int e) {   // 2^e for e in [-127, 127], exact
+  return e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// One thread per (stored column, 32-deep k block); adjacent threads take
+// adjacent columns, so the weight reads of a warp are contiguous.
+__global__ void __launch_bounds__(kFoldThreads) fold_mxfp8_kernel(const __nv_bfloat16* __restrict__ W0,
+                                                                  const __nv_bfloat16* __restrict__ W1,
+                                                                  const float* __restrict__ g, int64_t d,
+                                                                  int64_t N, uint8_t* __restrict__ Wq,
+                                                                  uint8_t* __restrict__ sf) {
+  const bool inter = W1 != nullptr;
+  const int64_t ncols = inter ? 2 * N : N;
+  const int64_t total = ncols * (d / 32);
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = t % ncols, j = t / ncols;
+    int src;
+    int64_t n;
+    stored_to_source(c, inter, src, n);
+    const __nv_bfloat16* W = src ? W1 : W0;
+    float p[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int64_t k = j * 32 + i;
+      p[i] = __fmul_rn(g[k], __bfloat162float(W[k * N + n]));
+      amax = fmaxf(amax, fabsf(p[i]));
+    }
+    int E = -127;
+    if (amax > 0.f) {
+      const uint32_t bits = __float_as_uint(amax);
+      const int e0 = static_cast<int>(bits >> 23) - 127;       // subnormal amax: E clamps to -127 below
+      E = e0 - 8 + ((bits & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+      E = E < -127 ? -127 : (E > 127 ? 127 : E);
+    }
+    const float inv = pow2f(-E);
+    sf[mx_sf_offset(c, j, ncols / 128)] = static_cast<uint8_t>(E + 127);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const uint16_t q2 = f32x2_to_e4m3x2(__fmul_rn(p[i], inv), __fmul_rn(p[i + 1], inv));
+      Wq[(j * 32 + i) * ncols + c] = static_cast<uint8_t>(q2 & 0xFFu);
+      Wq[(j * 32 + i + 1) * ncols + c] = static_cast<uint8_t>(q2 >> 8);
+    }
+  }
+}
+
+// MXFP8 -> bf16: W[k, c] = bf16(e4m3(q[k, c]) * 2^(s - 127)), exact for the
+// scales a fold produces (a byte of 255, the format's NaN, gives NaN).
+__global__ void __launch_bounds__(256) dequant_mxfp8_kernel(const uint8_t* __restrict__ q,
+                                                            const uint8_t* __restrict__ sf, int64_t d,
+                                                            int64_t ncols, __nv_bfloat16* __restrict__ W) {
+  const int64_t vec_per_row = ncols / 8;
+  const int64_t total = d * vec_per_row;
+  for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < total;
+       v += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t k = v / vec_per_row;
+    const int64_t c = (v - k * vec_per_row) * 8;
+    const uint2 b = *reinterpret_cast<const uint2*>(q + k * ncols + c);
+    const uint32_t in[2] = {b.x, b.y};
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t c0 = c + 4 * j + 2 * h;
+        const uint32_t e0 = sf[mx_sf_offset(c0, k >> 5, ncols / 128)], e1 = sf[mx_sf_offset(c0 + 1, k >> 5, ncols / 128)];
+        const float s0 = e0 == 255u ? __int_as_float(0x7fc00000) : pow2f(static_cast<int>(e0) - 127);
+        const float s1 = e1 == 255u ? __int_as_float(0x7fc00000) : pow2f(static_cast<int>(e1) - 127);
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+            static_cast<__nv_fp8x2_storage_t>((in[j] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+        out[2 * j + h] = pack_bf16x2(__fmul_rn(f.x, s0), __fmul_rn(f.y, s1));
+      }
+    }
+    *reinterpret_cast<uint4*>(W + k * ncols + c) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
 // Unfused chain, step 1: h = bf16((x * r) * g) per row, r = 1/sqrt(mean(x^2)+eps).
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t d,
                                                       const float* __restrict__ g, float eps,
@@ -229,6 +325,25 @@ cudaError_t launch_fold_fp8(const void* W0, const void* W1, const float* g, int6
   fold_fp8_kernel<<<grid, kFoldThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(W0),
                                                 static_cast<const __nv_bfloat16*>(W1), g, d, N,
                                                 static_cast<uint8_t*>(Wq), scales);
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launch();
+  return e;
+}
+
+cudaError_t launch_fold_mxfp8(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wq,
+                              void* sf, cudaStream_t s) {
+  const int64_t ncols = W1 ? 2 * N : N;
+  fold_mxfp8_kernel<<<grid_for(ncols * (d / 32), kFoldThreads), kFoldThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(W0), static_cast<const __nv_bfloat16*>(W1), g, d, N,
+      static_cast<uint8_t*>(Wq), static_cast<uint8_t*>(sf));
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launch();
+  return e;
+}
+
+cudaError_t launch_dequant_mxfp8(const void* q, const void* sf, int64_t d, int64_t ncols, void* W, cudaStream_t s) {
+  dequant_mxfp8_kernel<<<grid_for(d * ncols / 8, 256), 256, 0, s>>>(
+      static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(sf), d, ncols, static_cast<__nv_bfloat16*>(W));
   const cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) count_launch();
   return e;

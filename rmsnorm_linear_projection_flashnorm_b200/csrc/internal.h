@@ -27,8 +27,8 @@ struct CallArgs {
   const void* x;          // bf16 [M, d]
   int64_t M, d;
   const void* Wp;         // folded weight, bf16 or e4m3 [d, ncols]
-  const float* scales;    // fp8 block scales [d/128, ncols/128] or null
-  int wtype;              // 0 bf16, 1 e4m3 with 128x128 block scales
+  const float* scales;    // fp8 block scales [d/128, ncols/128], MXFP8 scale bytes (chunked), or null
+  int wtype;              // 0 bf16, 1 e4m3 with 128x128 block scales, 2 MXFP8
   int64_t N;              // output columns
   int64_t ncols;          // stored weight columns: N or 2N (SwiGLU)
   bool swiglu;
@@ -62,12 +62,17 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, in
 // Decode (M <= 64) path: stream-K split over all SMs with a deterministic
 // in-kernel fix-up through workspace partials.
 int decode_mpad(int64_t M);
-size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms, bool fp8);
+// wtype: 0 bf16, 1 e4m3 with 128x128 fp32 scales, 2 MXFP8 (e4m3 with ue8m0 per 32 k)
+size_t decode_workspace_bytes(int64_t M, int64_t d, int64_t ncols, bool swiglu, int num_sms, int wtype);
 // fp8 weights, 17..64 rows: workspace for x split once per call (decode_fp8.cu)
 size_t decode_fp8_presplit_bytes(int64_t M, int64_t d);
+// MXFP8 weights: workspace for x split once per call (decode_mx.cu)
+size_t decode_mx_presplit_bytes(int64_t M, int64_t d);
 cudaError_t launch_decode(const CallArgs& a);
 // fp8 weights on the decode path (decode_fp8.cu); mpad is decode_mpad(M).
 cudaError_t launch_decode_fp8(const CallArgs& a, int mpad);
+// MXFP8 weights on the decode path: block-scaled MMAs (decode_mx.cu).
+cudaError_t launch_decode_mx(const CallArgs& a, int mpad);
 
 // Tensor-core tile path (M > 64): persistent 128x256 tiles, tcgen05 + TMEM.
 cudaError_t launch_tc(const CallArgs& a);
@@ -77,6 +82,10 @@ cudaError_t launch_fold_bf16(const void* W0, const void* W1, const float* g, int
                              cudaStream_t s);
 cudaError_t launch_fold_fp8(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wq,
                             float* scales, cudaStream_t s);
+// MXFP8 weights: e4m3 codes and ue8m0 scale bytes in the chunked layout.
+cudaError_t launch_fold_mxfp8(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wq,
+                              void* sf, cudaStream_t s);
+cudaError_t launch_dequant_mxfp8(const void* q, const void* sf, int64_t d, int64_t ncols, void* W, cudaStream_t s);
 cudaError_t launch_rmsnorm(const void* x, int64_t M, int64_t d, const float* g, float eps, void* h,
                            cudaStream_t s);
 // Row-parallel split of d: the post-scale after the partials were summed (post_scale.cu).

@@ -169,6 +169,16 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, ui
       : "memory");
 }
 
+// Contiguous bulk copy global -> shared (no tensor map), completion as
+// transaction bytes on `bar`.  Both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Bring a 2D tile of a tensor into L2 only (no shared memory, no barrier).
 // L2 is the coherence point for global memory, so a prefetch can never leave
 // a stale copy behind: it is safe to issue before griddepcontrol.wait, even if
@@ -267,6 +277,48 @@ __device__ __forceinline__ void umma_e4m3(uint32_t tmem_d, uint64_t adesc, uint6
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Block-scaled MMAs (kind::mxf8f6f4.block_scale): e4m3 A and B, fp32
+// accumulator, one ue8m0 scale per 32 k values of every A row and B column,
+// read from TMEM.  Instruction descriptor fields as kind::f16's, except:
+//   bits 4-5 scale byte of B (which byte of each 32-bit TMEM scale word this
+//   MMA uses), bit 23 scale format (1 = ue8m0), bits 29-30 scale byte of A.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, bool a_mn_major, bool b_mn_major, int sf_id) {
+  return (static_cast<uint32_t>(sf_id & 3) << 4) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(sf_id & 3) << 29);
+}
+
+// D[tmem] (+)= (A * 2^sfa) (B * 2^sfb), K = 32 per instruction, scales in TMEM.
+__device__ __forceinline__ void umma_mx_e4m3(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t tmem_sfa, uint32_t tmem_sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(tmem_sfa), "r"(tmem_sfb), "r"(accumulate)
+      : "memory");
+}
+
+// Shared-memory descriptor of a plain (unswizzled) K-major operand: 8-row
+// groups of 16-byte lines, `sbo_bytes` apart.  Used for the 32 x 16-byte
+// scale chunks that tcgen05.cp copies into TMEM.
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  return d;   // layout type 0: no swizzle
+}
+
+// Copy 32 lines of 16 bytes from shared memory into 4 consecutive TMEM
+// columns of lanes 0-31, repeated in all four lane quarters (the layout the
+// block-scaled MMAs read their scales from).  Ordered with this thread's
+// later tcgen05.mma instructions; tracked by tcgen05.commit.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Arrive once on `bar` when all previously issued tcgen05 operations of this

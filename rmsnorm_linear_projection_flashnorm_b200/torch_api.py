@@ -7,9 +7,17 @@ from typing import Optional, Tuple
 
 import torch
 
-from . import (FN_W_BF16, FN_W_FP8_E4M3_B128, check, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
+from . import (FN_W_BF16, FN_W_FP8_E4M3_B128, FN_W_MXFP8_E4M3, check, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
                fn_norm_proj_partial, fn_norm_proj_swiglu_nvfp4, fn_post_scale, fn_query_device_status,
                fn_workspace_size)
+
+
+def weight_type(Wp: torch.Tensor, scales: Optional[torch.Tensor]) -> int:
+    """The fn_wtype of a folded weight: bf16, e4m3 with fp32 block scales, or
+    MXFP8 (e4m3 with ue8m0 scale bytes)."""
+    if Wp.dtype == torch.bfloat16:
+        return FN_W_BF16
+    return FN_W_MXFP8_E4M3 if scales is not None and scales.dtype == torch.uint8 else FN_W_FP8_E4M3_B128
 
 
 def fold(W0: torch.Tensor, g: torch.Tensor, W1: Optional[torch.Tensor] = None, wtype: int = FN_W_BF16,
@@ -21,6 +29,9 @@ def fold(W0: torch.Tensor, g: torch.Tensor, W1: Optional[torch.Tensor] = None, w
     if wtype == FN_W_BF16:
         Wp = torch.empty((d, ncols), dtype=torch.bfloat16, device=dev)
         scales = None
+    elif wtype == FN_W_MXFP8_E4M3:
+        Wp = torch.empty((d, ncols), dtype=torch.uint8, device=dev)
+        scales = torch.empty(d * ncols // 32, dtype=torch.uint8, device=dev)   # chunked ue8m0 bytes
     else:
         Wp = torch.empty((d, ncols), dtype=torch.uint8, device=dev)
         scales = torch.empty((d // 128, ncols // 128), dtype=torch.float32, device=dev)
@@ -50,7 +61,7 @@ def norm_proj(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float, swiglu: boo
               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """y = RMSNorm(x) @ W through the fused kernels (W' already folded)."""
     M, d = x.shape
-    wt = FN_W_BF16 if Wp.dtype == torch.bfloat16 else FN_W_FP8_E4M3_B128
+    wt = weight_type(Wp, scales)
     if ws is None:
         ws = Workspace(x.device)
     buf = ws.get(M, d, N, wt, swiglu)
@@ -68,7 +79,7 @@ def norm_proj_swiglu_nvfp4(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float
     """SwiGLU output in NVFP4: (codes uint8 [M, N/2], e4m3 scale bytes uint8
     [M, N/16]); global_scale is a one-element fp32 device tensor."""
     M, d = x.shape
-    wt = FN_W_BF16 if Wp.dtype == torch.bfloat16 else FN_W_FP8_E4M3_B128
+    wt = weight_type(Wp, scales)
     if ws is None:
         ws = Workspace(x.device)
     buf = ws.get(M, d, N, wt, True)
@@ -87,7 +98,7 @@ def norm_proj_partial(x: torch.Tensor, Wp: torch.Tensor, ncols: int, scales: Opt
     """One rank's share of a row-parallel projection: fp32 [M * ncols + M]
     (unscaled x @ Wp in stored column order, then the rows' sums of squares)."""
     M, d = x.shape
-    wt = FN_W_BF16 if Wp.dtype == torch.bfloat16 else FN_W_FP8_E4M3_B128
+    wt = weight_type(Wp, scales)
     if ws is None:
         ws = Workspace(x.device)
     buf = ws.get(M, d, ncols, wt, False)

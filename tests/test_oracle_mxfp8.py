@@ -154,9 +154,12 @@ def test_stored_mxfp8_fold_is_the_fold_in_chunks():
     inp = WL.case(4, 256, 384, False, seed=22)
     q, sb = O.fold_mxfp8(inp["W"], inp["g"])
     q2, flat = O.fold_mxfp8_stored(inp["W"], inp["g"])
-    assert np.array_equal(q, q2)
-    # column n, k block j of the stored scales: chunk (n div 128, j div 4)
+    assert np.array_equal(q, q2) and flat.size == 256 * 384 // 32
+    # column n, k block j: k group j div 4 (3 chunks of 128 columns each), chunk n div 128
     for n in (0, 31, 32, 127, 128, 300, 383):
         for j in (0, 3, 4, 7):
-            off = 512 * ((n // 128) * 2 + j // 4) + 16 * (n % 32) + 4 * ((n % 128) // 32) + j % 4
+            off = 512 * ((j // 4) * 3 + n // 128) + 16 * (n % 32) + 4 * ((n % 128) // 32) + j % 4
             assert flat[off] == sb[j, n]
+    # a 128-row slice of the weight owns a contiguous range of the scale bytes
+    q3, flat3 = O.fold_mxfp8_stored(inp["W"][128:], inp["g"][128:])
+    assert np.array_equal(flat3, flat[flat.size // 2:])
