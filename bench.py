@@ -181,6 +181,16 @@ def algorithmic(M: int, d: int, N: int, swiglu: bool, wbytes_per_elem: int = 2, 
     return by, fl
 
 
+def scale_bytes(wl: WL.Workload) -> int:
+    """Bytes of the weight's block scales: fp32 per 128x128 block, or one
+    ue8m0 byte per 32 k values per column (MXFP8)."""
+    if wl.wtype == "fp8_e4m3_b128":
+        return (wl.d // 128) * (wl.ncols // 128) * 4
+    if wl.wtype == "mxfp8_e4m3":
+        return wl.d * wl.ncols // 32
+    return 0
+
+
 def kernel_source_hash(names):
     h = hashlib.sha256()
     for n in names:
@@ -221,7 +231,8 @@ class Setup:
         self.fnb, self.T = fnb, T
         self.wl, self.Ms, self.dev = wl, list(Ms), device
         d, N, sw = wl.d, wl.N, wl.swiglu
-        self.wtype = fnb.FN_W_BF16 if wl.wtype == "bf16" else fnb.FN_W_FP8_E4M3_B128
+        self.wtype = {"bf16": fnb.FN_W_BF16, "fp8_e4m3_b128": fnb.FN_W_FP8_E4M3_B128,
+                      "mxfp8_e4m3": fnb.FN_W_MXFP8_E4M3}[wl.wtype]
         Mmax = max(self.Ms)
         if gen == "device":
             x_all, g, W = WL.device_inputs(wl, Mmax, device)
@@ -308,7 +319,8 @@ class Setup:
                 self.W_unf = torch.empty_like(self.Wp[0], dtype=torch.bfloat16)
                 self.g_one = torch.ones_like(self.g)
             ncols = self.Wp[c].shape[1]
-            st = self.fnb.fn_dequant_fp8(self.Wp[c], self.scales[c], wl.d, ncols, self.W_unf, stream)
+            deq = self.fnb.fn_dequant_mxfp8 if self.wtype == self.fnb.FN_W_MXFP8_E4M3 else self.fnb.fn_dequant_fp8
+            st = deq(self.Wp[c], self.scales[c], wl.d, ncols, self.W_unf, stream)
             if st != 0:
                 raise RuntimeError(self.fnb.status_string(st))
             W, g = self.W_unf, self.g_one
@@ -459,13 +471,14 @@ def roofline_entry(units_per_call: float, us_per_call: float, hbm_bound: bool, p
 def kernel_for(wl: WL.Workload, M: int, out: str):
     """Name of the dominant kernel of a call, its sources and its ncu summary file."""
     if M <= 64:
-        kname = "decode_kernel" if wl.wtype == "bf16" else "decode_fp8_kernel"
-        sources = ["decode.cu" if wl.wtype == "bf16" else "decode_fp8.cu", "decode_common.cuh", "ptx.cuh",
-                   "nvfp4.cuh"]
+        kname, src = {"bf16": ("decode_kernel", "decode.cu"), "fp8_e4m3_b128": ("decode_fp8_kernel", "decode_fp8.cu"),
+                      "mxfp8_e4m3": ("decode_mx_kernel", "decode_mx.cu")}[wl.wtype]
+        sources = [src, "decode_common.cuh", "ptx.cuh", "nvfp4.cuh"]
         label = f"{kname} (+ decode_fixup_kernel where a tile's k range is split)"
     else:
         kname, sources = "tc_kernel", ["tc.cu", "ptx.cuh", "nvfp4.cuh"]
-        label = "tc_kernel" + (" (after the dequantise-once kernel)" if wl.wtype != "bf16" and M >= 1024 else "")
+        once = wl.wtype == "mxfp8_e4m3" or (wl.wtype != "bf16" and M >= 1024)
+        label = "tc_kernel" + (" (after the dequantise-once kernel)" if once else "")
     src_hash = kernel_source_hash(sources)
     prof = f"{kname}_{wl.name}{'_nvfp4' if out == 'nvfp4' else ''}.md"
     return kname, label, src_hash, profile_traffic(prof, src_hash)
@@ -476,7 +489,7 @@ def kernel_for(wl: WL.Workload, M: int, out: str):
 # and unfused chain.
 SUB_RECORDS = (
     ("ffn_swiglu", 4096), ("prefill_swiglu_large", 16384), ("fp8_swiglu", 8192), ("fp8_swiglu", 256),
-    ("ffn_swiglu", 16), ("fp8_swiglu", 1), ("fp8_swiglu", 64),
+    ("ffn_swiglu", 16), ("fp8_swiglu", 1), ("fp8_swiglu", 64), ("mxfp8_swiglu", 1), ("mxfp8_swiglu", 64),
 )
 
 
@@ -490,8 +503,7 @@ def run_sub_record(name: str, M: int, dev, peaks, peaks_kind, world: int, target
     stream = torch.cuda.current_stream()
     wbyte = 2 if wl.wtype == "bf16" else 1
     by, fl = algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte)
-    if wl.wtype != "bf16":
-        by += (wl.d // 128) * (wl.ncols // 128) * 4       # fp32 block scales
+    by += scale_bytes(wl)
     hbm_bound = M <= 64
 
     def timed(fn, n):
@@ -528,8 +540,8 @@ def run_sub_record(name: str, M: int, dev, peaks, peaks_kind, world: int, target
     chain_us = max_over_ranks(chain_us, world, dev)
     rec["unfused_chain"] = {"us_per_call": chain_us, "fused_speedup": chain_us / rec["us_per_call"],
                             "clocks": cclk.summary(),
-                            "what": ("fn_dequant_fp8 (e4m3 W' -> bf16) -> fn_rmsnorm (no gain) -> torch.matmul "
-                                     "(cuBLAS)" if wl.wtype != "bf16" else
+                            "what": (f"fn_dequant_{'mx' if wl.wtype == 'mxfp8_e4m3' else ''}fp8 (e4m3 W' -> bf16) -> "
+                                     "fn_rmsnorm (no gain) -> torch.matmul (cuBLAS)" if wl.wtype != "bf16" else
                                      "fn_rmsnorm -> torch.matmul (cuBLAS) with unfolded W")
                                     + (" -> silu(gate)*up" if wl.swiglu else "")}
     del S
@@ -581,7 +593,7 @@ def main():
     stream = torch.cuda.current_stream()
     peaks, peaks_kind = load_peaks()
     wbyte = 2 if wl.wtype == "bf16" else 1
-    bytes_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte, args.out)[0] for M in Ms)
+    bytes_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte, args.out)[0] + scale_bytes(wl) for M in Ms)
     flops_per_step = sum(algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte, args.out)[1] for M in Ms)
     hbm_bound = max(Ms) <= 64
 
@@ -669,7 +681,7 @@ def main():
             e1.record(stream)
             torch.cuda.synchronize()
             us_m = max_over_ranks(e0.elapsed_time(e1), world, dev) / (reps * 16) * 1e3
-            by_m = algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte, args.out)[0]
+            by_m = algorithmic(M, wl.d, wl.N, wl.swiglu, wbyte, args.out)[0] + scale_bytes(wl)
             per_m[str(M)] = {"us_per_call": us_m, "GB/s": by_m / (us_m / 1e6) / 1e9,
                              "frac": by_m / (us_m / 1e6) / 1e9 / roofline["peak"]} if hbm_bound else \
                 {"us_per_call": us_m}

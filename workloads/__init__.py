@@ -40,7 +40,7 @@ class Workload:
     d: int
     N: int            # output columns (per half for SwiGLU)
     swiglu: bool
-    wtype: str        # "bf16" or "fp8_e4m3_b128"
+    wtype: str        # "bf16", "fp8_e4m3_b128" or "mxfp8_e4m3"
     outliers: bool
     seed: int
 
@@ -58,9 +58,12 @@ WORKLOADS: Dict[str, Workload] = {
         Workload("ffn_swiglu", (16, 4096), 4096, 14336, True, "bf16", False, 2),
         Workload("prefill_swiglu_large", (16384,), 8192, 28672, True, "bf16", True, 3),
         Workload("fp8_swiglu", (1, 64, 256, 8192), 5120, 13824, True, "fp8_e4m3_b128", False, 4),
+        # the fp8 workload's shapes and inputs with the weight folded to the
+        # block-scaled MXFP8 format instead of 128x128 fp32 block scales
+        Workload("mxfp8_swiglu", (1, 64), 5120, 13824, True, "mxfp8_e4m3", False, 4),
     )
 }
-WORKLOAD_ORDER = ("tiny", "decode_qkv", "ffn_swiglu", "prefill_swiglu_large", "fp8_swiglu")
+WORKLOAD_ORDER = ("tiny", "decode_qkv", "ffn_swiglu", "prefill_swiglu_large", "fp8_swiglu", "mxfp8_swiglu")
 
 _CHUNK = 1 << 22  # elements per draw, bounds host memory for the large weights
 
