@@ -67,6 +67,7 @@ __all__ = [
     "rowparallel_partial", "rowparallel_finish",
     "MX_BLOCK", "fold_mxfp8", "dequant_mxfp8",
     "sf_chunk_layout", "sf_chunk_unlayout", "mx_scale_store", "fold_mxfp8_stored",
+    "adaln_modulate", "norm_proj_adaln", "norm_proj_adaln_swiglu", "adaln_shift_bias",
 ]
 
 FP8_BLOCK = 128
@@ -504,3 +505,52 @@ def fold_mxfp8_stored(W, g) -> Tuple[np.ndarray, np.ndarray]:
     fold_mxfp8 and its scale bytes in the order of mx_scale_store."""
     q, sb = fold_mxfp8(W, g)
     return q, mx_scale_store(sb)
+
+
+# ---------------------------------------------------------------------------
+# AdaLN modulation after the norm (FlashInfer PR #5521 analysis, fused API)
+# ---------------------------------------------------------------------------
+# The PR #5521 analysis fuses "RMSNorm + AdaLN" into its FC1 and passes the
+# norm weight, an AdaLN scale, an AdaLN shift and an index for AdaLN; it
+# prints no formula.  Reading used here (adaptive layer norm applied to the
+# normalised row, one scale row and one shift row per condition, selected by
+# each token's index):
+#
+#     h[m, k] = RMSNorm(x; g, eps)[m, k] * scale[c_m, k] + shift[c_m, k],
+#     c_m = index[m],   y = h @ W   (SwiGLU: silu(h @ W_gate) * (h @ W_up))
+#
+# `scale` is the effective multiplier, as g is (a DiT-style 1 + scale is the
+# caller's conversion).
+
+
+def adaln_modulate(x, g, eps: float, scale, shift, index) -> np.ndarray:
+    """h = RMSNorm(x; g, eps) * scale[index] + shift[index], row by row."""
+    idx = np.asarray(index, dtype=np.int64)
+    with np.errstate(invalid="ignore"):
+        return rmsnorm(x, g, eps) * to_f64(scale)[idx] + to_f64(shift)[idx]
+
+
+def norm_proj_adaln(x, g, W, eps: float, scale, shift, index) -> np.ndarray:
+    """y = (RMSNorm(x; g, eps) * scale[index] + shift[index]) @ W, normalising
+    and modulating first (unfolded)."""
+    h = adaln_modulate(x, g, eps, scale, shift, index)
+    with np.errstate(invalid="ignore"):
+        return h @ to_f64(W)
+
+
+def norm_proj_adaln_swiglu(x, g, W_gate, W_up, eps: float, scale, shift, index) -> np.ndarray:
+    """silu(h @ W_gate) * (h @ W_up) with h the AdaLN-modulated norm."""
+    h = adaln_modulate(x, g, eps, scale, shift, index)
+    with np.errstate(invalid="ignore"):
+        return silu(h @ to_f64(W_gate)) * (h @ to_f64(W_up))
+
+
+def adaln_shift_bias(shift, W) -> np.ndarray:
+    """The shift's contribution to the projection, one row per condition:
+    B[c, n] = sum_k shift[c, k] W[k, n] with the unfolded weight (the shift is
+    added after the gain, so the gain does not multiply it).  With it the
+    modulated projection splits into the deferred form
+        y[m, :] = r[m] * ((x[m, :] * scale[c_m, :]) @ W') + B[c_m, :],
+    W' = diag(g) W, which the kernels compute (the scale multiplies the raw
+    activations, the 1/rms scalar stays deferred, the shift becomes a bias)."""
+    return to_f64(shift) @ to_f64(W)
