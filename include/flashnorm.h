@@ -187,6 +187,56 @@ fn_status fn_norm_proj_swiglu_nvfp4(const void* x, int64_t M, int64_t d, const v
                                     void* out_sf, void* workspace, size_t ws_bytes, fn_stream_t stream);
 
 /*
+ * AdaLN-modulated form (the "RMSNorm + AdaLN" front of the fused FC1 on the
+ * FlashInfer PR #5521 analysis: its API takes the norm weight, an AdaLN scale,
+ * an AdaLN shift and an index for AdaLN; the page prints no formula).
+ * Reading: each token m selects condition c = adaln_index[m], and the
+ * normalised row is modulated before the projection,
+ *   h[m, k] = RMSNorm(x; g, eps)[m, k] * scale[c, k] + shift[c, k],  y = h @ W
+ *   (SwiGLU: out = silu(h @ W_gate) * (h @ W_up)),
+ * scale being the effective multiplier (a DiT-style 1 + scale is the
+ * caller's conversion).  With W' = diag(g) W this is
+ *   y[m, :] = r[m] * ((x[m, :] * scale[c, :]) @ W') + B[c, :],
+ *   B[c, :] = shift[c, :] @ W   (the unfolded weight),
+ * so the scale multiplies the raw activations on chip (one rounding of
+ * x * scale to bf16 for the MMA; the sum of squares is taken from the raw x),
+ * the 1/rms scalar stays deferred, and the shift becomes a per-condition bias
+ * row, computed once by fn_adaln_shift_bias.
+ *
+ * fn_adaln_shift_bias — B fp32 [n_cond, ncols] = shift fp32 [n_cond, d] times
+ *   the unfolded weight (W0, and W1 for SwiGLU: columns in the interleaved
+ *   stored order of fn_fold_weights), fp32 products summed in ascending k.
+ *   Alignment: W0/W1 16 bytes, shift and B 4 bytes.  B must not overlap the
+ *   inputs (FN_ERR_ALIAS).
+ */
+fn_status fn_adaln_shift_bias(const float* shift, int64_t n_cond, const void* W0, const void* W1, int64_t d,
+                              int64_t N, float* B, fn_stream_t stream);
+
+/*
+ * fn_norm_proj_adaln — the AdaLN-modulated fn_norm_proj (swiglu = 0) or
+ * fn_norm_proj_swiglu (swiglu != 0).
+ *   adaln_scale  fp32 [n_cond, d], 16-byte aligned
+ *   shift_bias   fp32 [n_cond, ncols] from fn_adaln_shift_bias, 16-byte aligned
+ *   adaln_index  int32 [M]: the condition of each row; a row whose index lies
+ *                outside [0, n_cond) gets NaN outputs (nothing is read out of
+ *                range)
+ *   workspace    >= fn_workspace_size_adaln(d, N, wt, swiglu), zeroed before
+ *                first use
+ * Runs the tensor-core tile kernel at every M; e4m3 and MXFP8 weights are
+ * converted to bf16 once per call into the workspace first.  bf16 output only.
+ * Other arguments, layout and errors as fn_norm_proj.
+ */
+fn_status fn_norm_proj_adaln(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
+                             int64_t N, int swiglu, float eps, const float* adaln_scale, const float* shift_bias,
+                             const int32_t* adaln_index, int64_t n_cond, void* y, void* workspace, size_t ws_bytes,
+                             fn_stream_t stream);
+
+/* fn_workspace_size_adaln — workspace bytes of fn_norm_proj_adaln: the 256-byte
+ * header, plus a bf16 copy of the weight (2 d ncols bytes) for e4m3 and MXFP8
+ * weights. */
+size_t fn_workspace_size_adaln(int64_t d, int64_t N, fn_wtype wt, int swiglu);
+
+/*
  * Row-parallel (d-split) projection, for tensor parallelism that shards the
  * input width d across ranks.  The deferred normalisation (FlashNorm talk
  * summary, Proposal 2) makes 1/rms a per-row factor applied after the matmul,

@@ -67,7 +67,7 @@ __all__ = [
     "rowparallel_partial", "rowparallel_finish",
     "MX_BLOCK", "fold_mxfp8", "dequant_mxfp8",
     "sf_chunk_layout", "sf_chunk_unlayout", "mx_scale_store", "fold_mxfp8_stored",
-    "adaln_modulate", "norm_proj_adaln", "norm_proj_adaln_swiglu", "adaln_shift_bias",
+    "adaln_modulate", "norm_proj_adaln", "norm_proj_adaln_swiglu", "adaln_shift_bias", "adaln_scaled_operand",
 ]
 
 FP8_BLOCK = 128
@@ -554,3 +554,13 @@ def adaln_shift_bias(shift, W) -> np.ndarray:
     W' = diag(g) W, which the kernels compute (the scale multiplies the raw
     activations, the 1/rms scalar stays deferred, the shift becomes a bias)."""
     return to_f64(shift) @ to_f64(W)
+
+
+def adaln_scaled_operand(x, scale, index) -> np.ndarray:
+    """The scaled activations as the tensor cores receive them in the deferred
+    form: the fp32 product fp32(x[m, k]) * fp32(scale[c_m, k]) (IEEE
+    round-to-nearest), rounded once more to bf16 (the MMA's operand format).
+    Returned as float64 values."""
+    idx = np.asarray(index, dtype=np.int64)
+    prod = to_f64(x).astype(np.float32) * to_f64(scale).astype(np.float32)[idx]
+    return bf16_round(prod.astype(np.float64))

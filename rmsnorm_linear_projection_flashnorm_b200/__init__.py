@@ -48,6 +48,10 @@ _SIGNATURES = {
     "fn_norm_proj_partial": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _vp, _vp, _sz, _vp]),
     "fn_post_scale": (_int, [_vp, _i64, _i64, _int, _i64, _f32, _vp, _vp]),
     "fn_norm_proj_static": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp]),
+    "fn_adaln_shift_bias": (_int, [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp]),
+    "fn_norm_proj_adaln": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _int, _f32, _vp, _vp, _vp, _i64, _vp, _vp,
+                                  _sz, _vp]),
+    "fn_workspace_size_adaln": (_sz, [_i64, _i64, _int, _int]),
     "fn_query_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_uint), _vp]),
     "fn_query_static_status": (_int, [ctypes.POINTER(ctypes.c_uint), _vp]),
     "fn_rmsnorm": (_int, [_vp, _i64, _i64, _vp, _f32, _vp, _vp]),
@@ -191,3 +195,18 @@ def fn_dequant_fp8(q, scales, d: int, ncols: int, W, stream=None) -> int:
 
 def fn_dequant_mxfp8(q, scales, d: int, ncols: int, W, stream=None) -> int:
     return lib().fn_dequant_mxfp8(_ptr(q), _ptr(scales), d, ncols, _ptr(W), _stream(stream))
+
+
+def fn_adaln_shift_bias(shift, n_cond: int, W0, W1, d: int, N: int, B, stream=None) -> int:
+    return lib().fn_adaln_shift_bias(_ptr(shift), n_cond, _ptr(W0), _ptr(W1), d, N, _ptr(B), _stream(stream))
+
+
+def fn_norm_proj_adaln(x, M: int, d: int, Wp, scales, wt: int, N: int, swiglu: int, eps: float, adaln_scale,
+                       shift_bias, adaln_index, n_cond: int, y, workspace, ws_bytes: int, stream=None) -> int:
+    return lib().fn_norm_proj_adaln(_ptr(x), M, d, _ptr(Wp), _ptr(scales), wt, N, int(swiglu), eps,
+                                    _ptr(adaln_scale), _ptr(shift_bias), _ptr(adaln_index), n_cond, _ptr(y),
+                                    _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def fn_workspace_size_adaln(d: int, N: int, wt: int = FN_W_BF16, swiglu: int = 0) -> int:
+    return lib().fn_workspace_size_adaln(d, N, wt, int(swiglu))

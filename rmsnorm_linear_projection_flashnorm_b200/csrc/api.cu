@@ -118,10 +118,19 @@ fn_status check_device(int& sms) {
 
 // Fused call.  Output: bf16 y, or (SwiGLU only) NVFP4 codes yq, scale bytes
 // ysf and the global scale gscale, with y null.
+// AdaLN inputs of a fused call (all null: no AdaLN).
+struct AdaLN {
+  const float* scale = nullptr;   // fp32 [n_cond, d]
+  const float* bias = nullptr;    // fp32 [n_cond, ncols]
+  const int32_t* index = nullptr; // [M]
+  int64_t n_cond = 0;
+};
+
 fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
                            int64_t N, float eps, void* y, void* ws, size_t ws_bytes, fn_stream_t stream,
                            bool swiglu, void* yq = nullptr, void* ysf = nullptr, const float* gscale = nullptr,
-                           float* part_out = nullptr) {
+                           float* part_out = nullptr, const AdaLN& ad = AdaLN()) {
+  const bool adaln = ad.index != nullptr || ad.scale != nullptr || ad.bias != nullptr;
   const bool fp4 = yq != nullptr || ysf != nullptr || gscale != nullptr;
   const bool partial = part_out != nullptr;
   if (M < 0 || d <= 0 || N <= 0) return FN_ERR_INVALID_ARG;
@@ -136,6 +145,12 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   if (partial ? (y || fp4 || swiglu) : fp4 ? (!yq || !ysf || !gscale || y || !swiglu) : !y)
     return FN_ERR_INVALID_ARG;
   if (!ws) return FN_ERR_WORKSPACE;
+  if (adaln) {
+    if (!ad.index || !ad.scale || !ad.bias || ad.n_cond <= 0 || partial || fp4) return FN_ERR_INVALID_ARG;
+    if (ad.n_cond > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(ad.scale) || !aligned16(ad.bias) || (reinterpret_cast<uintptr_t>(ad.index) & 3u))
+      return FN_ERR_ALIGNMENT;
+  }
   if (wt != FN_W_BF16 && !scales) return FN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wp) || !aligned16(ws)) return FN_ERR_ALIGNMENT;
   if (partial ? !aligned16(part_out)
@@ -156,20 +171,27 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   const size_t qbytes = static_cast<size_t>(M) * (N / 2), fbytes = static_cast<size_t>(M) * (N / 16);
   const size_t pbytes = partial ? (static_cast<size_t>(M) * ncols + M) * 4 : 0;
   const struct { const void* p; size_t n; } outs[4] = {{y, ybytes}, {yq, qbytes}, {ysf, fbytes}, {part_out, pbytes}};
+  const size_t adsb = adaln ? static_cast<size_t>(ad.n_cond) * d * 4 : 0;
+  const size_t adbb = adaln ? static_cast<size_t>(ad.n_cond) * ncols * 4 : 0;
+  const size_t adib = adaln ? static_cast<size_t>(M) * 4 : 0;
+  if (adaln && (overlaps(ws, ws_bytes, ad.scale, adsb) || overlaps(ws, ws_bytes, ad.bias, adbb) ||
+                overlaps(ws, ws_bytes, ad.index, adib)))
+    return FN_ERR_ALIAS;
   for (int i = 0; i < 4; ++i) {
     if (!outs[i].p) continue;
     if (overlaps(outs[i].p, outs[i].n, x, xbytes) || overlaps(outs[i].p, outs[i].n, Wp, wbytes) ||
         overlaps(outs[i].p, outs[i].n, scales, sbytes) || overlaps(outs[i].p, outs[i].n, ws, ws_bytes) ||
-        overlaps(outs[i].p, outs[i].n, gscale, gscale ? 4 : 0))
+        overlaps(outs[i].p, outs[i].n, gscale, gscale ? 4 : 0) || overlaps(outs[i].p, outs[i].n, ad.scale, adsb) ||
+        overlaps(outs[i].p, outs[i].n, ad.bias, adbb) || overlaps(outs[i].p, outs[i].n, ad.index, adib))
       return FN_ERR_ALIAS;
     for (int j = i + 1; j < 4; ++j)
       if (outs[j].p && overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return FN_ERR_ALIAS;
   }
 
   int force = g_force_path.load();
-  bool use_decode = M <= 64;
+  bool use_decode = M <= 64 && !adaln;   // AdaLN runs on the tile kernel at every M
   if (force == 1) {
-    if (M > 64) return FN_ERR_INVALID_ARG;
+    if (M > 64 || adaln) return FN_ERR_INVALID_ARG;
     use_decode = true;
   } else if (force == 2) {
     use_decode = false;
@@ -181,7 +203,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   // fp8 weights at M >= kFp8DequantOnceM and MXFP8 weights on the tile path are
   // converted to bf16 once per call into the workspace
   const bool dequant_once =
-      !use_decode && ((wt == FN_W_FP8_E4M3_B128 && M >= kFp8DequantOnceM) || wt == FN_W_MXFP8_E4M3);
+      !use_decode && ((wt == FN_W_FP8_E4M3_B128 && (M >= kFp8DequantOnceM || adaln)) || wt == FN_W_MXFP8_E4M3);
   const size_t need = use_decode     ? decode_workspace_bytes(M, d, ncols, swiglu, sms, static_cast<int>(wt))
                       : dequant_once ? kWsHeaderBytes + wbytes * 2
                                      : kWsHeaderBytes;
@@ -212,6 +234,10 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.prefetch_iters = g_prefetch_iters.load();
   a.prefetch_mode = g_prefetch_mode.load();
   a.cluster_mode = g_cluster_mode.load();
+  a.ad_scale = ad.scale;
+  a.ad_bias = ad.bias;
+  a.ad_index = ad.index;
+  a.n_cond = ad.n_cond;
   if (dequant_once) {
     // the bf16 weight bf16(fp32(q) * s), the rounding the on-chip conversion uses
     void* wbf = static_cast<uint8_t*>(ws) + kWsHeaderBytes;
@@ -302,6 +328,47 @@ fn_status fn_norm_proj_partial(const void* x, int64_t M, int64_t d, const void* 
   if (M > 0 && !partial) return FN_ERR_INVALID_ARG;
   return norm_proj_common(x, M, d, Wp, scales, wt, ncols, 0.0f, nullptr, workspace, ws_bytes, stream, false,
                           nullptr, nullptr, nullptr, partial);
+}
+
+fn_status fn_norm_proj_adaln(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
+                             int64_t N, int swiglu, float eps, const float* adaln_scale, const float* shift_bias,
+                             const int32_t* adaln_index, int64_t n_cond, void* y, void* workspace, size_t ws_bytes,
+                             fn_stream_t stream) {
+  if (M > 0 && (!adaln_scale || !shift_bias || !adaln_index || n_cond <= 0)) return FN_ERR_INVALID_ARG;
+  AdaLN ad;
+  ad.scale = adaln_scale;
+  ad.bias = shift_bias;
+  ad.index = adaln_index;
+  ad.n_cond = n_cond;
+  return norm_proj_common(x, M, d, Wp, scales, wt, N, eps, y, workspace, ws_bytes, stream, swiglu != 0, nullptr,
+                          nullptr, nullptr, nullptr, ad);
+}
+
+size_t fn_workspace_size_adaln(int64_t d, int64_t N, fn_wtype wt, int swiglu) {
+  if (d <= 0 || N <= 0 || d % 64 != 0 || N % 128 != 0 || wt == FN_W_BF16) return kWsHeaderBytes;
+  const int64_t ncols = swiglu ? 2 * N : N;
+  return kWsHeaderBytes + static_cast<size_t>(d) * static_cast<size_t>(ncols) * 2;
+}
+
+fn_status fn_adaln_shift_bias(const float* shift, int64_t n_cond, const void* W0, const void* W1, int64_t d,
+                              int64_t N, float* B, fn_stream_t stream) {
+  if (n_cond <= 0 || d <= 0 || N <= 0 || !shift || !W0 || !B) return FN_ERR_INVALID_ARG;
+  if (d % 64 != 0 || N % 128 != 0) return FN_ERR_UNSUPPORTED_SHAPE;
+  const int64_t ncols = W1 ? 2 * N : N;
+  if (d > kMaxDim || ncols > kMaxDim || n_cond > kMaxDim) return FN_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W0) || (W1 && !aligned16(W1)) || (reinterpret_cast<uintptr_t>(shift) & 3u) ||
+      (reinterpret_cast<uintptr_t>(B) & 3u))
+    return FN_ERR_ALIGNMENT;
+  const size_t bb = static_cast<size_t>(n_cond) * ncols * 4;
+  if (overlaps(B, bb, shift, static_cast<size_t>(n_cond) * d * 4) || overlaps(B, bb, W0, static_cast<size_t>(d) * N * 2) ||
+      overlaps(B, bb, W1, W1 ? static_cast<size_t>(d) * N * 2 : 0))
+    return FN_ERR_ALIAS;
+  int sms = 0;
+  const fn_status st = check_device(sms);
+  if (st != FN_OK) return st;
+  return launch_adaln_shift_bias(shift, n_cond, W0, W1, d, N, B, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FN_OK
+             : FN_ERR_CUDA;
 }
 
 fn_status fn_post_scale(const float* partial, int64_t M, int64_t N, int swiglu, int64_t d_total, float eps, void* y,

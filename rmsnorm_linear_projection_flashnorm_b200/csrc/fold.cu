@@ -229,6 +229,31 @@ __global__ void __launch_bounds__(256) dequant_mxfp8_kernel(const uint8_t* __res
   }
 }
 
+// AdaLN shift bias (fold time): the shift row of each condition through the
+// unfolded weight, B[c, col] = sum_k shift[c, k] * W[k, n] for stored column
+// col (gate/up interleaved like the folded weight), fp32 products summed in
+// ascending k.  One thread per (condition, stored column); adjacent threads
+// read adjacent weight columns.
+__global__ void __launch_bounds__(256) adaln_shift_bias_kernel(const float* __restrict__ shift, int64_t n_cond,
+                                                               const __nv_bfloat16* __restrict__ W0,
+                                                               const __nv_bfloat16* __restrict__ W1, int64_t d,
+                                                               int64_t N, float* __restrict__ B) {
+  const bool inter = W1 != nullptr;
+  const int64_t ncols = inter ? 2 * N : N;
+  const int64_t total = n_cond * ncols;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = t / ncols, col = t - c * ncols;
+    int src;
+    int64_t n;
+    stored_to_source(col, inter, src, n);
+    const __nv_bfloat16* W = src ? W1 : W0;
+    const float* sr = shift + c * d;
+    float acc = 0.f;
+    for (int64_t k = 0; k < d; ++k) acc = fmaf(sr[k], __bfloat162float(W[k * N + n]), acc);
+    B[t] = acc;
+  }
+}
+
 // Unfused chain, step 1: h = bf16((x * r) * g) per row, r = 1/sqrt(mean(x^2)+eps).
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t d,
                                                       const float* __restrict__ g, float eps,
@@ -344,6 +369,16 @@ cudaError_t launch_fold_mxfp8(const void* W0, const void* W1, const float* g, in
 cudaError_t launch_dequant_mxfp8(const void* q, const void* sf, int64_t d, int64_t ncols, void* W, cudaStream_t s) {
   dequant_mxfp8_kernel<<<grid_for(d * ncols / 8, 256), 256, 0, s>>>(
       static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(sf), d, ncols, static_cast<__nv_bfloat16*>(W));
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) count_launch();
+  return e;
+}
+
+cudaError_t launch_adaln_shift_bias(const float* shift, int64_t n_cond, const void* W0, const void* W1, int64_t d,
+                                    int64_t N, float* B, cudaStream_t s) {
+  const int64_t ncols = W1 ? 2 * N : N;
+  adaln_shift_bias_kernel<<<grid_for(n_cond * ncols, 256), 256, 0, s>>>(
+      shift, n_cond, static_cast<const __nv_bfloat16*>(W0), static_cast<const __nv_bfloat16*>(W1), d, N, B);
   const cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) count_launch();
   return e;

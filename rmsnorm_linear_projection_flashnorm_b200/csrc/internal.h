@@ -47,6 +47,10 @@ struct CallArgs {
   int prefetch_iters;     // decode: weight k-blocks per CTA prefetched into L2 early
   int prefetch_mode;      // decode: 0 none, 1 TMA prefetch, 2 per-thread prefetch
   int cluster_mode;       // decode: 1 allow split-K inside clusters, 0 stream-K only
+  const float* ad_scale;  // AdaLN (tile path only): scale rows fp32 [n_cond, d], or null
+  const float* ad_bias;   //   shift bias rows fp32 [n_cond, ncols]
+  const int* ad_index;    //   condition index per row [M]; null: no AdaLN
+  int64_t n_cond;
 };
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -93,6 +97,9 @@ cudaError_t launch_post_scale(const float* part, int64_t M, int64_t N, bool swig
                               void* y, cudaStream_t s);
 cudaError_t launch_dequant_fp8(const void* q, const float* scales, int64_t d, int64_t ncols, void* W,
                                cudaStream_t s);
+// AdaLN shift bias B[c, n] = sum_k shift[c, k] W[k, n] in stored column order (fp32 accumulation).
+cudaError_t launch_adaln_shift_bias(const float* shift, int64_t n_cond, const void* W0, const void* W1, int64_t d,
+                                    int64_t N, float* B, cudaStream_t s);
 
 // Raise a kernel's dynamic shared-memory limit once per device (a host-only
 // call, done on the first launch so later launches can be graph-captured).

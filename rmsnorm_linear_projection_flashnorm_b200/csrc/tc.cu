@@ -27,6 +27,16 @@
 //   warps 6-9   epilogue: TMEM -> registers, post-scale (+SwiGLU), bf16 store
 // Accumulators are double-buffered in TMEM (2 x 256 columns) so the epilogue
 // of one tile overlaps the main loop of the next.
+//
+// AdaLN variant (the "RMSNorm + AdaLN" front of the fused FC1 on the
+// FlashInfer PR #5521 analysis: a per-token index selects a scale row and a
+// shift row applied after the norm).  With h = RMSNorm(x; g) * s[c] + t[c]
+// and W' = diag(g) W, the projection is r * ((x * s[c]) @ W') + (t[c] @ W):
+// the scale multiplies the raw activations, so the reducer warps, which read
+// every staged x row for the sum of squares anyway, also write x * s[c] (one
+// rounding to bf16) into a second operand tile that the MMA reads, while the
+// sum of squares still comes from the raw tile; the shift enters through the
+// unfolded weight as a per-condition bias row added in the epilogue.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -46,9 +56,10 @@ constexpr int TMEM_COLS = 2 * BN;
 
 // bf16 weights: 4 stages of 48 KB, 10 warps.  fp8 weights: 3 stages of 64 KB
 // (x, bf16 operand, e4m3 staging) and 8 more warps converting e4m3 to bf16.
-template <bool FP8> struct Cfg {
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + (FP8 ? E4_BYTES : 0);
-  static constexpr int STAGES = FP8 ? 3 : 4;
+// AdaLN (bf16 weights): 3 stages of 64 KB (raw x, modulated x, weight).
+template <bool FP8, bool ADALN = false> struct Cfg {
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + (FP8 ? E4_BYTES : 0) + (ADALN ? A_BYTES : 0);
+  static constexpr int STAGES = FP8 || ADALN ? 3 : 4;
   static constexpr int NUM_THREADS = FP8 ? 576 : 320;
 };
 constexpr int GROUP_M = 16;                     // tile raster: bands of 16 row blocks
@@ -70,12 +81,16 @@ struct Params {
   uint8_t* ysf;          //   and e4m3 scale codes [M][nout / 16]
   const float* gscale;   //   global scale (one fp32 value in device memory)
   float* part_out;       // partial output: fp32 [M][ncols] accumulators, then [M] sums of squares
+  const float* ad_scale; // AdaLN: scale rows fp32 [n_cond][d]
+  const float* ad_bias;  //   shift bias rows fp32 [n_cond][ncols] (the shift times the unfolded weight)
+  const int* ad_index;   //   per-token condition index [M]
+  int n_cond;
 };
 
 template <int STAGES>
 struct alignas(8) Bars {
   uint64_t full[STAGES], empty[STAGES];
-  uint64_t conv[STAGES];   // fp8: the stage's weight tile has been converted to bf16
+  uint64_t conv[STAGES];   // fp8: the stage's weight tile has been converted to bf16; AdaLN: x modulated
   uint64_t acc_full[2], acc_empty[2];
   uint64_t ssq_full[2], ssq_empty[2];
   uint64_t drain;
@@ -84,11 +99,49 @@ struct alignas(8) Bars {
   int abort_flag;
 };
 
-template <bool FP8>
+template <bool FP8, bool ADALN = false>
 constexpr size_t smem_bytes() {
-  return 1024 + Cfg<FP8>::STAGES * Cfg<FP8>::STAGE_BYTES + sizeof(Bars<Cfg<FP8>::STAGES>);
+  return 1024 + Cfg<FP8, ADALN>::STAGES * Cfg<FP8, ADALN>::STAGE_BYTES + sizeof(Bars<Cfg<FP8, ADALN>::STAGES>);
 }
-static_assert(smem_bytes<true>() <= 232448 && smem_bytes<false>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<true>() <= 232448 && smem_bytes<false>() <= 232448 && smem_bytes<false, true>() <= 232448,
+              "shared memory budget");
+
+// AdaLN: condition of tile row `grow`, or -1 for an index outside [0, n_cond)
+// (that row's outputs become NaN; padding rows past M take condition 0).
+__device__ __forceinline__ int adaln_cond(const Params& p, int grow) {
+  if (grow >= p.M) return 0;
+  const int c = __ldg(p.ad_index + grow);
+  return (c >= 0 && c < p.n_cond) ? c : -1;
+}
+
+// AdaLN: one staged x row (64 bf16, 128-byte swizzle) times the row's scale
+// values s[k0 .. k0+63], each product rounded once to bf16, written to the same
+// swizzled positions of the modulated operand tile.  srow is null for an
+// invalid condition (the products become NaN).
+__device__ __forceinline__ void modulate_row_sw128(const uint8_t* tile, uint8_t* mod, int row, const float* srow) {
+  const uint8_t* src = tile + row * 128;
+  uint8_t* dst = mod + row * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const int off = (c ^ (row & 7)) << 4;
+    const uint4 v = *reinterpret_cast<const uint4*>(src + off);
+    float4 s0, s1;
+    if (srow) {
+      s0 = __ldg(reinterpret_cast<const float4*>(srow + 8 * c));
+      s1 = __ldg(reinterpret_cast<const float4*>(srow + 8 * c + 4));
+    } else {
+      s0 = s1 = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                            __int_as_float(0x7fc00000));
+    }
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      o[j] = pack_bf16x2(bf16lo_to_f32(w[j]) * sv[2 * j], bf16hi_to_f32(w[j]) * sv[2 * j + 1]);
+    *reinterpret_cast<uint4*>(dst + off) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
   const int per_group = GROUP_M * p.num_n;
@@ -110,19 +163,21 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
 }
 
 // OUT: bf16 y, NVFP4 codes and scales (SwiGLU only), or fp32 partials (OutKind).
-template <bool SWIGLU, bool FP8, int OUT = kOutBf16>
-__global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
+template <bool SWIGLU, bool FP8, int OUT = kOutBf16, bool ADALN = false>
+__global__ void __launch_bounds__(Cfg<FP8, ADALN>::NUM_THREADS, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
               const Params p) {
   static_assert(OUT != kOutNvfp4 || SWIGLU, "NVFP4 output is a SwiGLU epilogue");
-  constexpr int STAGES = Cfg<FP8>::STAGES;
-  constexpr int STAGE_BYTES = Cfg<FP8>::STAGE_BYTES;
+  static_assert(!ADALN || (!FP8 && OUT == kOutBf16), "AdaLN: bf16 weights and bf16 output");
+  constexpr int STAGES = Cfg<FP8, ADALN>::STAGES;
+  constexpr int STAGE_BYTES = Cfg<FP8, ADALN>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars<STAGES>& bars = *reinterpret_cast<Bars<STAGES>*>(smem + STAGES * STAGE_BYTES);
   auto stage_a = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stage_b = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
   auto stage_e4 = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B_BYTES; };
+  auto stage_am = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B_BYTES; };   // AdaLN: modulated x
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -131,7 +186,7 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1 + 4);  // MMA commit + one arrival per reducer warp
-      mbar_init(&bars.conv[s], 256);     // fp8: every converter thread
+      mbar_init(&bars.conv[s], ADALN ? 4 : 256);   // fp8: every converter thread; AdaLN: the reducer warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
@@ -209,9 +264,9 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
         const uint32_t d_tmem = tmem_base + b * BN;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
-          if (FP8 && !mbar_wait(&bars.conv[s], ph, ctl, kSiteMmaConv)) { ok = false; break; }
+          if ((FP8 || ADALN) && !mbar_wait(&bars.conv[s], ph, ctl, kSiteMmaConv)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(stage_a(s));
+          const uint32_t a0 = smem_u32(ADALN ? stage_am(s) : stage_a(s));
           const uint32_t b0 = smem_u32(stage_b(s));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
@@ -276,9 +331,22 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++i) {
       float acc = 0.f;
+      const float* srow = nullptr;   // AdaLN: this row's scale row
+      if constexpr (ADALN) {
+        int mb, nb;
+        tile_coords(t, p, mb, nb);
+        const int c = adaln_cond(p, mb * BM + row);
+        srow = c >= 0 ? p.ad_scale + static_cast<int64_t>(c) * p.d : nullptr;
+      }
       for (int kb = 0; kb < p.kblocks; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[s], ph, ctl, kSiteRedFull))) { ok = false; break; }
         acc += row_sumsq_sw128(stage_a(s), row);
+        if constexpr (ADALN) {
+          modulate_row_sw128(stage_a(s), stage_am(s), row, srow ? srow + kb * BK : nullptr);
+          fence_proxy_async_smem();   // generic-proxy operand writes -> visible to tcgen05.mma
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.conv[s]);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.empty[s]);
         if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -362,17 +430,41 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
               make_uint2(static_cast<uint32_t>(sfw), static_cast<uint32_t>(sfw >> 32));
       } else if constexpr (SWIGLU) {
         __nv_bfloat16* yrow = p.y + static_cast<int64_t>(grow) * p.nout + nb * (BN / 2);
+        // AdaLN: the row's shift bias in stored column order (gate 128 | up 128)
+        const float* brow = nullptr;
+        if constexpr (ADALN) {
+          const int cnd = adaln_cond(p, grow);
+          brow = cnd >= 0 ? p.ad_bias + static_cast<int64_t>(cnd) * p.ncols + nb * BN : nullptr;
+        }
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
           uint32_t gv[32], uv[32];
           tmem_ld32(taddr + c, gv);
           tmem_ld32(taddr + BN / 2 + c, uv);
           tmem_ld_wait();
+          float bg[32], bu[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) bg[j] = bu[j] = 0.f;
+          if constexpr (ADALN) {
+            if (brow && row_ok) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(brow + c) + j);
+                const float4 b = __ldg(reinterpret_cast<const float4*>(brow + BN / 2 + c) + j);
+                bg[4 * j] = a.x; bg[4 * j + 1] = a.y; bg[4 * j + 2] = a.z; bg[4 * j + 3] = a.w;
+                bu[4 * j] = b.x; bu[4 * j + 1] = b.y; bu[4 * j + 2] = b.z; bu[4 * j + 3] = b.w;
+              }
+            }
+          }
           uint32_t o[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float g0 = __uint_as_float(gv[2 * j]) * r, g1 = __uint_as_float(gv[2 * j + 1]) * r;
-            const float u0 = __uint_as_float(uv[2 * j]) * r, u1 = __uint_as_float(uv[2 * j + 1]) * r;
+            float g0 = __uint_as_float(gv[2 * j]) * r, g1 = __uint_as_float(gv[2 * j + 1]) * r;
+            float u0 = __uint_as_float(uv[2 * j]) * r, u1 = __uint_as_float(uv[2 * j + 1]) * r;
+            if constexpr (ADALN) {
+              g0 += bg[2 * j]; g1 += bg[2 * j + 1];
+              u0 += bu[2 * j]; u1 += bu[2 * j + 1];
+            }
             o[j] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
           }
           if (row_ok) {
@@ -383,6 +475,11 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
         }
       } else {
         __nv_bfloat16* yrow = p.y + static_cast<int64_t>(grow) * p.nout;
+        const float* brow = nullptr;   // AdaLN: the row's shift bias
+        if constexpr (ADALN) {
+          const int cnd = adaln_cond(p, grow);
+          brow = cnd >= 0 ? p.ad_bias + static_cast<int64_t>(cnd) * p.ncols : nullptr;
+        }
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t v[32];
@@ -390,10 +487,22 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
           tmem_ld_wait();
           const int col = nb * BN + c;
           if (row_ok && col < p.nout) {
+            float bv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) bv[j] = 0.f;
+            if constexpr (ADALN) {
+              if (brow) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float4 a = __ldg(reinterpret_cast<const float4*>(brow + col) + j);
+                  bv[4 * j] = a.x; bv[4 * j + 1] = a.y; bv[4 * j + 2] = a.z; bv[4 * j + 3] = a.w;
+                }
+              }
+            }
             uint32_t o[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              o[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * r, __uint_as_float(v[2 * j + 1]) * r);
+              o[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * r + bv[2 * j], __uint_as_float(v[2 * j + 1]) * r + bv[2 * j + 1]);
             uint4* dst = reinterpret_cast<uint4*>(yrow + col);
 #pragma unroll
             for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
@@ -413,7 +522,7 @@ __global__ void __launch_bounds__(Cfg<FP8>::NUM_THREADS, 1)
   }
 }
 
-template <bool SWIGLU, bool FP8, int OUT = kOutBf16>
+template <bool SWIGLU, bool FP8, int OUT = kOutBf16, bool ADALN = false>
 cudaError_t launch_impl(const CallArgs& a) {
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, BM, BK)) return cudaErrorInvalidValue;
@@ -443,16 +552,23 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.ysf = static_cast<uint8_t*>(a.ysf);
   p.gscale = a.gscale;
   p.part_out = a.part_out;
-  constexpr size_t SMEM_BYTES = smem_bytes<FP8>();
-  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU, FP8, OUT>>(static_cast<int>(SMEM_BYTES));
+  p.ad_scale = a.ad_scale;
+  p.ad_bias = a.ad_bias;
+  p.ad_index = a.ad_index;
+  p.n_cond = static_cast<int>(a.n_cond);
+  constexpr size_t SMEM_BYTES = smem_bytes<FP8, ADALN>();
+  cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU, FP8, OUT, ADALN>>(static_cast<int>(SMEM_BYTES));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
-  return launch_pdl(tc_kernel<SWIGLU, FP8, OUT>, grid, Cfg<FP8>::NUM_THREADS, SMEM_BYTES, a.stream, tx, tw, p);
+  return launch_pdl(tc_kernel<SWIGLU, FP8, OUT, ADALN>, grid, Cfg<FP8, ADALN>::NUM_THREADS, SMEM_BYTES, a.stream, tx,
+                    tw, p);
 }
 
 }  // namespace tc
 
 cudaError_t launch_tc(const CallArgs& a) {
+  if (a.ad_index)   // AdaLN: bf16 weights (other types were converted to bf16 first), bf16 output
+    return a.swiglu ? tc::launch_impl<true, false, kOutBf16, true>(a) : tc::launch_impl<false, false, kOutBf16, true>(a);
   if (a.yq) return a.wtype == 1 ? tc::launch_impl<true, true, kOutNvfp4>(a) : tc::launch_impl<true, false, kOutNvfp4>(a);
   // partial output: no activation, so every weight is a plain projection of its stored columns
   if (a.part_out)

@@ -7,7 +7,8 @@ from typing import Optional, Tuple
 
 import torch
 
-from . import (FN_W_BF16, FN_W_FP8_E4M3_B128, FN_W_MXFP8_E4M3, check, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
+from . import (FN_W_BF16, FN_W_FP8_E4M3_B128, FN_W_MXFP8_E4M3, check, fn_adaln_shift_bias, fn_norm_proj_adaln,
+               fn_workspace_size_adaln, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
                fn_norm_proj_partial, fn_norm_proj_swiglu_nvfp4, fn_post_scale, fn_query_device_status,
                fn_workspace_size)
 
@@ -114,4 +115,34 @@ def post_scale(partial: torch.Tensor, M: int, N: int, d_total: int, eps: float, 
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=partial.device)
     check(fn_post_scale(partial, M, N, int(swiglu), d_total, eps, out, stream), "fn_post_scale")
+    return out
+
+
+def adaln_shift_bias(shift: torch.Tensor, W0: torch.Tensor, W1: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """fp32 [n_cond, ncols]: the AdaLN shift rows through the unfolded weight."""
+    n_cond, d = shift.shape
+    N = W0.shape[1]
+    ncols = 2 * N if W1 is not None else N
+    B = torch.empty((n_cond, ncols), dtype=torch.float32, device=shift.device)
+    check(fn_adaln_shift_bias(shift, n_cond, W0, W1, d, N, B, stream), "fn_adaln_shift_bias")
+    return B
+
+
+def norm_proj_adaln(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float, adaln_scale: torch.Tensor,
+                    shift_bias: torch.Tensor, adaln_index: torch.Tensor, swiglu: bool = False,
+                    scales: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The AdaLN-modulated fused call (see fn_norm_proj_adaln)."""
+    M, d = x.shape
+    wt = weight_type(Wp, scales)
+    if ws is None:
+        ws = Workspace(x.device)
+    need = fn_workspace_size_adaln(d, N, wt, int(swiglu))
+    if ws.buf.numel() < need:
+        ws.buf = torch.zeros(need, dtype=torch.uint8, device=ws.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    check(fn_norm_proj_adaln(x, M, d, Wp, scales, wt, N, int(swiglu), eps, adaln_scale, shift_bias, adaln_index,
+                             adaln_scale.shape[0], out, ws.buf, ws.buf.numel(), stream), "fn_norm_proj_adaln")
     return out

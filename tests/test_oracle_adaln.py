@@ -116,6 +116,18 @@ def test_adaln_rows_permute_with_their_index():
     assert np.array_equal(yp, y[perm])
 
 
+def test_adaln_scaled_operand_matches_torch_casts():
+    """fp32 product then one round-to-nearest-even to bf16, checked against
+    torch's own fp32 multiply and bf16 cast on the CPU."""
+    import torch
+    x = WL.activations(8, 256, 9)
+    rng = np.random.default_rng(9)
+    scale = (1.0 + 0.3 * rng.standard_normal((3, 256))).astype(np.float32)
+    index = rng.integers(0, 3, 8)
+    want = (x.float() * torch.from_numpy(scale)[torch.from_numpy(index)]).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.adaln_scaled_operand(x, scale, index), want)
+
+
 @pytest.mark.parametrize("mistake", ["shift_before_norm", "scale_dropped", "gain_on_shift", "index_off_by_one"])
 def test_adaln_planted_mistakes_are_caught(mistake, monkeypatch):
     def wrong(x, g, eps, scale, shift, index):
