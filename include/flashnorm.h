@@ -237,6 +237,22 @@ fn_status fn_norm_proj_adaln(const void* x, int64_t M, int64_t d, const void* Wp
 size_t fn_workspace_size_adaln(int64_t d, int64_t N, fn_wtype wt, int swiglu);
 
 /*
+ * fn_norm_proj_swiglu_nvfp4_swizzled — fn_norm_proj_swiglu_nvfp4 with the
+ * scale bytes in the layout block-scaled tensor-core GEMMs read directly (the
+ * "swizzled" scale factors, is_swizzled, of the FlashInfer PR #4040 analysis),
+ * so the down projection needs no re-layout pass.  Codes as
+ * fn_norm_proj_swiglu_nvfp4.  out_sf holds ceil(M/128)*128 * N/16 bytes: rows
+ * in blocks of 128 and scale columns (one per 16 output columns) in groups of
+ * 4 form 512-byte chunks; chunk (m div 128, j div 4) sits at byte
+ * 512 * ((m div 128) * (N/64) + j div 4), and inside it the scale of row m,
+ * column j at 16*(m mod 32) + 4*((m mod 128) div 32) + (j mod 4).  Bytes of
+ * the padding rows (M .. ceil(M/128)*128 - 1) are not written.
+ */
+fn_status fn_norm_proj_swiglu_nvfp4_swizzled(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                                             fn_wtype wt, int64_t N, float eps, const float* global_scale, void* out_q,
+                                             void* out_sf, void* workspace, size_t ws_bytes, fn_stream_t stream);
+
+/*
  * Row-parallel (d-split) projection, for tensor parallelism that shards the
  * input width d across ranks.  The deferred normalisation (FlashNorm talk
  * summary, Proposal 2) makes 1/rms a per-row factor applied after the matmul,

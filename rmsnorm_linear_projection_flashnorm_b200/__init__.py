@@ -45,6 +45,8 @@ _SIGNATURES = {
     "fn_norm_proj_swiglu": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp, _sz, _vp]),
     "fn_norm_proj_swiglu_nvfp4": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp, _vp, _vp, _sz,
                                          _vp]),
+    "fn_norm_proj_swiglu_nvfp4_swizzled": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp, _vp, _vp,
+                                                  _sz, _vp]),
     "fn_norm_proj_partial": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _vp, _vp, _sz, _vp]),
     "fn_post_scale": (_int, [_vp, _i64, _i64, _int, _i64, _f32, _vp, _vp]),
     "fn_norm_proj_static": (_int, [_vp, _i64, _i64, _vp, _vp, _int, _i64, _f32, _vp, _vp]),
@@ -210,3 +212,10 @@ def fn_norm_proj_adaln(x, M: int, d: int, Wp, scales, wt: int, N: int, swiglu: i
 
 def fn_workspace_size_adaln(d: int, N: int, wt: int = FN_W_BF16, swiglu: int = 0) -> int:
     return lib().fn_workspace_size_adaln(d, N, wt, int(swiglu))
+
+
+def fn_norm_proj_swiglu_nvfp4_swizzled(x, M: int, d: int, Wp, scales, wt: int, N: int, eps: float, global_scale,
+                                       out_q, out_sf, workspace, ws_bytes: int, stream=None) -> int:
+    return lib().fn_norm_proj_swiglu_nvfp4_swizzled(_ptr(x), M, d, _ptr(Wp), _ptr(scales), wt, N, eps,
+                                                    _ptr(global_scale), _ptr(out_q), _ptr(out_sf), _ptr(workspace),
+                                                    ws_bytes, _stream(stream))

@@ -129,7 +129,7 @@ struct AdaLN {
 fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
                            int64_t N, float eps, void* y, void* ws, size_t ws_bytes, fn_stream_t stream,
                            bool swiglu, void* yq = nullptr, void* ysf = nullptr, const float* gscale = nullptr,
-                           float* part_out = nullptr, const AdaLN& ad = AdaLN()) {
+                           float* part_out = nullptr, const AdaLN& ad = AdaLN(), bool sf_chunked = false) {
   const bool adaln = ad.index != nullptr || ad.scale != nullptr || ad.bias != nullptr;
   const bool fp4 = yq != nullptr || ysf != nullptr || gscale != nullptr;
   const bool partial = part_out != nullptr;
@@ -168,7 +168,8 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   if (overlaps(ws, ws_bytes, x, xbytes) || overlaps(ws, ws_bytes, Wp, wbytes) || overlaps(ws, ws_bytes, scales, sbytes))
     return FN_ERR_ALIAS;
   // every output region against every input region, the workspace and each other
-  const size_t qbytes = static_cast<size_t>(M) * (N / 2), fbytes = static_cast<size_t>(M) * (N / 16);
+  const size_t qbytes = static_cast<size_t>(M) * (N / 2);
+  const size_t fbytes = static_cast<size_t>(sf_chunked ? (M + 127) / 128 * 128 : M) * (N / 16);
   const size_t pbytes = partial ? (static_cast<size_t>(M) * ncols + M) * 4 : 0;
   const struct { const void* p; size_t n; } outs[4] = {{y, ybytes}, {yq, qbytes}, {ysf, fbytes}, {part_out, pbytes}};
   const size_t adsb = adaln ? static_cast<size_t>(ad.n_cond) * d * 4 : 0;
@@ -223,6 +224,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.y = y;
   a.yq = yq;
   a.ysf = ysf;
+  a.sf_chunked = sf_chunked ? 1 : 0;
   a.gscale = gscale;
   a.part_out = part_out;
   a.ws = ws;
@@ -320,6 +322,14 @@ fn_status fn_norm_proj_swiglu_nvfp4(const void* x, int64_t M, int64_t d, const v
   if (M > 0 && (!out_q || !out_sf || !global_scale)) return FN_ERR_INVALID_ARG;
   return norm_proj_common(x, M, d, Wp, scales, wt, N, eps, nullptr, workspace, ws_bytes, stream, true, out_q,
                           out_sf, global_scale);
+}
+
+fn_status fn_norm_proj_swiglu_nvfp4_swizzled(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,
+                                             fn_wtype wt, int64_t N, float eps, const float* global_scale, void* out_q,
+                                             void* out_sf, void* workspace, size_t ws_bytes, fn_stream_t stream) {
+  if (M > 0 && (!out_q || !out_sf || !global_scale)) return FN_ERR_INVALID_ARG;
+  return norm_proj_common(x, M, d, Wp, scales, wt, N, eps, nullptr, workspace, ws_bytes, stream, true, out_q,
+                          out_sf, global_scale, nullptr, AdaLN(), true);
 }
 
 fn_status fn_norm_proj_partial(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales,

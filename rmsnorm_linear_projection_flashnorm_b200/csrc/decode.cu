@@ -507,6 +507,7 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.xfac = nullptr;
   p.yq = static_cast<uint8_t*>(a.yq);
   p.ysf = static_cast<uint8_t*>(a.ysf);
+  p.sf_chunked = a.sf_chunked;
   p.gscale = a.gscale;
   p.part_out = a.part_out;
   p.wsf = nullptr;

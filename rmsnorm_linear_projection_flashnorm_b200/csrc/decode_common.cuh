@@ -54,6 +54,7 @@ struct Params {
   float* part_out;           // partial output: fp32 [M][ncols] accumulators, then [M] sums of squares
   const uint8_t* wsf;        // MXFP8 weights: ue8m0 scale chunks (k groups, then 128-column blocks)
   uint8_t* xsf;              // MXFP8 path, x split once per call: ue8m0 scale chunk per k group
+  int sf_chunked;            // NVFP4 output: scale bytes in the 128x4 chunked layout (else row-major)
 };
 
 // One partial-result slot: float4 groups [half][row / 4][column] for the
@@ -116,8 +117,8 @@ __device__ __forceinline__ void store_tile_fp4(const uint8_t* qbuf, int mpad, co
       *reinterpret_cast<uint4*>(p.yq + m * qrow + tile * 64 + c * 16) =
           *reinterpret_cast<const uint4*>(qbuf + m * 64 + c * 16);
     } else {
-      *reinterpret_cast<uint2*>(p.ysf + m * srow + tile * 8) =
-          *reinterpret_cast<const uint2*>(qbuf + mpad * 64 + m * 8);
+      fp4_store_sf8(p.ysf, m, tile * 8, static_cast<int>(srow), p.sf_chunked != 0,
+                    *reinterpret_cast<const uint2*>(qbuf + mpad * 64 + m * 8));
     }
   }
 }
@@ -241,7 +242,7 @@ __global__ void __launch_bounds__(FIX_THREADS) decode_fixup_kernel(const Params 
       const uint32_t sf = fp4_quantize_lane16(v, gs, pair);
       if ((n & 1) == 0) p.yq[static_cast<int64_t>(m) * (p.nout / 2) + (col >> 1)] = static_cast<uint8_t>(pair);
       if ((n & 15) == 0)
-        p.ysf[static_cast<int64_t>(m) * (p.nout / kFp4Block) + (col >> 4)] = static_cast<uint8_t>(sf);
+        p.ysf[fp4_sf_offset(m, col >> 4, p.nout / kFp4Block, p.sf_chunked != 0)] = static_cast<uint8_t>(sf);
     } else if (col < p.nout) {
       p.y[static_cast<int64_t>(m) * p.nout + col] = __float2bfloat16_rn(v);
     }

@@ -470,6 +470,7 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.xfac = reinterpret_cast<float*>(p.xsf + static_cast<size_t>(p.kblocks) * SF_CHUNK);
   p.yq = static_cast<uint8_t*>(a.yq);
   p.ysf = static_cast<uint8_t*>(a.ysf);
+  p.sf_chunked = a.sf_chunked;
   p.gscale = a.gscale;
   p.part_out = a.part_out;
   p.wsf = reinterpret_cast<const uint8_t*>(a.scales);

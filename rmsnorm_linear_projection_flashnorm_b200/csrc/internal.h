@@ -35,7 +35,8 @@ struct CallArgs {
   float eps;
   void* y;                // bf16 [M, N] (null with NVFP4 output)
   void* yq;               // NVFP4 output, SwiGLU only: e2m1 codes [M, N/2] bytes, or null
-  void* ysf;              //   e4m3 scale codes [M, N/16]
+  void* ysf;              //   e4m3 scale codes [M, N/16], row-major or chunked (sf_chunked)
+  int sf_chunked;         //   1: the 128x4 chunked scale layout
   const float* gscale;    //   global scale, one fp32 value in device memory
   float* part_out;        // kOutPartial: fp32 [M, ncols] accumulators, then [M] sums of squares
   void* ws;               // workspace (status word + decode scratch)

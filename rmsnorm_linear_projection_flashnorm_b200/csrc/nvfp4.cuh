@@ -10,7 +10,9 @@
 //   q    = RN_e2m1_satfinite(v * (gs / sf))        all zero when sf is zero
 // A block holding a non-finite value gets the e4m3 NaN code 0x7F and zero
 // codes.  Dequantised: e2m1(q) * e4m3(sf) / gs.  Two codes per byte with the
-// even column in the low nibble; scale codes row-major [M, N / 16].
+// even column in the low nibble; scale codes row-major [M, N / 16], or in the
+// 128 x 4 chunked layout that block-scaled tensor-core GEMMs read (the
+// "swizzled" scale factors of the PR #4040 analysis, fp4_sf_offset).
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -18,6 +20,27 @@
 namespace fn {
 
 constexpr int kFp4Block = 16;
+
+// Byte offset of the scale of row m, block j (C = N / 16 scale columns, a
+// multiple of 8): row-major, or chunked: rows in blocks of 128 and scale
+// columns in groups of 4 make 512-byte chunks, chunk (m / 128, j / 4) at
+// 512 * ((m / 128) * (C / 4) + j / 4), and inside a chunk row m, column j at
+// 16 * (m mod 32) + 4 * ((m mod 128) / 32) + (j mod 4).
+__device__ __forceinline__ int64_t fp4_sf_offset(int64_t m, int j, int C, bool chunked) {
+  if (!chunked) return m * C + j;
+  return 512 * ((m >> 7) * (C >> 2) + (j >> 2)) + 16 * (m & 31) + 4 * ((m & 127) >> 5) + (j & 3);
+}
+
+// The 8 scale bytes of row m, blocks j0 .. j0+7 (j0 a multiple of 8): one
+// 8-byte store row-major, two 4-byte stores chunked.
+__device__ __forceinline__ void fp4_store_sf8(uint8_t* ysf, int64_t m, int j0, int C, bool chunked, uint2 v) {
+  if (!chunked) {
+    *reinterpret_cast<uint2*>(ysf + m * C + j0) = v;
+    return;
+  }
+  *reinterpret_cast<uint32_t*>(ysf + fp4_sf_offset(m, j0, C, true)) = v.x;
+  *reinterpret_cast<uint32_t*>(ysf + fp4_sf_offset(m, j0 + 4, C, true)) = v.y;
+}
 
 // |v| as a bit pattern.  The unsigned maximum of these orders finite values by
 // magnitude and ranks inf and NaN above every finite value.

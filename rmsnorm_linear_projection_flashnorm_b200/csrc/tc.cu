@@ -85,6 +85,7 @@ struct Params {
   const float* ad_bias;  //   shift bias rows fp32 [n_cond][ncols] (the shift times the unfolded weight)
   const int* ad_index;   //   per-token condition index [M]
   int n_cond;
+  int sf_chunked;        // NVFP4 output: scale bytes in the 128x4 chunked layout (else row-major)
 };
 
 template <int STAGES>
@@ -426,8 +427,8 @@ __global__ void __launch_bounds__(Cfg<FP8, ADALN>::NUM_THREADS, 1)
           if (row_ok) *reinterpret_cast<uint4*>(qrow + c / 2) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         if (row_ok)
-          *reinterpret_cast<uint2*>(p.ysf + static_cast<int64_t>(grow) * (p.nout / kFp4Block) + nb * (BN / 32)) =
-              make_uint2(static_cast<uint32_t>(sfw), static_cast<uint32_t>(sfw >> 32));
+          fp4_store_sf8(p.ysf, grow, nb * (BN / 32), p.nout / kFp4Block, p.sf_chunked != 0,
+                        make_uint2(static_cast<uint32_t>(sfw), static_cast<uint32_t>(sfw >> 32)));
       } else if constexpr (SWIGLU) {
         __nv_bfloat16* yrow = p.y + static_cast<int64_t>(grow) * p.nout + nb * (BN / 2);
         // AdaLN: the row's shift bias in stored column order (gate 128 | up 128)
@@ -556,6 +557,7 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.ad_bias = a.ad_bias;
   p.ad_index = a.ad_index;
   p.n_cond = static_cast<int>(a.n_cond);
+  p.sf_chunked = a.sf_chunked;
   constexpr size_t SMEM_BYTES = smem_bytes<FP8, ADALN>();
   cudaError_t e = ensure_smem_limit<tc_kernel<SWIGLU, FP8, OUT, ADALN>>(static_cast<int>(SMEM_BYTES));
   if (e != cudaSuccess) return e;

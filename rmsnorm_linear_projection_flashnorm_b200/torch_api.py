@@ -8,7 +8,7 @@ from typing import Optional, Tuple
 import torch
 
 from . import (FN_W_BF16, FN_W_FP8_E4M3_B128, FN_W_MXFP8_E4M3, check, fn_adaln_shift_bias, fn_norm_proj_adaln,
-               fn_workspace_size_adaln, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
+               fn_norm_proj_swiglu_nvfp4_swizzled, fn_workspace_size_adaln, fn_fold_weights, fn_norm_proj, fn_norm_proj_swiglu,
                fn_norm_proj_partial, fn_norm_proj_swiglu_nvfp4, fn_post_scale, fn_query_device_status,
                fn_workspace_size)
 
@@ -90,6 +90,24 @@ def norm_proj_swiglu_nvfp4(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float
     q, sf = out
     check(fn_norm_proj_swiglu_nvfp4(x, M, d, Wp, scales, wt, N, eps, global_scale, q, sf, buf, buf.numel(), stream),
           "fn_norm_proj_swiglu_nvfp4")
+    return q, sf
+
+
+def norm_proj_swiglu_nvfp4_swizzled(x: torch.Tensor, Wp: torch.Tensor, N: int, eps: float,
+                                    global_scale: torch.Tensor, scales: Optional[torch.Tensor] = None,
+                                    ws: Optional[Workspace] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """SwiGLU output in NVFP4 with the scale bytes in the chunked (swizzled)
+    layout: (codes uint8 [M, N/2], scale bytes uint8 [ceil(M/128)*128 * N/16],
+    zero-initialised so the padding rows read as 0)."""
+    M, d = x.shape
+    wt = weight_type(Wp, scales)
+    if ws is None:
+        ws = Workspace(x.device)
+    buf = ws.get(M, d, N, wt, True)
+    q = torch.empty((M, N // 2), dtype=torch.uint8, device=x.device)
+    sf = torch.zeros(((M + 127) // 128) * 128 * (N // 16), dtype=torch.uint8, device=x.device)
+    check(fn_norm_proj_swiglu_nvfp4_swizzled(x, M, d, Wp, scales, wt, N, eps, global_scale, q, sf, buf, buf.numel(),
+                                             stream), "fn_norm_proj_swiglu_nvfp4_swizzled")
     return q, sf
 
 

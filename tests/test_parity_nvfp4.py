@@ -188,3 +188,35 @@ def test_nvfp4_fp8_workload(fp8_workload, M):
     gs = _gs_for(ref)
     q, sf = _run_nvfp4({"x": x, "eps": inp["eps"]}, Wq, s, w.N, gs)
     assert check_nvfp4(q, sf, ref, gs, FP8_TOL) > 0.99
+
+
+@pytest.mark.parametrize("M,d,N,wt", [
+    (1, 512, 256, 0),        # decode, fix-up kernel writes the scales
+    (5, 256, 19200, 0),      # decode, whole tiles staged and stored by the decode kernel
+    (200, 512, 384, 0),      # tile kernel, ragged M (padding rows of the last 128-row block)
+    (40, 384, 256, FP8),     # fp8 decode
+    (130, 256, 384, FP8),    # fp8 tile kernel
+    (300, 256, 512, 2),      # MXFP8 weights (tile path after the exact bf16 conversion)
+    (17, 256, 512, 2),       # MXFP8 decode
+])
+def test_nvfp4_swizzled_scales(M, d, N, wt):
+    """The swizzled entry point writes the same codes as the row-major one and
+    its scale bytes are exactly the row-major bytes in the oracle's chunked
+    layout (sf_chunk_layout, pinned on CPU); the row-major result itself is
+    checked against the oracle's encoding."""
+    inp = WL.case(M, d, N, True, seed=190 + M)
+    g = inp["g"]
+    Wq, s = T.fold(gpu(inp["W_gate"]), gpu(g), gpu(inp["W_up"]), wtype=wt)
+    gsd = torch.tensor([448.0 * 6.0 / 6.0], dtype=torch.float32, device="cuda")
+    x = gpu(inp["x"])
+    q0, sf0 = T.norm_proj_swiglu_nvfp4(x, Wq, N, inp["eps"], gsd, scales=s)
+    q1, sf1 = T.norm_proj_swiglu_nvfp4_swizzled(x, Wq, N, inp["eps"], gsd, scales=s)
+    torch.cuda.synchronize()
+    assert torch.equal(q0, q1)
+    sf_rm = sf0.cpu().numpy()
+    assert np.array_equal(sf1.cpu().numpy(), O.sf_chunk_layout(sf_rm))
+    assert np.array_equal(O.sf_chunk_unlayout(sf1.cpu().numpy(), M, N // 16), sf_rm)
+    if wt == 0:
+        Wg, Wu = fold_ref_bf16(inp["W_gate"], g), fold_ref_bf16(inp["W_up"], g)
+        ref = O.norm_proj_swiglu(inp["x"], np.ones(d), Wg, Wu, inp["eps"])
+        check_nvfp4(q0.cpu().numpy(), sf_rm, ref, float(gsd.item()), BF16_TOL)
