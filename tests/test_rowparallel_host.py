@@ -37,14 +37,14 @@ def _inputs(M, d, N, swiglu):
     return x, Wg, Wu
 
 
-def _worker(rank, world, port, swiglu, q):
+def _worker(rank, world, port, swiglu, q, exchange="allreduce", M=4):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     sys.path.insert(0, ROOT)
     import oracle as O
     from rmsnorm_linear_projection_flashnorm_b200 import torch_api as T
     from rmsnorm_linear_projection_flashnorm_b200 import tp
-    M, d, N = 4, 384, 256
+    d, N = 384, 256
     x, Wg, Wu = _inputs(M, d, N, swiglu)
     W = O.interleave128(Wg, Wu) if swiglu else Wg
     k0, k1 = tp.rowparallel_slices(d, world, align=64)[rank]
@@ -57,30 +57,35 @@ def _worker(rank, world, port, swiglu, q):
     def post_cpu(part, M_, N_, d_total, eps, swiglu=False):
         p = part.numpy()
         ncols = 2 * N_ if swiglu else N_
-        return O.rowparallel_finish(p[:M_ * ncols].reshape(M_, ncols), p[M_ * ncols:], d_total, eps, swiglu)
+        return torch.from_numpy(O.rowparallel_finish(p[:M_ * ncols].reshape(M_, ncols), p[M_ * ncols:], d_total, eps,
+                                                     swiglu))
 
     T.norm_proj_partial, T.post_scale = partial_cpu, post_cpu   # this worker process only
     y = tp.row_parallel_norm_proj(torch.from_numpy(x[:, k0:k1].copy()), torch.from_numpy(W[k0:k1].copy()), N, 1e-6,
-                                  d, swiglu=swiglu)
-    q.put((rank, (k0, k1), y))
+                                  d, swiglu=swiglu, exchange=exchange)
+    q.put((rank, (k0, k1), y.numpy()))
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,swiglu", [(2, False), (2, True), (3, True)])
-def test_row_parallel_exchange_gives_every_rank_the_full_result(world, swiglu):
+@pytest.mark.parametrize("world,swiglu,exchange,M", [
+    (2, False, "allreduce", 4), (2, True, "allreduce", 4), (3, True, "allreduce", 4),
+    (2, False, "reduce_scatter", 6), (3, True, "reduce_scatter", 6),
+    (3, False, "reduce_scatter", 4),    # M not divisible by the world size: the all-reduce path
+])
+def test_row_parallel_exchange_gives_every_rank_the_full_result(world, swiglu, exchange, M):
     sys.path.insert(0, ROOT)
     import oracle as O
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, swiglu, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, swiglu, q, exchange, M)) for r in range(world)]
     for p in procs:
         p.start()
     out = sorted([q.get(timeout=120) for _ in range(world)], key=lambda t: t[0])
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    M, d, N = 4, 384, 256
+    d, N = 384, 256
     x, Wg, Wu = _inputs(M, d, N, swiglu)
     want = O.norm_proj_swiglu(x, np.ones(d), Wg, Wu, 1e-6) if swiglu else O.norm_proj(x, np.ones(d), Wg, 1e-6)
     spans = [s for _, s, _ in out]
