@@ -476,9 +476,12 @@ def kernel_for(wl: WL.Workload, M: int, out: str):
         sources = [src, "decode_common.cuh", "ptx.cuh", "nvfp4.cuh"]
         label = f"{kname} (+ decode_fixup_kernel where a tile's k range is split)"
     else:
-        kname, sources = "tc_kernel", ["tc.cu", "ptx.cuh", "nvfp4.cuh"]
         once = wl.wtype == "mxfp8_e4m3" or (wl.wtype != "bf16" and M >= 1024)
-        label = "tc_kernel" + (" (after the dequantise-once kernel)" if once else "")
+        # bf16 weights (or a bf16 copy) at M >= 512 with bf16 output run on pairs of SMs
+        pair = (wl.wtype == "bf16" or once) and M >= 512 and out == "bf16"
+        kname = "tc2_kernel" if pair else "tc_kernel"
+        sources = ["tc2.cu" if pair else "tc.cu", "ptx.cuh"] + ([] if pair else ["nvfp4.cuh"])
+        label = kname + (" (after the dequantise-once kernel)" if once else "")
     src_hash = kernel_source_hash(sources)
     prof = f"{kname}_{wl.name}{'_nvfp4' if out == 'nvfp4' else ''}.md"
     return kname, label, src_hash, profile_traffic(prof, src_hash)

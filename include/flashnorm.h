@@ -372,7 +372,8 @@ uint64_t fn_kernel_launches(void);
  *   FN_DEBUG_WAIT_BUDGET_NS   per-wait time limit inside the kernels (default 2e9)
  *   FN_DEBUG_WITHHOLD_ARRIVE  1: the reducers withhold their first arrival, so the
  *                             epilogue's wait must run out (exercises FN_ERR_TIMEOUT)
- *   FN_DEBUG_FORCE_PATH       0 auto, 1 decode kernel (M <= 64 only), 2 tile kernel
+ *   FN_DEBUG_FORCE_PATH       0 auto, 1 decode kernel (M <= 64 only), 2 tile kernel,
+ *                             3 tile kernel on single SMs (never the pair kernel)
  *   FN_DEBUG_PREFETCH         decode path: weight prefetch into L2 before waiting on
  *                             the previous kernel; value = mode | (k_blocks << 8),
  *                             mode 0 off, 1 TMA prefetch, 2 per-thread prefetch

@@ -194,7 +194,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   if (force == 1) {
     if (M > 64 || adaln) return FN_ERR_INVALID_ARG;
     use_decode = true;
-  } else if (force == 2) {
+  } else if (force >= 2) {
     use_decode = false;
   }
 
@@ -236,6 +236,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.prefetch_iters = g_prefetch_iters.load();
   a.prefetch_mode = g_prefetch_mode.load();
   a.cluster_mode = g_cluster_mode.load();
+  a.single_sm_tiles = force == 3 ? 1 : 0;
   a.ad_scale = ad.scale;
   a.ad_bias = ad.bias;
   a.ad_index = ad.index;
@@ -498,7 +499,7 @@ fn_status fn_set_debug(int key, int64_t value) {
       g_withhold.store(value ? 1 : 0);
       return FN_OK;
     case FN_DEBUG_FORCE_PATH:
-      if (value < 0 || value > 2) return FN_ERR_INVALID_ARG;
+      if (value < 0 || value > 3) return FN_ERR_INVALID_ARG;
       g_force_path.store(static_cast<int>(value));
       return FN_OK;
     case FN_DEBUG_CLUSTER:

@@ -48,6 +48,7 @@ struct CallArgs {
   int prefetch_iters;     // decode: weight k-blocks per CTA prefetched into L2 early
   int prefetch_mode;      // decode: 0 none, 1 TMA prefetch, 2 per-thread prefetch
   int cluster_mode;       // decode: 1 allow split-K inside clusters, 0 stream-K only
+  int single_sm_tiles;    // tile path: 1 keeps the one-SM kernel where the pair kernel would run
   const float* ad_scale;  // AdaLN (tile path only): scale rows fp32 [n_cond, d], or null
   const float* ad_bias;   //   shift bias rows fp32 [n_cond, ncols]
   const int* ad_index;    //   condition index per row [M]; null: no AdaLN
@@ -81,6 +82,11 @@ cudaError_t launch_decode_mx(const CallArgs& a, int mpad);
 
 // Tensor-core tile path (M > 64): persistent 128x256 tiles, tcgen05 + TMEM.
 cudaError_t launch_tc(const CallArgs& a);
+// The same on pairs of SMs (2-CTA clusters, 256x256 tiles, cta_group::2 MMAs):
+// bf16 weights, bf16 output, no AdaLN (tc2.cu).
+cudaError_t launch_tc_pair(const CallArgs& a);
+// Rows from which the tile path runs on pairs of SMs.
+constexpr int64_t kPairTileMinM = 512;
 
 // Offline fold and the unfused-chain helper kernels.
 cudaError_t launch_fold_bf16(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wp,

@@ -69,12 +69,14 @@ struct WaitCtl {
   volatile int* abort_flag;   // shared memory, per CTA
   unsigned int* status;       // global status word (first error wins)
   uint64_t budget_ns;         // per-wait limit
+  uint32_t peer_abort = 0;    // CTA pairs: the partner's abort flag (shared::cluster address), or 0
 };
 
 enum : unsigned int { kStatusTimeout = 7u };  // == FN_ERR_TIMEOUT
 
 __device__ __forceinline__ void raise_timeout(const WaitCtl& c, unsigned int site) {
   *c.abort_flag = 1;
+  if (c.peer_abort) asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(c.peer_abort), "r"(1u) : "memory");
   if (c.status) atomicCAS(c.status, 0u, kStatusTimeout | (site << 8));
 }
 
@@ -123,6 +125,42 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
       : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
       : "memory");
   return ok != 0;
+}
+
+// The same test with cluster-scope acquire, for barriers that other CTAs of
+// the cluster arrive on (their earlier writes become visible to this thread).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on a barrier that other CTAs of the cluster arrive on: the
+// phase is polled like any local barrier (see mbar_wait), and one
+// cluster-scope fence after it completes makes the arriving CTAs' earlier
+// writes visible to this thread.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const WaitCtl& c,
+                                                  unsigned int site) {
+  bool ok = mbar_try_wait(bar, parity);
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!ok) {
+      if (mbar_try_wait_suspend(bar, parity, 20000u)) { ok = true; break; }
+      if (*c.abort_flag) return false;
+      if (globaltimer_ns() - t0 > c.budget_ns) {
+        raise_timeout(c, site);
+        return false;
+      }
+    }
+  }
+  asm volatile("fence.acq_rel.cluster;" ::: "memory");
+  return true;
 }
 
 // Wait for the phase with the given parity to complete; false on timeout or
@@ -176,6 +214,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 2D tile load into this CTA's shared memory whose completion is counted on
+// a barrier of the even CTA of a CTA pair (`bar_cluster`, a shared::cluster
+// address from dsmem_addr).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap, uint32_t bar_cluster, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1)
       : "memory");
 }
 
@@ -319,6 +368,54 @@ __device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t lbo_byt
 // later tcgen05.mma instructions; tracked by tcgen05.commit.
 __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Pairs of CTAs (cta_group::2): one MMA spans the tensor cores of both SMs of
+// a 2-CTA cluster.  TMEM allocation and release are executed by the same warp
+// in both CTAs; the leader (rank 0) issues the MMAs; a commit can arrive on
+// the barrier at the same offset in both CTAs.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* holder_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_u32(holder_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem of both CTAs] * B[smem of both CTAs]:
+// M = 256 rows (128 from each CTA's A), N columns (N/2 from each CTA's B),
+// each CTA's TMEM receiving its own 128 rows x N.  Leader only.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the barrier at `bar`'s offset in every CTA of `cta_mask`
+// when this thread's earlier pair MMAs have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               ::"r"(smem_u32(bar)), "h"(cta_mask) : "memory");
+}
+
+// Arrive on a barrier of another CTA of the cluster (address from
+// dsmem_addr), releasing this thread's earlier writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Store to another CTA's shared memory.
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // Arrive once on `bar` when all previously issued tcgen05 operations of this

@@ -572,6 +572,8 @@ cudaError_t launch_tc(const CallArgs& a) {
   if (a.ad_index)   // AdaLN: bf16 weights (other types were converted to bf16 first), bf16 output
     return a.swiglu ? tc::launch_impl<true, false, kOutBf16, true>(a) : tc::launch_impl<false, false, kOutBf16, true>(a);
   if (a.yq) return a.wtype == 1 ? tc::launch_impl<true, true, kOutNvfp4>(a) : tc::launch_impl<true, false, kOutNvfp4>(a);
+  // bf16 weights and output at large M: the kernel on pairs of SMs
+  if (!a.yq && !a.part_out && a.wtype == 0 && a.M >= kPairTileMinM && !a.single_sm_tiles) return launch_tc_pair(a);
   // partial output: no activation, so every weight is a plain projection of its stored columns
   if (a.part_out)
     return a.wtype == 1 ? tc::launch_impl<false, true, kOutPartial>(a) : tc::launch_impl<false, false, kOutPartial>(a);
