@@ -475,6 +475,10 @@ def kernel_for(wl: WL.Workload, M: int, out: str):
                       "mxfp8_e4m3": ("decode_mx_kernel", "decode_mx.cu")}[wl.wtype]
         sources = [src, "decode_common.cuh", "ptx.cuh", "nvfp4.cuh"]
         label = f"{kname} (+ decode_fixup_kernel where a tile's k range is split)"
+    elif wl.wtype == "fp8_e4m3_b128" and out == "bf16":
+        # x split once per call, then the block-scale promotion kernel
+        kname, sources = "tc8_kernel", ["tc8.cu", "ptx.cuh"]
+        label = "tc8_kernel (after xsplit_rows_kernel)"
     else:
         once = wl.wtype == "mxfp8_e4m3" or (wl.wtype != "bf16" and M >= 1024)
         # bf16 weights (or a bf16 copy) at M >= 512 with bf16 output run on pairs of SMs

@@ -115,10 +115,12 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
  * M <= 64, the per-CTA partial sums of the split-K decode path; with fp8
  * weights and 17 <= M <= 64 also the activations split once per call into
  * the two e4m3 operand parts (2 x 64 x d bytes at most) with their scale
- * factors and per-block sums of squares; with fp8 weights and M >= 1024 one
- * bf16 copy of the weight, converted once per call with the same rounding the
- * on-chip conversion uses (bf16(fp32(q) * s)), because converting each weight
- * tile once per 128-row tile would repeat that work M/128 times; with MXFP8
+ * factors and per-block sums of squares; with fp8 weights and M > 64 the
+ * activations split once per call for the block-scale promotion kernel
+ * (2 M d bytes of e4m3 codes, 4 bytes per row and 128-deep k block, 4 bytes
+ * per row), and at M >= 1024 at least one bf16 copy of the weight (2 d ncols
+ * bytes), which the NVFP4 and partial-output calls convert once per call with
+ * the rounding of the on-chip conversion (bf16(fp32(q) * s)); with MXFP8
  * weights the same bf16 copy at every M > 64, and at M <= 64 the activations
  * split once per call (2 x 64 x d bytes at most, their scale chunks and
  * per-group sums of squares).  Zero it once
@@ -141,7 +143,11 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
  *   M == 0 is a no-op.  M <= 64 runs the split-K decode kernel (plus a small
  *   fix-up kernel for the column tiles whose k range it split), larger M the
  *   tensor-core tile kernel; both are deterministic (repeated calls with the
- *   same inputs give the same bits).  MXFP8 weights: at M <= 64 the e4m3
+ *   same inputs give the same bits).  fp8 weights at M > 64: the stored
+ *   e4m3 codes go to the tensor cores as they are, against the activations
+ *   split exactly into two e4m3 parts per row and 128-deep k block (one
+ *   power-of-two scale each); each k block's exact sums are scaled by the
+ *   block scale and added to fp32 sums in k order.  MXFP8 weights: at M <= 64 the e4m3
  *   codes and their scales go to block-scaled MMAs as stored (the bf16
  *   activations split exactly into two e4m3 parts sharing one power-of-two
  *   scale per 32 k values); at M > 64 the weight is converted to bf16 once per
@@ -304,17 +310,17 @@ fn_status fn_post_scale(const float* partial, int64_t M, int64_t N, int swiglu, 
  * because it can synchronise the device.  The pages have no counterpart of
  * this entry point; it only moves the scratch memory.
  *   Arguments, layout and results as fn_norm_proj, minus the workspace.  The
- *   call's scratch (status word, split-K partials, and for fp8 weights at
- *   17..64 rows the activations split once per call) lives in a fixed 8 MiB
- *   array inside the library that every GPU loading the library holds until
- *   the process exits.  A shape is served exactly when
- *   fn_workspace_size(M, d, N, wt, 0) <= 8 MiB; larger ones are rejected with
- *   FN_ERR_WORKSPACE before any launch.  On a 148-SM B200 that admits bf16
- *   weights at every M > 64 and at M <= 32, M in 33..64 while the split-K
- *   partials stay under 8 MiB, and fp8 weights at M <= 64 and 65..1023 under
- *   the same rule; fp8 weights at M >= 1024 need a bf16 copy of the weight
- *   (2 d N bytes) in the scratch and are rejected for any weight over 4 Mi
- *   elements.
+ *   call's scratch (status word, split-K partials, and for fp8 weights the
+ *   activations split once per call) lives in a fixed 8 MiB array inside the
+ *   library that every GPU loading the library holds until the process
+ *   exits.  A shape is served exactly when fn_workspace_size(M, d, N, wt, 0)
+ *   <= 8 MiB; larger ones are rejected with FN_ERR_WORKSPACE before any
+ *   launch.  On a 148-SM B200 that admits bf16 weights at every M > 64 and at
+ *   M <= 32, M in 33..64 while the split-K partials stay under 8 MiB; fp8
+ *   weights at M <= 64 under the same rule, and at M > 64 while the split
+ *   activations (2 M d bytes, plus 4 bytes per row and 128-deep k block) fit,
+ *   and at M >= 1024 only while a bf16 copy of the weight (2 d N bytes) would
+ *   fit too.
  *   The array is zero when the library loads, so no set-up copy is made; the
  *   first call on a device only fetches the array's device address (a host
  *   query): make that first call before any stream capture.  All calls on a
@@ -373,7 +379,10 @@ uint64_t fn_kernel_launches(void);
  *   FN_DEBUG_WITHHOLD_ARRIVE  1: the reducers withhold their first arrival, so the
  *                             epilogue's wait must run out (exercises FN_ERR_TIMEOUT)
  *   FN_DEBUG_FORCE_PATH       0 auto, 1 decode kernel (M <= 64 only), 2 tile kernel,
- *                             3 tile kernel on single SMs (never the pair kernel)
+ *                             3 tile kernel on single SMs (never the pair kernel),
+ *                             4 tile path, with fp8 weights through the on-chip
+ *                             weight conversion (M < 1024) or the dequantised copy
+ *                             instead of the block-scale promotion kernel
  *   FN_DEBUG_PREFETCH         decode path: weight prefetch into L2 before waiting on
  *                             the previous kernel; value = mode | (k_blocks << 8),
  *                             mode 0 off, 1 TMA prefetch, 2 per-thread prefetch

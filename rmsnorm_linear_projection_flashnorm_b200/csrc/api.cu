@@ -201,11 +201,18 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   int sms = 0;
   fn_status st = check_device(sms);
   if (st != FN_OK) return st;
-  // fp8 weights at M >= kFp8DequantOnceM and MXFP8 weights on the tile path are
-  // converted to bf16 once per call into the workspace
+  // fp8 weights with bf16 output on the tile path: the block-scale promotion
+  // kernel (tc8.cu), which multiplies the stored e4m3 codes.  The other tile
+  // forms with fp8 weights (NVFP4 or partial output, AdaLN, or forced) convert
+  // the staged weight tiles to bf16 (M < kFp8DequantOnceM) or the whole weight
+  // once per call into the workspace; MXFP8 weights on the tile path take the
+  // latter route.
+  const bool fp8_tc8 = !use_decode && wt == FN_W_FP8_E4M3_B128 && !adaln && !fp4 && !partial && force != 4;
   const bool dequant_once =
-      !use_decode && ((wt == FN_W_FP8_E4M3_B128 && (M >= kFp8DequantOnceM || adaln)) || wt == FN_W_MXFP8_E4M3);
+      !use_decode && !fp8_tc8 &&
+      ((wt == FN_W_FP8_E4M3_B128 && (M >= kFp8DequantOnceM || adaln)) || wt == FN_W_MXFP8_E4M3);
   const size_t need = use_decode     ? decode_workspace_bytes(M, d, ncols, swiglu, sms, static_cast<int>(wt))
+                      : fp8_tc8      ? tc8_workspace_bytes(M, d)
                       : dequant_once ? kWsHeaderBytes + wbytes * 2
                                      : kWsHeaderBytes;
   if (ws_bytes < need) return FN_ERR_WORKSPACE;
@@ -251,7 +258,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
     a.wtype = FN_W_BF16;
     a.scales = nullptr;
   }
-  const cudaError_t e = use_decode ? launch_decode(a) : launch_tc(a);
+  const cudaError_t e = use_decode ? launch_decode(a) : fp8_tc8 ? launch_tc8(a) : launch_tc(a);
   return e == cudaSuccess ? FN_OK : FN_ERR_CUDA;
 }
 
@@ -299,8 +306,14 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
   if (M <= 0 || d <= 0 || N <= 0 || d % 64 != 0 || N % 128 != 0) return kWsHeaderBytes;
   const int64_t ncols = swiglu ? 2 * N : N;
   if (M > 64) {
-    if ((wt == FN_W_FP8_E4M3_B128 && M >= kFp8DequantOnceM) || wt == FN_W_MXFP8_E4M3)
-      return kWsHeaderBytes + static_cast<size_t>(d) * static_cast<size_t>(ncols) * 2;
+    const size_t copy = kWsHeaderBytes + static_cast<size_t>(d) * static_cast<size_t>(ncols) * 2;
+    if (wt == FN_W_MXFP8_E4M3) return copy;
+    if (wt == FN_W_FP8_E4M3_B128) {
+      // the promotion kernel's split x, or (NVFP4 / partial output at large M)
+      // the dequantised weight
+      const size_t t8 = tc8_workspace_bytes(M, d);
+      return M >= kFp8DequantOnceM && copy > t8 ? copy : t8;
+    }
     return kWsHeaderBytes;
   }
   return decode_workspace_bytes(M, d, ncols, swiglu != 0, current_sms_or_default(), static_cast<int>(wt));
@@ -499,7 +512,7 @@ fn_status fn_set_debug(int key, int64_t value) {
       g_withhold.store(value ? 1 : 0);
       return FN_OK;
     case FN_DEBUG_FORCE_PATH:
-      if (value < 0 || value > 3) return FN_ERR_INVALID_ARG;
+      if (value < 0 || value > 4) return FN_ERR_INVALID_ARG;
       g_force_path.store(static_cast<int>(value));
       return FN_OK;
     case FN_DEBUG_CLUSTER:

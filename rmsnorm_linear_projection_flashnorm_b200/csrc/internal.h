@@ -87,6 +87,11 @@ cudaError_t launch_tc(const CallArgs& a);
 cudaError_t launch_tc_pair(const CallArgs& a);
 // Rows from which the tile path runs on pairs of SMs.
 constexpr int64_t kPairTileMinM = 512;
+// fp8 weights (128x128 block scales) at M > 64 with bf16 output: x split once
+// into exact e4m3 hi/lo planes, the stored codes multiplied as they are, the
+// block scales applied per 128-deep k block to fp32 sums (tc8.cu).
+size_t tc8_workspace_bytes(int64_t M, int64_t d);
+cudaError_t launch_tc8(const CallArgs& a);
 
 // Offline fold and the unfused-chain helper kernels.
 cudaError_t launch_fold_bf16(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wp,

@@ -1,0 +1,439 @@
+// Fused RMSNorm + projection, tile path (M > 64) for fp8 e4m3 weights with an
+// fp32 scale per 128 x 128 block, sm_100a.
+//
+// The arithmetic is FlashNorm's (FlashNorm talk summary, Proposal 2: matmul on
+// raw x, the sum of squares alongside, 1/rms applied after; the folded weight
+// may be quantised, Proposal 1):
+//
+//   y[m, n] = r[m] * sum_b s[b, n] * sum_{k in block b} q[k, n] x[m, k]
+//
+// The e4m3 weight codes go to the tensor cores as they are stored: TMA copies
+// them into shared memory with the 128-byte swizzle and they are the B operand
+// (N-major) of tcgen05.mma kind::f8f6f4.  The activations are converted
+// instead, exactly, once per call: a small kernel splits each row and
+// 128-deep k block of x into hi = e4m3(a) and lo = e4m3(a - hi) with
+// a = x * 2^e (the power of two that puts the block's largest magnitude in
+// [128, 256)), writes the two code planes, 2^-e per (block, row), and each
+// row's sum of squares.  In the tile kernel every 128-deep k block is one
+// pipeline stage: eight MMAs (four 32-deep steps for x_hi, four for x_lo) sum
+// the exact products into a TMEM buffer of its own, and scaler warps read the
+// buffer back and add it, times s[b, n] * 2^-e[b, m], to fp32 running sums in
+// registers, in ascending k order.  This is the block-scale promotion of the
+// Marlin explainer's section 4 (dequantisation hidden under the MMA stream),
+// applied to the sums instead of the weights: no weight tile is converted and
+// no bf16 copy of the weight is written.
+//
+// Compared with converting the staged weight tiles to bf16 on chip, the weight
+// bytes per flop in shared memory are the same (B is read once per half of the
+// split), and the conversion work moves off the MMA's critical path; compared
+// with dequantising the whole weight into the workspace first, it saves a
+// write and a read of a bf16 weight copy per call.
+//
+// Layout (persistent, one CTA per SM, 128 x 256 output tiles):
+//   warp 0      TMA producer (x_hi, x_lo, two e4m3 weight boxes per stage)
+//   warp 1      TMEM owner and MMA issuer
+//   warps 2-9   scalers and epilogue: warp w reads TMEM lane quarter w % 4;
+//               the two warps of a quarter take the two halves of the tile's
+//               columns (SwiGLU: matching 64-column halves of gate and up)
+#include <cstddef>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fn {
+namespace tc8 {
+
+constexpr int BM = 128, BN = 256, BKQ = 128;
+constexpr int XQ_BYTES = BM * BKQ;                    // one e4m3 code plane tile: 128 rows x 128 k (16 KB)
+constexpr int WQ_BOX = 128 * BKQ;                     // 128 weight columns x 128 k rows (16 KB)
+constexpr int STAGE_BYTES = 2 * XQ_BYTES + 2 * WQ_BOX;   // x_hi, x_lo, weight: 64 KB
+constexpr int STAGES = 3;
+constexpr int NUM_THREADS = 320;
+constexpr int TMEM_COLS = 2 * BN;                     // two per-k-block accumulators
+constexpr int GROUP_M = 16;                           // tile raster: bands of 16 row blocks
+
+enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteScaleAccFull };
+
+struct Params {
+  int M, d, ncols, nout;
+  int num_m, num_n, num_tiles, kblocks, nblk;
+  float eps, inv_d;
+  __nv_bfloat16* y;
+  unsigned int* status;
+  unsigned long long budget_ns;
+  int withhold;
+  const float* scales;   // weight block scales [kblocks][nblk]
+  const float* fac;      // 2^-e of each (k block, row) of the split [kblocks][M]; NaN: non-finite block
+  const float* ssq;      // sum of squares of each row [M]
+};
+
+struct alignas(8) Bars {
+  uint64_t full[STAGES], empty[STAGES];
+  uint64_t accf[2], acce[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr size_t smem_bytes() { return 1024 + STAGES * STAGE_BYTES + sizeof(Bars); }
+static_assert(smem_bytes() <= 232448, "shared memory budget");
+
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
+  const int per_group = GROUP_M * p.num_n;
+  const int group = t / per_group;
+  const int first_m = group * GROUP_M;
+  const int gm = min(p.num_m - first_m, GROUP_M);
+  const int r = t - group * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long budget) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > budget) return;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Split x once per call.  One warp per row; lane l takes k values 4l .. 4l+3 of
+// every 128-deep block, so each block is one coalesced 256-byte read and two
+// 128-byte writes.  The row's sum of squares accumulates per lane in k order
+// and is reduced over the lanes in a fixed tree (repeated calls agree bit for
+// bit).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) xsplit_rows_kernel(const __nv_bfloat16* __restrict__ x, int M, int d,
+                                                          uint8_t* __restrict__ xhi, uint8_t* __restrict__ xlo,
+                                                          float* __restrict__ fac, float* __restrict__ ssq) {
+  grid_launch_dependents();     // the tile kernel may set up meanwhile
+  grid_dependency_wait();       // x may have been written by the preceding kernel
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const int kblocks = d / BKQ;
+  const __nv_bfloat16* xr = x + static_cast<int64_t>(row) * d + lane * 4;
+  uint64_t ss2 = 0;   // (+0.0f, +0.0f)
+#pragma unroll 4
+  for (int kb = 0; kb < kblocks; ++kb) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(xr + kb * BKQ));
+    uint32_t amax = max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu), max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    // amax is a bf16 bit pattern (|x| orders like its bits): exponent field in
+    // bits 7..14, 255 for inf / NaN
+    const int E = static_cast<int>(amax >> 7);
+    int e = amax == 0 ? 0 : 134 - E;          // amax * 2^e in [128, 256)
+    e = e > 126 ? 126 : (e < -126 ? -126 : e);
+    const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+    const uint64_t sc2 = f2_pack(sc, sc);
+    const uint64_t a = f2_pack_u(v.x << 16, v.x & 0xFFFF0000u), b = f2_pack_u(v.y << 16, v.y & 0xFFFF0000u);
+    ss2 = f2_fma(b, b, f2_fma(a, a, ss2));
+    uint16_t h0, l0, h1, l1;
+    split_e4m3x2(f2_mul(a, sc2), h0, l0);
+    split_e4m3x2(f2_mul(b, sc2), h1, l1);
+    const int64_t off = static_cast<int64_t>(row) * d + kb * BKQ + lane * 4;
+    *reinterpret_cast<uint32_t*>(xhi + off) = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+    *reinterpret_cast<uint32_t*>(xlo + off) = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+    if (lane == 0)
+      fac[static_cast<int64_t>(kb) * M + row] =
+          E == 255 ? __int_as_float(0x7fc00000) : __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+  }
+  float ss = f2_lo(ss2) + f2_hi(ss2);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) ssq[row] = ss;
+}
+
+// ---------------------------------------------------------------------------
+// The tile kernel.
+// ---------------------------------------------------------------------------
+template <bool SWIGLU>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc8_kernel(const __grid_constant__ CUtensorMap tmap_xh, const __grid_constant__ CUtensorMap tmap_xl,
+               const __grid_constant__ CUtensorMap tmap_w, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars& bars = *reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
+  // stage: [x_hi 128 x 128][x_lo 128 x 128][weight: two 128-column boxes], 1024-byte multiples
+  auto stage_xh = [&](int s) { return smem + s * STAGE_BYTES; };
+  auto stage_xl = [&](int s) { return smem + s * STAGE_BYTES + XQ_BYTES; };
+  auto stage_w = [&](int s) { return smem + s * STAGE_BYTES + 2 * XQ_BYTES; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], 1);       // MMA commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.accf[b], 1);        // MMA commit
+      mbar_init(&bars.acce[b], 8);        // one arrival per scaler warp
+    }
+    mbar_init(&bars.drain, 1);
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_xh);
+    tma_prefetch_desc(&tmap_xl);
+    tma_prefetch_desc(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // Everything above overlaps the preceding kernel (the x split); nothing
+  // below touches global memory before it has completed.
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const uint32_t tmem_base = bars.tmem_base;
+  const WaitCtl ctl{&bars.abort_flag, p.status, p.budget_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued = 0, last_ph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, p, mb, nb);
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(&bars.empty[s], ph ^ 1, ctl, kSiteProdEmpty)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars.full[s], STAGE_BYTES);
+          tma_load_2d(stage_xh(s), &tmap_xh, &bars.full[s], kb * BKQ, mb * BM);
+          tma_load_2d(stage_xl(s), &tmap_xl, &bars.full[s], kb * BKQ, mb * BM);
+          // a plain projection with an odd number of 128-column blocks has a
+          // last tile whose second box lies past the weight: TMA fills zeros
+          tma_load_2d(stage_w(s), &tmap_w, &bars.full[s], nb * BN, kb * BKQ);
+          tma_load_2d(stage_w(s) + WQ_BOX, &tmap_w, &bars.full[s], nb * BN + 128, kb * BKQ);
+          issued |= 1u << s;
+          last_ph = (last_ph & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      // no copy may still be landing in shared memory when the CTA exits
+      for (int i = 0; i < STAGES; ++i)
+        if (issued & (1u << i)) drain_wait(&bars.full[i], (last_ph >> i) & 1u, p.budget_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      // A = x_hi / x_lo rows, K-major; B = e4m3 weight, N-major
+      constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN, /*a MN-major*/ false, /*b MN-major*/ true);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      uint32_t it = 0;   // k blocks processed by this CTA: selects the TMEM buffer
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+          const uint32_t b = it & 1, aph = (it >> 1) & 1;
+          if (!mbar_wait(&bars.acce[b], aph ^ 1, ctl, kSiteMmaAccEmpty)) { ok = false; break; }
+          if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + b * BN;
+          const uint32_t xh = smem_u32(stage_xh(s)), xl = smem_u32(stage_xl(s)), w0 = smem_u32(stage_w(s));
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+#pragma unroll
+            for (int kk = 0; kk < BKQ / 32; ++kk) {
+              // A: 128-byte rows of e4m3 codes, 8-row groups 1024 B apart; a
+              //    32-deep step is 32 bytes further along the (swizzled) row.
+              const uint64_t adesc = sdesc_sw128((part == 0 ? xh : xl) + kk * 32, 16, 1024);
+              // B: k rows of 128 columns (128 bytes), the two column boxes
+              //    16 KB apart (LBO), 8-row k groups 1024 B apart (SBO); a
+              //    32-deep step is 32 rows = 4096 B.
+              const uint64_t bdesc = sdesc_sw128(w0 + kk * 4096, WQ_BOX, 1024);
+              umma_e4m3(d_tmem, adesc, bdesc, IDESC, (part | kk) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&bars.empty[s]);
+          umma_commit(&bars.accf[b]);
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      umma_commit(&bars.drain);
+      drain_wait(&bars.drain, 0, p.budget_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ scalers and epilogue
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;       // 0: warps 2-5, 1: warps 6-9
+    // the two 64-column chunks of the 256-column accumulator this thread adds up
+    const int c0 = SWIGLU ? half * 64 : half * 128;
+    const int c1 = SWIGLU ? BN / 2 + half * 64 : half * 128 + 64;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      const int row = mb * BM + q * 32 + lane;
+      const bool live = row < p.M;
+      // 128-column weight blocks of the two chunks (the scale columns)
+      const int blk0 = SWIGLU ? 2 * nb : 2 * nb + half;
+      const int blk1 = SWIGLU ? 2 * nb + 1 : 2 * nb + half;
+      const bool have0 = blk0 < p.nblk, have1 = blk1 < p.nblk;
+      const float ssq = live ? __ldg(p.ssq + row) : 0.f;
+      uint64_t acc[64];   // packed fp32 pairs: chunk 0 columns in acc[0..31], chunk 1 in acc[32..63]
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] = 0;
+      // 2^-e and the block scales, loaded one k block ahead
+      auto load_fac = [&](int kb) { return live ? __ldg(p.fac + static_cast<int64_t>(kb) * p.M + row) : 0.f; };
+      auto load_s = [&](int kb, int blk, bool have) {
+        return have ? __ldg(p.scales + static_cast<int64_t>(kb) * p.nblk + blk) : 0.f;
+      };
+      float f_n = load_fac(0), s0_n = load_s(0, blk0, have0), s1_n = load_s(0, blk1, have1);
+      for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+        const float f = f_n, s0 = s0_n, s1 = s1_n;
+        if (kb + 1 < p.kblocks) {
+          f_n = load_fac(kb + 1);
+          s0_n = load_s(kb + 1, blk0, have0);
+          s1_n = load_s(kb + 1, blk1, have1);
+        }
+        const uint32_t b = it & 1, aph = (it >> 1) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.accf[b], aph, ctl, kSiteScaleAccFull))) { ok = false; break; }
+        tc_fence_after();
+        // s * 2^-e: the product is exact unless it leaves the normal range
+        const float k0 = f * s0, k1 = f * s1;
+        const uint64_t kk0 = f2_pack(k0, k0), kk1 = f2_pack(k1, k1);
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+        // four rounds of 32 columns (two 16-column loads each), so that the
+        // loaded values and the 128 running sums fit the register budget of
+        // 10 warps per SM (at most 3 warps on a scheduler: 168 registers)
+#pragma unroll
+        for (int rd = 0; rd < 4; ++rd) {
+          uint32_t v0[16], v1[16];
+          const uint32_t col = (rd < 2 ? c0 : c1) + (rd & 1) * 32;
+          tmem_ld16(taddr + col, v0);
+          tmem_ld16(taddr + col + 16, v1);
+          tmem_ld_wait();
+          if (rd == 3) {
+            // every TMEM read of this buffer has completed: hand it back
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && !(p.withhold && it == 0)) mbar_arrive(&bars.acce[b]);
+          }
+          const uint64_t kc = rd < 2 ? kk0 : kk1;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            acc[rd * 16 + j] = f2_fma(kc, f2_pack_u(v0[2 * j], v0[2 * j + 1]), acc[rd * 16 + j]);
+            acc[rd * 16 + 8 + j] = f2_fma(kc, f2_pack_u(v1[2 * j], v1[2 * j + 1]), acc[rd * 16 + 8 + j]);
+          }
+        }
+      }
+      if (!ok) break;
+      // epilogue: 1/rms of the raw row (FlashNorm's deferred normalisation), then SwiGLU
+      if (live) {
+        const float r = inv_rms(ssq, p.inv_d, p.eps);
+        if constexpr (SWIGLU) {
+          // chunk 0 holds gate columns, chunk 1 the matching up columns
+          __nv_bfloat16* yrow = p.y + static_cast<int64_t>(row) * p.nout + nb * (BN / 2) + half * 64;
+#pragma unroll
+          for (int g16 = 0; g16 < 8; ++g16) {
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t gv = acc[g16 * 4 + j], uv = acc[32 + g16 * 4 + j];
+              const float g0 = f2_lo(gv) * r, g1 = f2_hi(gv) * r, u0 = f2_lo(uv) * r, u1 = f2_hi(uv) * r;
+              o[j] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+            }
+            reinterpret_cast<uint4*>(yrow)[g16] = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        } else {
+          const int col0 = nb * BN + half * 128;
+          if (col0 < p.nout) {
+            __nv_bfloat16* yrow = p.y + static_cast<int64_t>(row) * p.nout + col0;
+#pragma unroll
+            for (int g16 = 0; g16 < 16; ++g16) {
+              uint32_t o[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint64_t v = acc[g16 * 4 + j];
+                o[j] = pack_bf16x2(f2_lo(v) * r, f2_hi(v) * r);
+              }
+              reinterpret_cast<uint4*>(yrow)[g16] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace tc8
+
+size_t tc8_workspace_bytes(int64_t M, int64_t d) {
+  const size_t planes = (static_cast<size_t>(M) * d + 255) / 256 * 256;
+  const size_t facb = (static_cast<size_t>(d / tc8::BKQ) * M * 4 + 255) / 256 * 256;
+  const size_t ssqb = (static_cast<size_t>(M) * 4 + 255) / 256 * 256;
+  return kWsHeaderBytes + 2 * planes + facb + ssqb;
+}
+
+cudaError_t launch_tc8(const CallArgs& a) {
+  using namespace tc8;
+  if (a.ws_bytes < tc8_workspace_bytes(a.M, a.d)) return cudaErrorInvalidValue;
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  const size_t planes = (static_cast<size_t>(a.M) * a.d + 255) / 256 * 256;
+  const size_t facb = (static_cast<size_t>(a.d / BKQ) * a.M * 4 + 255) / 256 * 256;
+  uint8_t* xhi = ws + kWsHeaderBytes;
+  uint8_t* xlo = xhi + planes;
+  float* fac = reinterpret_cast<float*>(xlo + planes);
+  float* ssq = reinterpret_cast<float*>(xlo + planes + facb);
+
+  const int M = static_cast<int>(a.M), d = static_cast<int>(a.d);
+  cudaError_t e = launch_pdl(xsplit_rows_kernel, static_cast<unsigned>((M + 7) / 8), 256, 0, a.stream,
+                             static_cast<const __nv_bfloat16*>(a.x), M, d, xhi, xlo, fac, ssq);
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap th, tl, tw;
+  if (!make_tmap_2d(&th, xhi, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.d, BM, BKQ)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tl, xlo, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.d, BM, BKQ)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.d, a.ncols, BKQ, 128)) return cudaErrorInvalidValue;
+  Params p;
+  p.M = M;
+  p.d = d;
+  p.ncols = static_cast<int>(a.ncols);
+  p.nout = static_cast<int>(a.N);
+  p.num_m = (M + BM - 1) / BM;
+  p.num_n = static_cast<int>((a.ncols + BN - 1) / BN);
+  p.num_tiles = p.num_m * p.num_n;
+  p.kblocks = d / BKQ;
+  p.nblk = static_cast<int>(a.ncols / 128);
+  p.eps = a.eps;
+  p.inv_d = 1.0f / static_cast<float>(a.d);
+  p.y = static_cast<__nv_bfloat16*>(a.y);
+  p.status = reinterpret_cast<unsigned int*>(ws);
+  p.budget_ns = a.budget_ns;
+  p.withhold = a.withhold;
+  p.scales = a.scales;
+  p.fac = fac;
+  p.ssq = ssq;
+  const int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
+  constexpr size_t SMEM = smem_bytes();
+  if (a.swiglu) {
+    e = ensure_smem_limit<tc8_kernel<true>>(static_cast<int>(SMEM));
+    if (e != cudaSuccess) return e;
+    return launch_pdl(tc8_kernel<true>, grid, NUM_THREADS, SMEM, a.stream, th, tl, tw, p);
+  }
+  e = ensure_smem_limit<tc8_kernel<false>>(static_cast<int>(SMEM));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(tc8_kernel<false>, grid, NUM_THREADS, SMEM, a.stream, th, tl, tw, p);
+}
+
+}  // namespace fn

@@ -50,15 +50,18 @@ def test_dequant_step_bit_exact():
 
 def _tile_path(M, force=0):
     """True where the e4m3 weight reaches the tensor cores as bf16(q * s): the
-    tile kernel's converter warps (65 <= M < 1024, or forced) and the
-    dequantise-once route (M >= 1024).  The decode kernels (M <= 64) multiply
-    the e4m3 codes exactly and apply s to the fp32 sums."""
-    return force == 2 or (force == 0 and M > 64)
+    tile kernel's converter warps and the dequantise-once route, which the
+    library takes for fp8 weights only when forced (FN_DEBUG_FORCE_PATH = 4)
+    or for NVFP4, partial and AdaLN outputs.  The decode kernels (M <= 64) and
+    the block-scale promotion kernel (M > 64) multiply the e4m3 codes exactly
+    and apply s to fp32 sums."""
+    return force == 4
 
 
 def _stored_weight(q, sr, tile):
-    """The weight each path multiplies: the exact q * s for the decode kernels,
-    its one bf16 rounding for the tile paths (the oracle's own rounding)."""
+    """The weight each path multiplies: the exact q * s for the decode and
+    promotion kernels, its one bf16 rounding for the converting paths (the
+    oracle's own rounding)."""
     if tile:
         return O.bf16_from_bits(O.dequant_fp8_bf16_bits(q, sr))
     return O.dequant_fp8(q, sr)
@@ -117,6 +120,75 @@ def test_fp8_both_paths_at_small_m(path):
             _check(*_case(M, 256, 256, sw, seed=132, force=path))
     finally:
         fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 0)
+
+
+@pytest.mark.parametrize("M,d,N,swiglu", [
+    (65, 256, 384, False),     # smallest tile-path M; 3 column blocks: the last tile's second half is past N
+    (200, 1024, 512, True),
+    (333, 4096, 256, False),   # long k range, ragged rows
+    (130, 512, 1280, True),
+])
+def test_fp8_promotion_kernel(M, d, N, swiglu):
+    """The block-scale promotion kernel (x split once into exact e4m3 parts,
+    each 128-deep k block's exact sums scaled and added in fp32) is held to the
+    bf16-weight bound against the exact dequantised weight."""
+    y, ref, ref_exact = _case(M, d, N, swiglu, seed=160 + M)
+    assert rel_err(y, ref_exact) <= BF16_TOL
+    _check(y, ref, ref_exact)
+
+
+@pytest.mark.parametrize("M,d,N,swiglu", [(200, 256, 384, False), (300, 512, 384, True), (1100, 256, 256, True)])
+def test_fp8_converting_routes(M, d, N, swiglu):
+    """The routes that convert the weight to bf16 (on chip per tile below 1024
+    rows, once per call into the workspace from 1024), which NVFP4, partial and
+    AdaLN outputs use, forced here for bf16 output."""
+    fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 4)
+    try:
+        _check(*_case(M, d, N, swiglu, seed=170 + M, force=4))
+    finally:
+        fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 0)
+
+
+def test_fp8_promotion_wide_dynamic_range_is_exact():
+    """Activations spanning 2^-18 .. 2^10 inside one k block still meet the
+    bf16-weight bound: the split of each (row, k block) is exact above 2^-9 of
+    the block's largest magnitude."""
+    M, d, N = 100, 512, 384
+    x = WL.activations(M, d, 161).float()
+    mult = torch.ones(d)
+    mult[0::4] = 2.0 ** 10
+    mult[1::8] = 2.0 ** -12
+    mult[3::16] = 2.0 ** -18
+    x = (x * mult).to(torch.bfloat16)
+    for swiglu in (False, True):
+        y, ref, _ = _case(M, d, N, swiglu, seed=161, x=x)
+        assert rel_err(y, ref) <= BF16_TOL
+
+
+def test_fp8_promotion_repeated_calls_and_timeout():
+    """Bit-identical repeats, and a withheld scaler arrival times out cleanly:
+    the status word reports it and the next call is correct."""
+    M, d, N = 300, 1024, 512
+    inp = WL.case(M, d, N, True, seed=162)
+    Wq, s = T.fold(gpu(inp["W_gate"]), gpu(inp["g"]), gpu(inp["W_up"]), wtype=FP8)
+    x = gpu(inp["x"])
+    ws = T.Workspace()
+    first = run(x, Wq, N, 1e-6, swiglu=True, scales=s, ws=ws).clone()
+    for _ in range(100):
+        assert torch.equal(run(x, Wq, N, 1e-6, swiglu=True, scales=s, ws=ws), first)
+    assert ws.status()[0] == fnb.FN_OK
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 20_000_000) == fnb.FN_OK
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_WITHHOLD_ARRIVE, 1) == fnb.FN_OK
+    try:
+        T.norm_proj(x, Wq, N, 1e-6, swiglu=True, scales=s, ws=ws)
+        st, word = ws.status()
+    finally:
+        fnb.fn_set_debug(fnb.FN_DEBUG_WITHHOLD_ARRIVE, 0)
+        fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 2_000_000_000)
+    assert st == fnb.FN_ERR_TIMEOUT and (word >> 8) != 0
+    ws.buf.zero_()
+    assert torch.equal(run(x, Wq, N, 1e-6, swiglu=True, scales=s, ws=ws), first)
+    assert ws.status()[0] == fnb.FN_OK
 
 
 @pytest.mark.parametrize("M", [1, 2, 15, 16, 17, 31, 32, 33, 63, 64])
