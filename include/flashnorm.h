@@ -117,8 +117,8 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
  * the two e4m3 operand parts (2 x 64 x d bytes at most) with their scale
  * factors and per-block sums of squares; with fp8 weights and M > 64 the
  * activations split once per call for the block-scale promotion kernel
- * (2 M d bytes of e4m3 codes, 4 bytes per row and 128-deep k block, 4 bytes
- * per row), and at M >= 1024 at least one bf16 copy of the weight (2 d ncols
+ * (2 M d bytes of e4m3 codes, 8 bytes per row and 128-deep k block), and at
+ * M >= 1024 at least one bf16 copy of the weight (2 d ncols
  * bytes), which the NVFP4 and partial-output calls convert once per call with
  * the rounding of the on-chip conversion (bf16(fp32(q) * s)); with MXFP8
  * weights the same bf16 copy at every M > 64, and at M <= 64 the activations
@@ -318,7 +318,7 @@ fn_status fn_post_scale(const float* partial, int64_t M, int64_t N, int swiglu, 
  *   launch.  On a 148-SM B200 that admits bf16 weights at every M > 64 and at
  *   M <= 32, M in 33..64 while the split-K partials stay under 8 MiB; fp8
  *   weights at M <= 64 under the same rule, and at M > 64 while the split
- *   activations (2 M d bytes, plus 4 bytes per row and 128-deep k block) fit,
+ *   activations (2 M d bytes, plus 8 bytes per row and 128-deep k block) fit,
  *   and at M >= 1024 only while a bf16 copy of the weight (2 d N bytes) would
  *   fit too.
  *   The array is zero when the library loads, so no set-up copy is made; the

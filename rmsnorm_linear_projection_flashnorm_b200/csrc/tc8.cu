@@ -13,8 +13,8 @@
 // instead, exactly, once per call: a small kernel splits each row and
 // 128-deep k block of x into hi = e4m3(a) and lo = e4m3(a - hi) with
 // a = x * 2^e (the power of two that puts the block's largest magnitude in
-// [128, 256)), writes the two code planes, 2^-e per (block, row), and each
-// row's sum of squares.  In the tile kernel every 128-deep k block is one
+// [128, 256)), writes the two code planes, 2^-e per (block, row), and the
+// partial sums of squares per (block, row).  In the tile kernel every 128-deep k block is one
 // pipeline stage: eight MMAs (four 32-deep steps for x_hi, four for x_lo) sum
 // the exact products into a TMEM buffer of its own, and scaler warps read the
 // buffer back and add it, times s[b, n] * 2^-e[b, m], to fp32 running sums in
@@ -66,8 +66,39 @@ struct Params {
   int withhold;
   const float* scales;   // weight block scales [kblocks][nblk]
   const float* fac;      // 2^-e of each (k block, row) of the split [kblocks][M]; NaN: non-finite block
-  const float* ssq;      // sum of squares of each row [M]
+  const float* ssq_part; // sum of squares of each (k block, row) [kblocks][M]
+  int split_tail;        // 1: launched as 2-CTA clusters; the tiles after the full waves are split in k
+  int full_waves;        //   between the two CTAs of a cluster (tile full_waves * grid + cluster index)
+  int tail;              //   number of such tiles (<= clusters)
 };
+
+// The i-th work item of this CTA: a tile and its k-block range.  Without the
+// split tail, tiles are dealt round-robin over the CTAs.  With it, every CTA
+// first takes full_waves whole tiles the same way, and then the two CTAs of
+// cluster c share tile full_waves * grid + c (c < tail): rank 0 takes the
+// lower half of the k blocks, rank 1 the upper half.  A last wave that would
+// leave more than half of the SMs idle thus takes half as long.
+struct Work {
+  int t, kb0, kb1;
+  bool split;
+};
+__device__ __forceinline__ bool work_item(const Params& p, int i, Work& w) {
+  const int G = static_cast<int>(gridDim.x);
+  w.split = false;
+  w.kb0 = 0;
+  w.kb1 = p.kblocks;
+  if (!p.split_tail || i < p.full_waves) {
+    w.t = static_cast<int>(blockIdx.x) + i * G;
+    return w.t < p.num_tiles && (!p.split_tail || i < p.full_waves);
+  }
+  const int c = static_cast<int>(blockIdx.x) >> 1, r = static_cast<int>(blockIdx.x) & 1;
+  if (i != p.full_waves || c >= p.tail) return false;
+  w.t = p.full_waves * G + c;
+  w.kb0 = r * p.kblocks / 2;
+  w.kb1 = (r + 1) * p.kblocks / 2;
+  w.split = true;
+  return true;
+}
 
 struct alignas(8) Bars {
   uint64_t full[STAGES], empty[STAGES];
@@ -98,52 +129,88 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
 }
 
 // ---------------------------------------------------------------------------
-// Split x once per call.  One warp per row; lane l takes k values 4l .. 4l+3 of
-// every 128-deep block, so each block is one coalesced 256-byte read and two
-// 128-byte writes.  The row's sum of squares accumulates per lane in k order
-// and is reduced over the lanes in a fixed tree (repeated calls agree bit for
-// bit).
+// Split x once per call.  One warp per (row, 128-deep k block); lane l takes
+// k values 4l .. 4l+3, so the eight warps of a block read 2 KB of one row in
+// one coalesced sweep.  Each warp writes its 128 hi and lo codes, 2^-e and the
+// block's partial sum of squares (lane sums reduced in a fixed tree); the tile
+// kernel adds a row's partial sums in k order, so repeated calls agree bit for
+// bit.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) xsplit_rows_kernel(const __nv_bfloat16* __restrict__ x, int M, int d,
                                                           uint8_t* __restrict__ xhi, uint8_t* __restrict__ xlo,
-                                                          float* __restrict__ fac, float* __restrict__ ssq) {
+                                                          float* __restrict__ fac, float* __restrict__ ssq_part) {
   grid_launch_dependents();     // the tile kernel may set up meanwhile
   grid_dependency_wait();       // x may have been written by the preceding kernel
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= M) return;
   const int kblocks = d / BKQ;
-  const __nv_bfloat16* xr = x + static_cast<int64_t>(row) * d + lane * 4;
-  uint64_t ss2 = 0;   // (+0.0f, +0.0f)
-#pragma unroll 4
-  for (int kb = 0; kb < kblocks; ++kb) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(xr + kb * BKQ));
-    uint32_t amax = max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu), max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu));
+  const long long wg = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int row = static_cast<int>(wg / kblocks), kb = static_cast<int>(wg - static_cast<long long>(row) * kblocks);
+  if (row >= M) return;
+  const int64_t off = static_cast<int64_t>(row) * d + kb * BKQ + lane * 4;
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(x + off));
+  uint32_t amax = max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu), max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu));
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    // amax is a bf16 bit pattern (|x| orders like its bits): exponent field in
-    // bits 7..14, 255 for inf / NaN
-    const int E = static_cast<int>(amax >> 7);
-    int e = amax == 0 ? 0 : 134 - E;          // amax * 2^e in [128, 256)
-    e = e > 126 ? 126 : (e < -126 ? -126 : e);
-    const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-    const uint64_t sc2 = f2_pack(sc, sc);
-    const uint64_t a = f2_pack_u(v.x << 16, v.x & 0xFFFF0000u), b = f2_pack_u(v.y << 16, v.y & 0xFFFF0000u);
-    ss2 = f2_fma(b, b, f2_fma(a, a, ss2));
-    uint16_t h0, l0, h1, l1;
-    split_e4m3x2(f2_mul(a, sc2), h0, l0);
-    split_e4m3x2(f2_mul(b, sc2), h1, l1);
-    const int64_t off = static_cast<int64_t>(row) * d + kb * BKQ + lane * 4;
-    *reinterpret_cast<uint32_t*>(xhi + off) = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-    *reinterpret_cast<uint32_t*>(xlo + off) = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
-    if (lane == 0)
-      fac[static_cast<int64_t>(kb) * M + row] =
-          E == 255 ? __int_as_float(0x7fc00000) : __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-  }
+  for (int o = 16; o >= 1; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  // amax is a bf16 bit pattern (|x| orders like its bits): exponent field in
+  // bits 7..14, 255 for inf / NaN
+  const int E = static_cast<int>(amax >> 7);
+  int e = amax == 0 ? 0 : 134 - E;          // amax * 2^e in [128, 256)
+  e = e > 126 ? 126 : (e < -126 ? -126 : e);
+  const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+  const uint64_t sc2 = f2_pack(sc, sc);
+  const uint64_t a = f2_pack_u(v.x << 16, v.x & 0xFFFF0000u), b = f2_pack_u(v.y << 16, v.y & 0xFFFF0000u);
+  const uint64_t ss2 = f2_fma(b, b, f2_mul(a, a));
+  uint16_t h0, l0, h1, l1;
+  split_e4m3x2(f2_mul(a, sc2), h0, l0);
+  split_e4m3x2(f2_mul(b, sc2), h1, l1);
+  *reinterpret_cast<uint32_t*>(xhi + off) = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+  *reinterpret_cast<uint32_t*>(xlo + off) = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
   float ss = f2_lo(ss2) + f2_hi(ss2);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) ssq[row] = ss;
+  if (lane == 0) {
+    fac[static_cast<int64_t>(kb) * M + row] =
+        E == 255 ? __int_as_float(0x7fc00000) : __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+    ssq_part[static_cast<int64_t>(kb) * M + row] = ss;
+  }
+}
+
+// Epilogue of one thread's share of a tile: row `row`, column half `half`.
+// 1/rms of the raw row (FlashNorm's deferred normalisation), then SwiGLU (the
+// two chunks hold matching gate and up columns) or the plain projection (the
+// two chunks are 128 consecutive columns), one RN to bf16, 16-byte stores.
+template <bool SWIGLU>
+__device__ __forceinline__ void store_tile_half(const Params& p, const uint64_t (&acc)[64], int row, int nb, int half,
+                                                float ssq) {
+  const float r = inv_rms(ssq, p.inv_d, p.eps);
+  if constexpr (SWIGLU) {
+    __nv_bfloat16* yrow = p.y + static_cast<int64_t>(row) * p.nout + nb * (BN / 2) + half * 64;
+#pragma unroll
+    for (int g16 = 0; g16 < 8; ++g16) {
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint64_t gv = acc[g16 * 4 + j], uv = acc[32 + g16 * 4 + j];
+        const float g0 = f2_lo(gv) * r, g1 = f2_hi(gv) * r, u0 = f2_lo(uv) * r, u1 = f2_hi(uv) * r;
+        o[j] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+      }
+      reinterpret_cast<uint4*>(yrow)[g16] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  } else {
+    const int col0 = nb * BN + half * 128;
+    if (col0 >= p.nout) return;   // the half of a last tile that lies past the weight
+    __nv_bfloat16* yrow = p.y + static_cast<int64_t>(row) * p.nout + col0;
+#pragma unroll
+    for (int g16 = 0; g16 < 16; ++g16) {
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint64_t v = acc[g16 * 4 + j];
+        o[j] = pack_bf16x2(f2_lo(v) * r, f2_hi(v) * r);
+      }
+      reinterpret_cast<uint4*>(yrow)[g16] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -202,10 +269,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int s = 0;
       uint32_t ph = 0, issued = 0, last_ph = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      Work w;
+      for (int i = 0; ok && work_item(p, i, w); ++i) {
         int mb, nb;
-        tile_coords(t, p, mb, nb);
-        for (int kb = 0; kb < p.kblocks; ++kb) {
+        tile_coords(w.t, p, mb, nb);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&bars.empty[s], ph ^ 1, ctl, kSiteProdEmpty)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars.full[s], STAGE_BYTES);
           tma_load_2d(stage_xh(s), &tmap_xh, &bars.full[s], kb * BKQ, mb * BM);
@@ -224,6 +292,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (issued & (1u << i)) drain_wait(&bars.full[i], (last_ph >> i) & 1u, p.budget_ns);
     }
     __syncwarp();
+    if (p.split_tail) {   // the exchange of the scalers below: every thread takes part
+      cluster_sync_all();
+      cluster_sync_all();
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -233,8 +305,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t ph = 0;
       bool ok = true;
       uint32_t it = 0;   // k blocks processed by this CTA: selects the TMEM buffer
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+      Work w;
+      for (int i = 0; ok && work_item(p, i, w); ++i) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const uint32_t b = it & 1, aph = (it >> 1) & 1;
           if (!mbar_wait(&bars.acce[b], aph ^ 1, ctl, kSiteMmaAccEmpty)) { ok = false; break; }
           if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
@@ -264,6 +337,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_wait(&bars.drain, 0, p.budget_ns);
     }
     __syncwarp();
+    if (p.split_tail) {
+      cluster_sync_all();
+      cluster_sync_all();
+    }
   } else {
     // ------------------------------------------------------------ scalers and epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
@@ -273,28 +350,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int c1 = SWIGLU ? BN / 2 + half * 64 : half * 128 + 64;
     uint32_t it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+    uint64_t acc[64];   // packed fp32 pairs: chunk 0 columns in acc[0..31], chunk 1 in acc[32..63]
+    bool split_pending = false;             // a k-split tile's partial sums wait for the exchange
+    int s_row = 0, s_nb = 0;
+    float s_ssq = 0.f;
+    Work w;
+    for (int i = 0; ok && work_item(p, i, w); ++i) {
       int mb, nb;
-      tile_coords(t, p, mb, nb);
+      tile_coords(w.t, p, mb, nb);
       const int row = mb * BM + q * 32 + lane;
       const bool live = row < p.M;
       // 128-column weight blocks of the two chunks (the scale columns)
       const int blk0 = SWIGLU ? 2 * nb : 2 * nb + half;
       const int blk1 = SWIGLU ? 2 * nb + 1 : 2 * nb + half;
       const bool have0 = blk0 < p.nblk, have1 = blk1 < p.nblk;
-      const float ssq = live ? __ldg(p.ssq + row) : 0.f;
-      uint64_t acc[64];   // packed fp32 pairs: chunk 0 columns in acc[0..31], chunk 1 in acc[32..63]
+      // the row's sum of squares: its k blocks' partial sums, in k order
+      float ssq = 0.f;
+      if (live) {
+#pragma unroll 8
+        for (int kb = 0; kb < p.kblocks; ++kb) ssq += __ldg(p.ssq_part + static_cast<int64_t>(kb) * p.M + row);
+      }
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0;
+      for (int j = 0; j < 64; ++j) acc[j] = 0;
       // 2^-e and the block scales, loaded one k block ahead
       auto load_fac = [&](int kb) { return live ? __ldg(p.fac + static_cast<int64_t>(kb) * p.M + row) : 0.f; };
       auto load_s = [&](int kb, int blk, bool have) {
         return have ? __ldg(p.scales + static_cast<int64_t>(kb) * p.nblk + blk) : 0.f;
       };
-      float f_n = load_fac(0), s0_n = load_s(0, blk0, have0), s1_n = load_s(0, blk1, have1);
-      for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+      float f_n = load_fac(w.kb0), s0_n = load_s(w.kb0, blk0, have0), s1_n = load_s(w.kb0, blk1, have1);
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
         const float f = f_n, s0 = s0_n, s1 = s1_n;
-        if (kb + 1 < p.kblocks) {
+        if (kb + 1 < w.kb1) {
           f_n = load_fac(kb + 1);
           s0_n = load_s(kb + 1, blk0, have0);
           s1_n = load_s(kb + 1, blk1, have1);
@@ -331,39 +417,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       if (!ok) break;
-      // epilogue: 1/rms of the raw row (FlashNorm's deferred normalisation), then SwiGLU
-      if (live) {
-        const float r = inv_rms(ssq, p.inv_d, p.eps);
-        if constexpr (SWIGLU) {
-          // chunk 0 holds gate columns, chunk 1 the matching up columns
-          __nv_bfloat16* yrow = p.y + static_cast<int64_t>(row) * p.nout + nb * (BN / 2) + half * 64;
+      if (w.split) {   // the CTA's last item: its partner holds the other half of the k range
+        split_pending = true;
+        s_row = row;
+        s_nb = nb;
+        s_ssq = ssq;
+        break;
+      }
+      if (live) store_tile_half<SWIGLU>(p, acc, row, nb, half, ssq);
+    }
+    if (p.split_tail) {
+      // Both CTAs of the cluster are past their main loops (their loads have
+      // landed and their MMAs completed), so the pipeline memory of each is
+      // free.  Each CTA finishes one column half of a split tile: rank r the
+      // half r.  The other half's partial sums go to the partner's shared
+      // memory, [pair j][tile row] in 8-byte words, and come back added in a
+      // fixed order (fp32 a + b is the same either way round).
+      const uint32_t rank = blockIdx.x & 1u;
+      cluster_sync_all();
+      if (split_pending && static_cast<uint32_t>(half) != rank) {
+        const uint32_t dst = dsmem_addr(smem, rank ^ 1u) + 8u * static_cast<uint32_t>(q * 32 + lane);
 #pragma unroll
-          for (int g16 = 0; g16 < 8; ++g16) {
-            uint32_t o[4];
+        for (int j = 0; j < 64; ++j) st_cluster_u64(dst + 1024u * j, acc[j]);
+      }
+      cluster_sync_all();
+      if (split_pending && static_cast<uint32_t>(half) == rank && ok && s_row < p.M) {
+        const uint64_t* src = reinterpret_cast<const uint64_t*>(smem) + (q * 32 + lane);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint64_t gv = acc[g16 * 4 + j], uv = acc[32 + g16 * 4 + j];
-              const float g0 = f2_lo(gv) * r, g1 = f2_hi(gv) * r, u0 = f2_lo(uv) * r, u1 = f2_hi(uv) * r;
-              o[j] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
-            }
-            reinterpret_cast<uint4*>(yrow)[g16] = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-        } else {
-          const int col0 = nb * BN + half * 128;
-          if (col0 < p.nout) {
-            __nv_bfloat16* yrow = p.y + static_cast<int64_t>(row) * p.nout + col0;
-#pragma unroll
-            for (int g16 = 0; g16 < 16; ++g16) {
-              uint32_t o[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint64_t v = acc[g16 * 4 + j];
-                o[j] = pack_bf16x2(f2_lo(v) * r, f2_hi(v) * r);
-              }
-              reinterpret_cast<uint4*>(yrow)[g16] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-          }
-        }
+        for (int j = 0; j < 64; ++j) acc[j] = f2_add(acc[j], src[128 * j]);
+        store_tile_half<SWIGLU>(p, acc, s_row, s_nb, half, s_ssq);
       }
     }
   }
@@ -376,13 +458,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+template <bool SWIGLU>
+cudaError_t launch_kernel(int grid, cudaStream_t stream, const CUtensorMap& th, const CUtensorMap& tl,
+                          const CUtensorMap& tw, const Params& p) {
+  constexpr size_t SMEM = smem_bytes();
+  const cudaError_t e = ensure_smem_limit<tc8_kernel<SWIGLU>>(static_cast<int>(SMEM));
+  if (e != cudaSuccess) return e;
+  if (p.split_tail)
+    return launch_pdl_cluster(tc8_kernel<SWIGLU>, static_cast<unsigned>(grid), 2, NUM_THREADS, SMEM, stream, th, tl,
+                              tw, p);
+  return launch_pdl(tc8_kernel<SWIGLU>, grid, NUM_THREADS, SMEM, stream, th, tl, tw, p);
+}
+
 }  // namespace tc8
 
 size_t tc8_workspace_bytes(int64_t M, int64_t d) {
   const size_t planes = (static_cast<size_t>(M) * d + 255) / 256 * 256;
   const size_t facb = (static_cast<size_t>(d / tc8::BKQ) * M * 4 + 255) / 256 * 256;
-  const size_t ssqb = (static_cast<size_t>(M) * 4 + 255) / 256 * 256;
-  return kWsHeaderBytes + 2 * planes + facb + ssqb;
+  return kWsHeaderBytes + 2 * planes + 2 * facb;   // x_hi, x_lo, 2^-e, partial sums of squares
 }
 
 cudaError_t launch_tc8(const CallArgs& a) {
@@ -394,11 +487,12 @@ cudaError_t launch_tc8(const CallArgs& a) {
   uint8_t* xhi = ws + kWsHeaderBytes;
   uint8_t* xlo = xhi + planes;
   float* fac = reinterpret_cast<float*>(xlo + planes);
-  float* ssq = reinterpret_cast<float*>(xlo + planes + facb);
+  float* ssq_part = reinterpret_cast<float*>(xlo + planes + facb);
 
   const int M = static_cast<int>(a.M), d = static_cast<int>(a.d);
-  cudaError_t e = launch_pdl(xsplit_rows_kernel, static_cast<unsigned>((M + 7) / 8), 256, 0, a.stream,
-                             static_cast<const __nv_bfloat16*>(a.x), M, d, xhi, xlo, fac, ssq);
+  const long long warps = static_cast<long long>(M) * (d / BKQ);
+  cudaError_t e = launch_pdl(xsplit_rows_kernel, static_cast<unsigned>((warps + 7) / 8), 256, 0, a.stream,
+                             static_cast<const __nv_bfloat16*>(a.x), M, d, xhi, xlo, fac, ssq_part);
   if (e != cudaSuccess) return e;
 
   CUtensorMap th, tl, tw;
@@ -423,17 +517,18 @@ cudaError_t launch_tc8(const CallArgs& a) {
   p.withhold = a.withhold;
   p.scales = a.scales;
   p.fac = fac;
-  p.ssq = ssq;
-  const int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
-  constexpr size_t SMEM = smem_bytes();
-  if (a.swiglu) {
-    e = ensure_smem_limit<tc8_kernel<true>>(static_cast<int>(SMEM));
-    if (e != cudaSuccess) return e;
-    return launch_pdl(tc8_kernel<true>, grid, NUM_THREADS, SMEM, a.stream, th, tl, tw, p);
-  }
-  e = ensure_smem_limit<tc8_kernel<false>>(static_cast<int>(SMEM));
-  if (e != cudaSuccess) return e;
-  return launch_pdl(tc8_kernel<false>, grid, NUM_THREADS, SMEM, a.stream, th, tl, tw, p);
+  p.ssq_part = ssq_part;
+  // Whole waves of tiles over all SMs; a last partial wave that would leave
+  // more than half of the SMs idle is split in k between CTA pairs instead.
+  const int G = a.num_sms & ~1;
+  const int W = p.num_tiles / G, R = p.num_tiles % G;
+  p.split_tail = (R > 0 && 2 * R <= G && p.kblocks >= 2) ? 1 : 0;
+  p.full_waves = W;
+  p.tail = R;
+  int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
+  if (p.split_tail) grid = W > 0 ? G : 2 * R;
+  if (a.swiglu) return launch_kernel<true>(grid, a.stream, th, tl, tw, p);
+  return launch_kernel<false>(grid, a.stream, th, tl, tw, p);
 }
 
 }  // namespace fn
