@@ -199,9 +199,12 @@ def kernel_source_hash(names):
     return h.hexdigest()[:16]
 
 
-def profile_traffic(profile_name: str, src_hash: str):
+def profile_traffic(profile_name: str, src_hash: str, M=None):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source; None otherwise."""
+    the current kernel source; None otherwise.  A summary may give the bytes
+    per M ("dram_bytes_per_launch_M256"); the plain key is the figure for the
+    workload's own mix of M (the main line).  A record whose M the summary
+    does not cover gets None."""
     path = os.path.join(ROOT, "profiles", profile_name)
     try:
         kv = {}
@@ -212,6 +215,9 @@ def profile_traffic(profile_name: str, src_hash: str):
                     kv[k.strip().strip("-* ")] = v.strip().strip("`")
         if kv.get("source_sha256") != src_hash:
             return None
+        if M is not None:
+            v = kv.get(f"dram_bytes_per_launch_M{M}")
+            return float(v) if v is not None else None
         return float(kv["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
         return None
@@ -468,7 +474,7 @@ def roofline_entry(units_per_call: float, us_per_call: float, hbm_bound: bool, p
             "flops_per_launch": units_per_call, "avg_launch_us": us_per_call}
 
 
-def kernel_for(wl: WL.Workload, M: int, out: str):
+def kernel_for(wl: WL.Workload, M: int, out: str, per_m: bool = True):
     """Name of the dominant kernel of a call, its sources and its ncu summary file."""
     if M <= 64:
         kname, src = {"bf16": ("decode_kernel", "decode.cu"), "fp8_e4m3_b128": ("decode_fp8_kernel", "decode_fp8.cu"),
@@ -488,7 +494,7 @@ def kernel_for(wl: WL.Workload, M: int, out: str):
         label = kname + (" (after the dequantise-once kernel)" if once else "")
     src_hash = kernel_source_hash(sources)
     prof = f"{kname}_{wl.name}{'_nvfp4' if out == 'nvfp4' else ''}.md"
-    return kname, label, src_hash, profile_traffic(prof, src_hash)
+    return kname, label, src_hash, profile_traffic(prof, src_hash, M if per_m else None)
 
 
 # Same-run records for the rest of the metric: the prefill half (tensor-bound
@@ -662,7 +668,7 @@ def main():
                                   world, dev)
     gpu_launches = K * kernels_per_step
     us_per_call = max_over_ranks(elapsed_ms, world, dev) / (K * n_calls) * 1e3
-    kname, label, src_hash, traffic = kernel_for(wl, max(Ms), args.out)
+    kname, label, src_hash, traffic = kernel_for(wl, max(Ms), args.out, per_m=len(Ms) == 1)
     ck = clocks.summary()
     units_per_call = (bytes_per_step if hbm_bound else flops_per_step) / n_calls
     roofline = roofline_entry(units_per_call, us_per_call, hbm_bound, peaks, peaks_kind, ck,

@@ -417,9 +417,6 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
-__device__ __forceinline__ void st_cluster_u64(uint32_t cluster_addr, uint64_t v) {
-  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(cluster_addr), "l"(v) : "memory");
-}
 
 // Arrive once on `bar` when all previously issued tcgen05 operations of this
 // thread have completed (their smem operands may then be overwritten).

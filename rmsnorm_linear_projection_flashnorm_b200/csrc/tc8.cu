@@ -121,6 +121,11 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int
   nb = r / gm;
 }
 
+// Store 8 bytes into another CTA's shared memory (a shared::cluster address).
+__device__ __forceinline__ void st_cluster_u64(uint32_t cluster_addr, uint64_t v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(cluster_addr), "l"(v) : "memory");
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long budget) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
