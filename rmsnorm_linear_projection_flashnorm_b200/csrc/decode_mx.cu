@@ -17,9 +17,13 @@
 // over the partial sums.  The bf16 activations enter the same way as on the
 // fp8 path, exactly: per row and 32-deep k block, x * 2^e (largest magnitude
 // in [128, 256)) is split into hi = e4m3(x 2^e) and lo = e4m3(x 2^e - hi);
-// the two parts share the scale 2^-e, so the hi MMA and the lo MMA accumulate
-// into the same columns.  A small kernel splits x once per call (codes, scale
-// bytes, and each row's sum of squares per 128-deep k group).
+// the two parts share the scale 2^-e.  x_hi and x_lo rows are stacked as the
+// 2 x MPAD rows of one B operand (each with its row's scale byte), so one MMA
+// per 32-deep k step gives both parts in adjacent accumulator columns, which
+// the epilogue adds: an M = 128 MMA costs about the same for any N <= 64, so
+// the stacked form halves the MMA time per weight byte.  A small kernel splits
+// x once per call (codes, scale bytes, and each row's sum of squares per
+// 128-deep k group).
 //
 // The weight stream, the stream-K split over all SMs and the fix-up kernel
 // for tiles whose k range spans CTAs are those of the other decode kernels
@@ -56,9 +60,12 @@ struct Cfg {
   static constexpr int STAGE_BYTES = (W_BYTES + X_BYTES + SF_BYTES + 1023) / 1024 * 1024;
   static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-  static constexpr int ACC_COLS = HALVES * MPAD;                      // one accumulator buffer
+  static constexpr int ACC_COLS = HALVES * 2 * MPAD;                  // one buffer: [half][hi | lo rows]
   static constexpr int SF_COLS = (HALVES + 1) * 4;                    // TMEM scale words per stage
-  static constexpr int SF_BASE = 2 * ACC_COLS;                        // after the two accumulator buffers
+  // two accumulator buffers (the epilogue of one segment overlaps the next
+  // segment's MMAs) when they fit TMEM beside the scale words, else one
+  static constexpr int NBUF = 2 * ACC_COLS + STAGES * SF_COLS <= 512 ? 2 : 1;
+  static constexpr int SF_BASE = NBUF * ACC_COLS;                     // after the accumulator buffers
   static constexpr int TMEM_NEED = SF_BASE + STAGES * SF_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                    : TMEM_NEED <= 256 ? 256 : 512;
@@ -87,9 +94,10 @@ struct alignas(16) Bars {
 // Split x once per call: one warp per (128-deep k group, padded row); lane l
 // takes k values 4l .. 4l+3, so each group of 8 lanes holds one 32-deep scale
 // block.  Writes the x_hi row r and x_lo row MPAD + r of the group's operand
-// slab, the row's scale byte 127 - e for each block in the group's chunk
-// (line r mod 32, word r div 32, byte = block), and the row's sum of squares
-// over the group.  Padding rows are zero with scale byte 127.
+// slab, the row's scale byte 127 - e for each block in the group's chunk at
+// both operand rows r and MPAD + r (line row mod 32, word row div 32, byte =
+// block), and the row's sum of squares over the group.  Padding rows are zero
+// with scale byte 127.
 template <int MPAD>
 __global__ void __launch_bounds__(256) mxsplit_kernel(const Params p) {
   grid_launch_dependents();     // the decode kernel may set up meanwhile
@@ -126,9 +134,13 @@ __global__ void __launch_bounds__(256) mxsplit_kernel(const Params p) {
   *reinterpret_cast<uint32_t*>(slab + row * BKQ + lane * 4) = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
   *reinterpret_cast<uint32_t*>(slab + (MPAD + row) * BKQ + lane * 4) =
       static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
-  if ((lane & 7) == 0)
-    p.xsf[static_cast<int64_t>(kg) * SF_CHUNK + 16 * (row & 31) + 4 * (row >> 5) + (lane >> 3)] =
-        static_cast<uint8_t>(live ? 127 - e : 127);
+  if ((lane & 7) == 0) {
+    const uint8_t sb = static_cast<uint8_t>(live ? 127 - e : 127);
+    uint8_t* chunk = p.xsf + static_cast<int64_t>(kg) * SF_CHUNK + (lane >> 3);
+    const int rl = MPAD + row;   // the same row's x_lo operand row
+    chunk[16 * (row & 31) + 4 * (row >> 5)] = sb;
+    chunk[16 * (rl & 31) + 4 * (rl >> 5)] = sb;
+  }
   if (lane == 0) p.xfac[static_cast<int64_t>(kg) * MPAD + row] = live ? ss : 0.f;
 }
 
@@ -246,8 +258,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int tile = static_cast<int>(it / p.kblocks);
         const int kb0 = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
         const int kb1 = static_cast<int>(min(static_cast<long long>(p.kblocks), kb0 + (it1 - it)));
-        const int b = seg & 1;
-        if (!mbar_wait(&bars.acc_empty[b], ((seg >> 1) & 1) ^ 1u, ctl, dec::kSiteMmaAccEmpty)) break;
+        const int b = seg % C::NBUF;
+        if (!mbar_wait(&bars.acc_empty[b], ((seg / C::NBUF) & 1) ^ 1u, ctl, dec::kSiteMmaAccEmpty)) break;
         tc_fence_after();
         for (int kg = kb0; kg < kb1; ++kg) {
           if (!mbar_wait(&bars.full[s], ph, ctl, dec::kSiteMmaFull)) { ok = false; break; }
@@ -262,18 +274,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BKQ / 32; ++kk) {
             // A = q^T: 128 weight columns (one 128-byte swizzle row), MN-major, 8-row
-            //     k groups 1024 B apart, so K = 32 is 4096 B.  B = x_hi or x_lo rows,
-            //     K-major; the scale byte of this 32-deep block is byte kk of each word.
-            const uint32_t idesc = idesc_mx_e4m3(128, MPAD, /*a MN-major*/ true, /*b MN-major*/ false, kk);
+            //     k groups 1024 B apart, so K = 32 is 4096 B.  B = the x_hi rows
+            //     followed by the x_lo rows, K-major; the scale byte of this 32-deep
+            //     block is byte kk of each word.
+            const uint32_t idesc = idesc_mx_e4m3(128, 2 * MPAD, /*a MN-major*/ true, /*b MN-major*/ false, kk);
 #pragma unroll
             for (int h = 0; h < HALVES; ++h) {
-              const uint32_t d_tmem = tmem_base + (b * HALVES + h) * MPAD;
+              const uint32_t d_tmem = tmem_base + (b * HALVES + h) * 2 * MPAD;
               const uint64_t adesc = sdesc_sw128(w0 + h * WQ_BOX + kk * 4096, WQ_BOX, 1024);
               const uint32_t acc = (kg != kb0 || kk != 0) ? 1u : 0u;
               umma_mx_e4m3(d_tmem, adesc, sdesc_sw128(x0 + kk * 32, 16, 1024), idesc, sf_t + 4 * h,
                            sf_t + 4 * HALVES, acc);
-              umma_mx_e4m3(d_tmem, adesc, sdesc_sw128(x0 + MPAD * BKQ + kk * 32, 16, 1024), idesc, sf_t + 4 * h,
-                           sf_t + 4 * HALVES, 1u);
             }
           }
           umma_commit(&bars.empty[s]);
@@ -335,24 +346,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int kb0 = static_cast<int>(it - static_cast<long long>(tile) * p.kblocks);
       const int kb1 = static_cast<int>(min(static_cast<long long>(p.kblocks), kb0 + (it1 - it)));
       it += kb1 - kb0;
-      const int b = seg & 1;
-      const uint32_t aph = (seg >> 1) & 1;
+      const int ab = seg % C::NBUF;               // accumulator buffer
+      const uint32_t aph = (seg / C::NBUF) & 1;
+      const int b = seg & 1;                      // sums-of-squares buffer
+      const uint32_t sph = (seg >> 1) & 1;
       // One thread waits and the whole epilogue group follows its decision, so
       // the group never splits at the named barriers or the .sync.aligned loads.
       if (et == 0) {
-        bool ok = mbar_wait(&bars.acc_full[b], aph, ctl, dec::kSiteEpiAccFull);
-        ok = ok && mbar_wait(&bars.ssq_full[b], aph, ctl, dec::kSiteEpiSsqFull);
+        bool ok = mbar_wait(&bars.acc_full[ab], aph, ctl, dec::kSiteEpiAccFull);
+        ok = ok && mbar_wait(&bars.ssq_full[b], sph, ctl, dec::kSiteEpiSsqFull);
         bars.epi_ok[seg & 1] = ok ? 1 : 0;
       }
       named_bar_sync(1, 128);
       if (!bars.epi_ok[seg & 1]) break;
       tc_fence_after();
+      // each half's x_hi columns plus its x_lo columns, 16 rows at a time
       float acc[HALVES][MPAD];
 #pragma unroll
-      for (int h = 0; h < HALVES; ++h)
-        dec::tmem_ld_cols<MPAD>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (b * HALVES + h) * MPAD, acc[h]);
+      for (int h = 0; h < HALVES; ++h) {
+        const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (ab * HALVES + h) * 2 * MPAD;
+#pragma unroll
+        for (int m0 = 0; m0 < MPAD; m0 += 16) {
+          uint32_t hv[16], lv[16];
+          tmem_ld16(ta + m0, hv);
+          tmem_ld16(ta + MPAD + m0, lv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc[h][m0 + j] = __uint_as_float(hv[j]) + __uint_as_float(lv[j]);
+        }
+      }
       tc_fence_before();
-      mbar_arrive(&bars.acc_empty[b]);
+      mbar_arrive(&bars.acc_empty[ab]);
       // A row holding a non-finite activation in this k range has a non-finite
       // sum of squares; its (saturated) products become NaN, as they would in
       // a bf16 matmul.
