@@ -150,10 +150,27 @@ def test_workspace_size_is_monotone_in_m_bucket(L):
     assert fnb.fn_workspace_size(8, 4096, 14336, 0, 1) > fnb.fn_workspace_size(8, 4096, 14336, 0, 0)
 
 
+def test_workspace_size_fp8_tile_path(L):
+    """fp8 weights above 64 rows: the header, the x_hi and x_lo code planes
+    (M d bytes each), and per (row, 128-deep k block) 2^-e and a partial sum
+    of squares; from 1024 rows at least the bf16 weight copy that the NVFP4
+    and partial outputs use.  The fixed 8 MiB array of the no-allocation entry
+    point therefore cannot hold fp8 at 8192 rows of the fp8 workload."""
+    fp8 = fnb.FN_W_FP8_E4M3_B128
+    r256 = lambda n: (n + 255) // 256 * 256
+    M, d, N = 256, 5120, 13824
+    assert fnb.fn_workspace_size(M, d, N, fp8, 1) == 256 + 2 * r256(M * d) + 2 * r256((d // 128) * M * 4)
+    assert fnb.fn_workspace_size(8192, d, N, fp8, 1) >= 256 + d * 2 * N * 2
+    assert fnb.fn_workspace_size(8192, d, N, fp8, 0) > 8 << 20
+    assert fnb.fn_workspace_size(65, 1024, 1024, fp8, 0) <= 8 << 20
+
+
 def test_set_debug_validates_keys(L):
     assert fnb.fn_set_debug(99, 1) == fnb.FN_ERR_INVALID_ARG
     assert fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 0) == fnb.FN_ERR_INVALID_ARG
     assert fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 5) == fnb.FN_ERR_INVALID_ARG
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 4) == fnb.FN_OK
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 0) == fnb.FN_OK
     assert fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 2_000_000_000) == fnb.FN_OK
 
 

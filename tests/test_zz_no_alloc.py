@@ -80,9 +80,10 @@ def test_static_scratch_matches_workspace_entry_point(M, d, N, fp8):
 
 def test_static_scratch_rejects_sizes_beyond_its_maximum():
     # M = 64 on the decode QKV shape needs about 9.8 MB of split-K partials on
-    # 148 SMs, more than the 8 MiB array; fp8 weights at M >= 1024 need a bf16
-    # copy of the weight.  Small real buffers stand in for the operands: the
-    # size check rejects the call before anything is launched.
+    # 148 SMs, more than the 8 MiB array; fp8 weights at 8192 rows need the
+    # split activations (84 MB) and, for NVFP4 or partial outputs, a bf16 copy
+    # of the weight.  Small real buffers stand in for the operands: the size
+    # check rejects the call before anything is launched.
     d, N = 4096, 6144
     assert fnb.fn_workspace_size(64, d, N, fnb.FN_W_BF16, 0) > STATIC_BYTES
     assert fnb.fn_workspace_size(32, d, N, fnb.FN_W_BF16, 0) <= STATIC_BYTES
