@@ -476,12 +476,13 @@ def roofline_entry(units_per_call: float, us_per_call: float, hbm_bound: bool, p
 
 def kernel_for(wl: WL.Workload, M: int, out: str, per_m: bool = True):
     """Name of the dominant kernel of a call, its sources and its ncu summary file."""
-    if M <= 64:
+    promotion = wl.wtype == "fp8_e4m3_b128" and out == "bf16" and M >= 48   # the library's fp8 tile threshold
+    if M <= 64 and not promotion:
         kname, src = {"bf16": ("decode_kernel", "decode.cu"), "fp8_e4m3_b128": ("decode_fp8_kernel", "decode_fp8.cu"),
                       "mxfp8_e4m3": ("decode_mx_kernel", "decode_mx.cu")}[wl.wtype]
         sources = [src, "decode_common.cuh", "ptx.cuh", "nvfp4.cuh"]
         label = f"{kname} (+ decode_fixup_kernel where a tile's k range is split)"
-    elif wl.wtype == "fp8_e4m3_b128" and out == "bf16":
+    elif promotion:
         # x split once per call, then the block-scale promotion kernel
         kname, sources = "tc8_kernel", ["tc8.cu", "ptx.cuh"]
         label = "tc8_kernel (after xsplit_rows_kernel)"

@@ -191,6 +191,8 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
 
   int force = g_force_path.load();
   bool use_decode = M <= 64 && !adaln;   // AdaLN runs on the tile kernel at every M
+  // fp8 weights with bf16 output: the promotion tile kernel from kFp8PromotionMinM rows
+  if (wt == FN_W_FP8_E4M3_B128 && M >= kFp8PromotionMinM && !fp4 && !partial && force != 4) use_decode = false;
   if (force == 1) {
     if (M > 64 || adaln) return FN_ERR_INVALID_ARG;
     use_decode = true;
@@ -316,7 +318,13 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
     }
     return kWsHeaderBytes;
   }
-  return decode_workspace_bytes(M, d, ncols, swiglu != 0, current_sms_or_default(), static_cast<int>(wt));
+  const size_t dec = decode_workspace_bytes(M, d, ncols, swiglu != 0, current_sms_or_default(), static_cast<int>(wt));
+  if (wt == FN_W_FP8_E4M3_B128 && M >= kFp8PromotionMinM) {
+    // bf16 output runs the promotion kernel; NVFP4 and partial outputs the decode kernel
+    const size_t t8 = tc8_workspace_bytes(M, d);
+    return t8 > dec ? t8 : dec;
+  }
+  return dec;
 }
 
 fn_status fn_norm_proj(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
