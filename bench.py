@@ -476,7 +476,8 @@ def roofline_entry(units_per_call: float, us_per_call: float, hbm_bound: bool, p
 
 def kernel_for(wl: WL.Workload, M: int, out: str, per_m: bool = True):
     """Name of the dominant kernel of a call, its sources and its ncu summary file."""
-    promotion = wl.wtype == "fp8_e4m3_b128" and out == "bf16" and M >= 48   # the library's fp8 tile threshold
+    # the library's promotion-kernel thresholds: fp8 from 48 rows, MXFP8 above 64
+    promotion = out == "bf16" and ((wl.wtype == "fp8_e4m3_b128" and M >= 48) or (wl.wtype == "mxfp8_e4m3" and M > 64))
     if M <= 64 and not promotion:
         kname, src = {"bf16": ("decode_kernel", "decode.cu"), "fp8_e4m3_b128": ("decode_fp8_kernel", "decode_fp8.cu"),
                       "mxfp8_e4m3": ("decode_mx_kernel", "decode_mx.cu")}[wl.wtype]
@@ -485,7 +486,8 @@ def kernel_for(wl: WL.Workload, M: int, out: str, per_m: bool = True):
     elif promotion:
         # x split once per call, then the block-scale promotion kernel
         kname, sources = "tc8_kernel", ["tc8.cu", "ptx.cuh"]
-        label = "tc8_kernel (after xsplit_rows_kernel)"
+        label = "tc8_kernel (after xsplit_rows_kernel)" if wl.wtype == "fp8_e4m3_b128" else \
+            "tc8_kernel, block-scaled MMAs (after xsplit_mx_rows_kernel)"
     else:
         once = wl.wtype == "mxfp8_e4m3" or (wl.wtype != "bf16" and M >= 1024)
         # bf16 weights (or a bf16 copy) at M >= 512 with bf16 output run on pairs of SMs
@@ -503,6 +505,7 @@ def kernel_for(wl: WL.Workload, M: int, out: str, per_m: bool = True):
 # and unfused chain.
 SUB_RECORDS = (
     ("ffn_swiglu", 4096), ("prefill_swiglu_large", 16384), ("fp8_swiglu", 8192), ("fp8_swiglu", 256),
+    ("mxfp8_swiglu", 8192), ("mxfp8_swiglu", 256),
     ("ffn_swiglu", 16), ("fp8_swiglu", 1), ("fp8_swiglu", 64), ("mxfp8_swiglu", 1), ("mxfp8_swiglu", 64),
 )
 

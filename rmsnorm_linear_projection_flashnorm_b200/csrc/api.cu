@@ -203,18 +203,19 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   int sms = 0;
   fn_status st = check_device(sms);
   if (st != FN_OK) return st;
-  // fp8 weights with bf16 output on the tile path: the block-scale promotion
-  // kernel (tc8.cu), which multiplies the stored e4m3 codes.  The other tile
-  // forms with fp8 weights (NVFP4 or partial output, AdaLN, or forced) convert
-  // the staged weight tiles to bf16 (M < kFp8DequantOnceM) or the whole weight
-  // once per call into the workspace; MXFP8 weights on the tile path take the
-  // latter route.
-  const bool fp8_tc8 = !use_decode && wt == FN_W_FP8_E4M3_B128 && !adaln && !fp4 && !partial && force != 4;
+  // fp8 and MXFP8 weights with bf16 output on the tile path: the promotion
+  // kernel (tc8.cu), which multiplies the stored e4m3 codes (fp8: block scales
+  // applied per 128-deep k block in registers; MXFP8: block-scaled MMAs).  The
+  // other tile forms with 8-bit weights (NVFP4 or partial output, AdaLN, or
+  // forced) convert the staged fp8 weight tiles to bf16 (M < kFp8DequantOnceM)
+  // or the whole weight once per call into the workspace (MXFP8 always).
+  const bool fp8_tc8 = !use_decode && (wt == FN_W_FP8_E4M3_B128 || wt == FN_W_MXFP8_E4M3) && !adaln && !fp4 &&
+                       !partial && force != 4;
   const bool dequant_once =
       !use_decode && !fp8_tc8 &&
       ((wt == FN_W_FP8_E4M3_B128 && (M >= kFp8DequantOnceM || adaln)) || wt == FN_W_MXFP8_E4M3);
   const size_t need = use_decode     ? decode_workspace_bytes(M, d, ncols, swiglu, sms, static_cast<int>(wt))
-                      : fp8_tc8      ? tc8_workspace_bytes(M, d)
+                      : fp8_tc8      ? tc8_workspace_bytes(M, d, wt == FN_W_MXFP8_E4M3)
                       : dequant_once ? kWsHeaderBytes + wbytes * 2
                                      : kWsHeaderBytes;
   if (ws_bytes < need) return FN_ERR_WORKSPACE;
@@ -309,7 +310,12 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
   const int64_t ncols = swiglu ? 2 * N : N;
   if (M > 64) {
     const size_t copy = kWsHeaderBytes + static_cast<size_t>(d) * static_cast<size_t>(ncols) * 2;
-    if (wt == FN_W_MXFP8_E4M3) return copy;
+    if (wt == FN_W_MXFP8_E4M3) {
+      // the promotion kernel's split x and scale chunks, or (NVFP4, partial
+      // or AdaLN output) the dequantised weight
+      const size_t t8 = tc8_workspace_bytes(M, d, true);
+      return copy > t8 ? copy : t8;
+    }
     if (wt == FN_W_FP8_E4M3_B128) {
       // the promotion kernel's split x, or (NVFP4 / partial output at large M)
       // the dequantised weight

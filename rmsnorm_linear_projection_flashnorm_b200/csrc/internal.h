@@ -89,8 +89,10 @@ cudaError_t launch_tc_pair(const CallArgs& a);
 constexpr int64_t kPairTileMinM = 512;
 // fp8 weights (128x128 block scales) at M > 64 with bf16 output: x split once
 // into exact e4m3 hi/lo planes, the stored codes multiplied as they are, the
-// block scales applied per 128-deep k block to fp32 sums (tc8.cu).
-size_t tc8_workspace_bytes(int64_t M, int64_t d);
+// block scales applied per 128-deep k block to fp32 sums (tc8.cu).  MXFP8
+// weights: the split per 32-deep block, its powers of two as ue8m0 x scales,
+// block-scaled MMAs over a tile's whole k range (mx = true).
+size_t tc8_workspace_bytes(int64_t M, int64_t d, bool mx = false);
 cudaError_t launch_tc8(const CallArgs& a);
 // fp8 weights with bf16 output take the promotion kernel from this many rows:
 // at 48 and 64 rows of the fp8 SwiGLU workload (d=5120, N=13824) it ran 5-10 %

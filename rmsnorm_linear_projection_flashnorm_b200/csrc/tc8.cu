@@ -48,10 +48,14 @@ namespace tc8 {
 constexpr int BM = 128, BN = 256, BKQ = 128;
 constexpr int XQ_BYTES = BM * BKQ;                    // one e4m3 code plane tile: 128 rows x 128 k (16 KB)
 constexpr int WQ_BOX = 128 * BKQ;                     // 128 weight columns x 128 k rows (16 KB)
-constexpr int STAGE_BYTES = 2 * XQ_BYTES + 2 * WQ_BOX;   // x_hi, x_lo, weight: 64 KB
+constexpr int OPERAND_BYTES = 2 * XQ_BYTES + 2 * WQ_BOX;   // x_hi, x_lo, weight: 64 KB
+constexpr int SF_CHUNK = 512;                         // MXFP8: 128 rows or columns x 4 scale bytes
+// MXFP8 stages also hold the x scale chunk and the two weight scale chunks
+template <bool MX> __host__ __device__ constexpr int stage_bytes() { return OPERAND_BYTES + (MX ? 2048 : 0); }
 constexpr int STAGES = 3;
 constexpr int NUM_THREADS = 320;
-constexpr int TMEM_COLS = 2 * BN;                     // two per-k-block accumulators
+constexpr int TMEM_COLS = 2 * BN;   // fp8: two per-k-block accumulators; MXFP8: one accumulator + scales
+constexpr int SF_TMEM = BN;         // MXFP8: per stage 12 scale words (x, then two weight chunks) from here
 constexpr int GROUP_M = 16;                           // tile raster: bands of 16 row blocks
 
 enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteScaleAccFull };
@@ -67,6 +71,8 @@ struct Params {
   const float* scales;   // weight block scales [kblocks][nblk]
   const float* fac;      // 2^-e of each (k block, row) of the split [kblocks][M]; NaN: non-finite block
   const float* ssq_part; // sum of squares of each (k block, row) [kblocks][M]
+  const uint8_t* wsf;    // MXFP8: weight scale chunks [kblocks][nblk][512] (none for fp8)
+  const uint8_t* xsf;    // MXFP8: x scale chunks [kblocks][num_m][512]
   int split_tail;        // 1: launched as 2-CTA clusters; the tiles after the full waves are split in k
   int full_waves;        //   between the two CTAs of a cluster (tile full_waves * grid + cluster index)
   int tail;              //   number of such tiles (<= clusters)
@@ -108,8 +114,9 @@ struct alignas(8) Bars {
   int abort_flag;
 };
 
-constexpr size_t smem_bytes() { return 1024 + STAGES * STAGE_BYTES + sizeof(Bars); }
-static_assert(smem_bytes() <= 232448, "shared memory budget");
+template <bool MX> constexpr size_t smem_bytes() { return 1024 + STAGES * stage_bytes<MX>() + sizeof(Bars); }
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
+static_assert(SF_TMEM + STAGES * 12 <= TMEM_COLS, "MXFP8 scale words fit TMEM beside the accumulator");
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
   const int per_group = GROUP_M * p.num_n;
@@ -180,6 +187,56 @@ __global__ void __launch_bounds__(256) xsplit_rows_kernel(const __nv_bfloat16* _
   }
 }
 
+// MXFP8 weights: the same split per 32-deep block instead of per 128-deep
+// block, the power of two stored as a ue8m0 byte (127 - e) in the chunk layout
+// the block-scaled MMA reads (per 128-row block and 128-deep k group, a
+// 512-byte chunk; row r's byte for 32-deep block b at 16 (r mod 32) +
+// 4 (r div 32 mod 4) + b).  Rows from M up to the last 128-row block get
+// byte 127 (their operand rows are TMA zero fill).  The partial sums of
+// squares per (128-deep group, row) are those of the fp8 split.
+__global__ void __launch_bounds__(256) xsplit_mx_rows_kernel(const __nv_bfloat16* __restrict__ x, int M, int Mpad,
+                                                             int d, uint8_t* __restrict__ xhi,
+                                                             uint8_t* __restrict__ xlo, uint8_t* __restrict__ xsf,
+                                                             float* __restrict__ ssq_part) {
+  grid_launch_dependents();
+  grid_dependency_wait();
+  const int kblocks = d / BKQ;
+  const long long wg = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int row = static_cast<int>(wg / kblocks), kb = static_cast<int>(wg - static_cast<long long>(row) * kblocks);
+  if (row >= Mpad) return;
+  const bool live = row < M;
+  const int64_t off = static_cast<int64_t>(row) * d + kb * BKQ + lane * 4;
+  uint2 v = make_uint2(0u, 0u);
+  if (live) v = __ldg(reinterpret_cast<const uint2*>(x + off));
+  uint32_t amax = max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu), max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu));
+#pragma unroll
+  for (int o = 4; o >= 1; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));   // 8 lanes: 32 k
+  const int E = static_cast<int>(amax >> 7);
+  int e = amax == 0 ? 0 : 134 - E;
+  e = e > 126 ? 126 : (e < -126 ? -126 : e);
+  const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+  const uint64_t sc2 = f2_pack(sc, sc);
+  const uint64_t a = f2_pack_u(v.x << 16, v.x & 0xFFFF0000u), b = f2_pack_u(v.y << 16, v.y & 0xFFFF0000u);
+  const uint64_t ss2 = f2_fma(b, b, f2_mul(a, a));
+  if (live) {
+    uint16_t h0, l0, h1, l1;
+    split_e4m3x2(f2_mul(a, sc2), h0, l0);
+    split_e4m3x2(f2_mul(b, sc2), h1, l1);
+    *reinterpret_cast<uint32_t*>(xhi + off) = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+    *reinterpret_cast<uint32_t*>(xlo + off) = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+  }
+  if ((lane & 7) == 0) {
+    const int r = row & 127;
+    xsf[(static_cast<int64_t>(kb) * (Mpad / BM) + row / BM) * SF_CHUNK + 16 * (r & 31) + 4 * (r >> 5) + (lane >> 3)] =
+        static_cast<uint8_t>(live ? 127 - e : 127);
+  }
+  float ss = f2_lo(ss2) + f2_hi(ss2);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0 && live) ssq_part[static_cast<int64_t>(kb) * M + row] = ss;
+}
+
 // Epilogue of one thread's share of a tile: row `row`, column half `half`.
 // 1/rms of the raw row (FlashNorm's deferred normalisation), then SwiGLU (the
 // two chunks hold matching gate and up columns) or the plain projection (the
@@ -187,7 +244,9 @@ __global__ void __launch_bounds__(256) xsplit_rows_kernel(const __nv_bfloat16* _
 template <bool SWIGLU>
 __device__ __forceinline__ void store_tile_half(const Params& p, const uint64_t (&acc)[64], int row, int nb, int half,
                                                 float ssq) {
-  const float r = inv_rms(ssq, p.inv_d, p.eps);
+  // a row holding inf or NaN has a non-finite sum of squares: all its
+  // outputs are NaN, as in a bf16 matmul (the fp8 factors already carry it)
+  const float r = isfinite(ssq) ? inv_rms(ssq, p.inv_d, p.eps) : __int_as_float(0x7fc00000);
   if constexpr (SWIGLU) {
     __nv_bfloat16* yrow = p.y + static_cast<int64_t>(row) * p.nout + nb * (BN / 2) + half * 64;
 #pragma unroll
@@ -221,17 +280,25 @@ __device__ __forceinline__ void store_tile_half(const Params& p, const uint64_t 
 // ---------------------------------------------------------------------------
 // The tile kernel.
 // ---------------------------------------------------------------------------
-template <bool SWIGLU>
+// MX: MXFP8 weights (e4m3 with a ue8m0 scale per 32 k values and column):
+// the same stages plus the scale chunks, block-scaled MMAs
+// (kind::mxf8f6f4.block_scale, x_hi and x_lo under the same x scales) that
+// accumulate a work item's whole k range in one TMEM accumulator, and scaler
+// warps that only read the accumulator once per item for the epilogue.
+template <bool SWIGLU, bool MX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc8_kernel(const __grid_constant__ CUtensorMap tmap_xh, const __grid_constant__ CUtensorMap tmap_xl,
                const __grid_constant__ CUtensorMap tmap_w, const Params p) {
+  constexpr int STAGE_BYTES = stage_bytes<MX>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars& bars = *reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
-  // stage: [x_hi 128 x 128][x_lo 128 x 128][weight: two 128-column boxes], 1024-byte multiples
+  // stage: [x_hi 128 x 128][x_lo 128 x 128][weight: two 128-column boxes]
+  //        (MXFP8: [x scale chunk][weight scale chunks]), 1024-byte multiples
   auto stage_xh = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stage_xl = [&](int s) { return smem + s * STAGE_BYTES + XQ_BYTES; };
   auto stage_w = [&](int s) { return smem + s * STAGE_BYTES + 2 * XQ_BYTES; };
+  auto stage_sf = [&](int s) { return smem + s * STAGE_BYTES + OPERAND_BYTES; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -280,7 +347,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tile_coords(w.t, p, mb, nb);
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&bars.empty[s], ph ^ 1, ctl, kSiteProdEmpty)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars.full[s], STAGE_BYTES);
+          mbar_arrive_expect_tx(&bars.full[s], OPERAND_BYTES + (MX ? 3 * SF_CHUNK : 0));
+          if constexpr (MX) {
+            // x scale chunk of (k group, row block); weight chunks of the tile's two
+            // 128-column blocks (a block past the weight reuses the last chunk:
+            // its weight box is zero fill)
+            bulk_load(stage_sf(s), p.xsf + (static_cast<int64_t>(kb) * p.num_m + mb) * SF_CHUNK, SF_CHUNK,
+                      &bars.full[s]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int cb = min(2 * nb + h, p.nblk - 1);
+              bulk_load(stage_sf(s) + (1 + h) * SF_CHUNK, p.wsf + (static_cast<int64_t>(kb) * p.nblk + cb) * SF_CHUNK,
+                        SF_CHUNK, &bars.full[s]);
+            }
+          }
           tma_load_2d(stage_xh(s), &tmap_xh, &bars.full[s], kb * BKQ, mb * BM);
           tma_load_2d(stage_xl(s), &tmap_xl, &bars.full[s], kb * BKQ, mb * BM);
           // a plain projection with an odd number of 128-column blocks has a
@@ -303,7 +383,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (MX && lane == 0) {
+      // One accumulator per work item over its whole k range.  Per stage the
+      // three scale chunks go to this stage's TMEM scale words (tcgen05.cp,
+      // ordered with the MMAs after it), then per 32-deep k step one
+      // block-scaled MMA for x_hi and one for x_lo, both under the x scales.
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      Work w;
+      for (int i = 0; ok && work_item(p, i, w); ++i) {
+        if (!mbar_wait(&bars.acce[0], (static_cast<uint32_t>(i) & 1u) ^ 1u, ctl, kSiteMmaAccEmpty)) break;
+        tc_fence_after();
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&bars.full[s], ph, ctl, kSiteMmaFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sf_t = tmem_base + SF_TMEM + s * 12;
+          const uint32_t sf_s = smem_u32(stage_sf(s));
+#pragma unroll
+          for (int c = 0; c < 3; ++c) tmem_cp_32x128b_x4(sf_t + 4 * c, sdesc_plain(sf_s + c * SF_CHUNK, 128, 128));
+          const uint32_t xh = smem_u32(stage_xh(s)), xl = smem_u32(stage_xl(s)), w0 = smem_u32(stage_w(s));
+#pragma unroll
+          for (int kk = 0; kk < BKQ / 32; ++kk) {
+            // the scale byte of this 32-deep block is byte kk of each scale word
+            const uint32_t idesc = idesc_mx_e4m3(BM, BN, /*a MN-major*/ false, /*b MN-major*/ true, kk);
+            const uint64_t bdesc = sdesc_sw128(w0 + kk * 4096, WQ_BOX, 1024);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+              const uint64_t adesc = sdesc_sw128((part == 0 ? xh : xl) + kk * 32, 16, 1024);
+              umma_mx_e4m3(tmem_base, adesc, bdesc, idesc, sf_t, sf_t + 4,
+                           (kb != w.kb0 || kk != 0 || part != 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&bars.empty[s]);
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&bars.accf[0]);
+      }
+      umma_commit(&bars.drain);
+      drain_wait(&bars.drain, 0, p.budget_ns);
+    } else if (!MX && lane == 0) {
       // A = x_hi / x_lo rows, K-major; B = e4m3 weight, N-major
       constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN, /*a MN-major*/ false, /*b MN-major*/ true);
       int s = 0;
@@ -375,6 +495,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 8
         for (int kb = 0; kb < p.kblocks; ++kb) ssq += __ldg(p.ssq_part + static_cast<int64_t>(kb) * p.M + row);
       }
+      if constexpr (MX) {
+        // the accumulator holds the item's whole sums: read it once
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.accf[0], static_cast<uint32_t>(i) & 1u, ctl,
+                                               kSiteScaleAccFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+        for (int rd = 0; rd < 4; ++rd) {
+          uint32_t v0[16], v1[16];
+          const uint32_t col = (rd < 2 ? c0 : c1) + (rd & 1) * 32;
+          tmem_ld16(taddr + col, v0);
+          tmem_ld16(taddr + col + 16, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            acc[rd * 16 + j] = f2_pack_u(v0[2 * j], v0[2 * j + 1]);
+            acc[rd * 16 + 8 + j] = f2_pack_u(v1[2 * j], v1[2 * j + 1]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && !(p.withhold && i == 0)) mbar_arrive(&bars.acce[0]);
+      } else {
 #pragma unroll
       for (int j = 0; j < 64; ++j) acc[j] = 0;
       // 2^-e and the block scales, loaded one k block ahead
@@ -421,6 +567,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      }
       if (!ok) break;
       if (w.split) {   // the CTA's last item: its partner holds the other half of the k range
         split_pending = true;
@@ -463,41 +610,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool MX>
 cudaError_t launch_kernel(int grid, cudaStream_t stream, const CUtensorMap& th, const CUtensorMap& tl,
                           const CUtensorMap& tw, const Params& p) {
-  constexpr size_t SMEM = smem_bytes();
-  const cudaError_t e = ensure_smem_limit<tc8_kernel<SWIGLU>>(static_cast<int>(SMEM));
+  constexpr size_t SMEM = smem_bytes<MX>();
+  const cudaError_t e = ensure_smem_limit<tc8_kernel<SWIGLU, MX>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
   if (p.split_tail)
-    return launch_pdl_cluster(tc8_kernel<SWIGLU>, static_cast<unsigned>(grid), 2, NUM_THREADS, SMEM, stream, th, tl,
-                              tw, p);
-  return launch_pdl(tc8_kernel<SWIGLU>, grid, NUM_THREADS, SMEM, stream, th, tl, tw, p);
+    return launch_pdl_cluster(tc8_kernel<SWIGLU, MX>, static_cast<unsigned>(grid), 2, NUM_THREADS, SMEM, stream, th,
+                              tl, tw, p);
+  return launch_pdl(tc8_kernel<SWIGLU, MX>, grid, NUM_THREADS, SMEM, stream, th, tl, tw, p);
 }
 
 }  // namespace tc8
 
-size_t tc8_workspace_bytes(int64_t M, int64_t d) {
+size_t tc8_workspace_bytes(int64_t M, int64_t d, bool mx) {
   const size_t planes = (static_cast<size_t>(M) * d + 255) / 256 * 256;
-  const size_t facb = (static_cast<size_t>(d / tc8::BKQ) * M * 4 + 255) / 256 * 256;
-  return kWsHeaderBytes + 2 * planes + 2 * facb;   // x_hi, x_lo, 2^-e, partial sums of squares
+  // per (k block, row): 2^-e of the split, or (MXFP8) the x scale chunks over
+  // whole 128-row blocks; then the partial sums of squares
+  const int64_t rows = mx ? (M + tc8::BM - 1) / tc8::BM * tc8::BM : M;
+  const size_t facb = (static_cast<size_t>(d / tc8::BKQ) * rows * 4 + 255) / 256 * 256;
+  const size_t ssqb = (static_cast<size_t>(d / tc8::BKQ) * M * 4 + 255) / 256 * 256;
+  return kWsHeaderBytes + 2 * planes + facb + ssqb;
 }
 
 cudaError_t launch_tc8(const CallArgs& a) {
   using namespace tc8;
-  if (a.ws_bytes < tc8_workspace_bytes(a.M, a.d)) return cudaErrorInvalidValue;
+  const bool mx = a.wtype == 2;   // MXFP8
+  if (a.ws_bytes < tc8_workspace_bytes(a.M, a.d, mx)) return cudaErrorInvalidValue;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  const int M = static_cast<int>(a.M), d = static_cast<int>(a.d);
+  const int Mpad = (M + BM - 1) / BM * BM;
   const size_t planes = (static_cast<size_t>(a.M) * a.d + 255) / 256 * 256;
-  const size_t facb = (static_cast<size_t>(a.d / BKQ) * a.M * 4 + 255) / 256 * 256;
+  const size_t facb = (static_cast<size_t>(a.d / BKQ) * (mx ? Mpad : M) * 4 + 255) / 256 * 256;
   uint8_t* xhi = ws + kWsHeaderBytes;
   uint8_t* xlo = xhi + planes;
   float* fac = reinterpret_cast<float*>(xlo + planes);
   float* ssq_part = reinterpret_cast<float*>(xlo + planes + facb);
 
-  const int M = static_cast<int>(a.M), d = static_cast<int>(a.d);
-  const long long warps = static_cast<long long>(M) * (d / BKQ);
-  cudaError_t e = launch_pdl(xsplit_rows_kernel, static_cast<unsigned>((warps + 7) / 8), 256, 0, a.stream,
-                             static_cast<const __nv_bfloat16*>(a.x), M, d, xhi, xlo, fac, ssq_part);
+  cudaError_t e;
+  if (mx) {
+    const long long warps = static_cast<long long>(Mpad) * (d / BKQ);
+    e = launch_pdl(xsplit_mx_rows_kernel, static_cast<unsigned>((warps + 7) / 8), 256, 0, a.stream,
+                   static_cast<const __nv_bfloat16*>(a.x), M, Mpad, d, xhi, xlo, reinterpret_cast<uint8_t*>(fac),
+                   ssq_part);
+  } else {
+    const long long warps = static_cast<long long>(M) * (d / BKQ);
+    e = launch_pdl(xsplit_rows_kernel, static_cast<unsigned>((warps + 7) / 8), 256, 0, a.stream,
+                   static_cast<const __nv_bfloat16*>(a.x), M, d, xhi, xlo, fac, ssq_part);
+  }
   if (e != cudaSuccess) return e;
 
   CUtensorMap th, tl, tw;
@@ -520,9 +681,11 @@ cudaError_t launch_tc8(const CallArgs& a) {
   p.status = reinterpret_cast<unsigned int*>(ws);
   p.budget_ns = a.budget_ns;
   p.withhold = a.withhold;
-  p.scales = a.scales;
-  p.fac = fac;
+  p.scales = mx ? nullptr : a.scales;
+  p.fac = mx ? nullptr : fac;
   p.ssq_part = ssq_part;
+  p.wsf = mx ? reinterpret_cast<const uint8_t*>(a.scales) : nullptr;
+  p.xsf = mx ? reinterpret_cast<const uint8_t*>(fac) : nullptr;
   // Whole waves of tiles over all SMs; a last partial wave that would leave
   // more than half of the SMs idle is split in k between CTA pairs instead.
   const int G = a.num_sms & ~1;
@@ -532,8 +695,10 @@ cudaError_t launch_tc8(const CallArgs& a) {
   p.tail = R;
   int grid = p.num_tiles < a.num_sms ? p.num_tiles : a.num_sms;
   if (p.split_tail) grid = W > 0 ? G : 2 * R;
-  if (a.swiglu) return launch_kernel<true>(grid, a.stream, th, tl, tw, p);
-  return launch_kernel<false>(grid, a.stream, th, tl, tw, p);
+  if (mx) return a.swiglu ? launch_kernel<true, true>(grid, a.stream, th, tl, tw, p)
+                          : launch_kernel<false, true>(grid, a.stream, th, tl, tw, p);
+  return a.swiglu ? launch_kernel<true, false>(grid, a.stream, th, tl, tw, p)
+                  : launch_kernel<false, false>(grid, a.stream, th, tl, tw, p);
 }
 
 }  // namespace fn

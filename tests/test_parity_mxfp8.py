@@ -6,8 +6,10 @@ The fold must be bit-identical to the oracle's (codes and scale bytes, plain
 and gate/up interleaved).  At M <= 64 the codes and scales go to the
 block-scaled MMAs as stored and the bf16 activations are split exactly into
 two e4m3 parts sharing a power-of-two scale, so the products are those of the
-stored weight; at M > 64 the weight is converted to bf16 once per call (an
-exact conversion, checked bit for bit) for the tile kernel.  Kernel parity is
+stored weight; at M > 64 with bf16 output the promotion tile kernel does the
+same with block-scaled MMAs over each tile's whole k range, and the other
+tile-path forms (and FN_DEBUG_FORCE_PATH 4) convert the weight to bf16 once
+per call (an exact conversion, checked bit for bit).  Kernel parity is
 therefore against the oracle on the dequantised stored weight e4m3(q) * 2^E
 (exact in fp64) with g = 1, and every case holds the bf16 bound
 1e-2 (1 + |y_ref|), tighter than the 6e-2 bound stated for fp8 weights.
@@ -104,7 +106,7 @@ def test_mxfp8_decode_m_ladder(M, swiglu):
     (40, 384, 256, True),
     (64, 128, 128, False),     # single k group, single tile
     (8, 2048, 1024, True),     # k split across CTAs: fix-up kernel
-    (200, 256, 384, False),    # tile path: the weight is converted to bf16 once
+    (200, 256, 384, False),    # tile path: block-scaled promotion kernel
     (300, 512, 384, True),
 ])
 def test_mxfp8_small(M, d, N, swiglu):
@@ -112,62 +114,62 @@ def test_mxfp8_small(M, d, N, swiglu):
     assert rel_err(y, ref) <= BF16_TOL
 
 
-def test_mxfp8_wide_dynamic_range():
-    """Activations spanning 2^-20 .. 2^12 inside one 32-deep block: the split
-    keeps them exact, so the bf16-weight bound still holds."""
-    M, d, N = 6, 512, 384
-    x = WL.activations(M, d, 172).float()
-    mult = torch.ones(d)
-    mult[0::4] = 2.0 ** 10
-    mult[1::8] = 2.0 ** -12
-    mult[3::16] = 2.0 ** -18
-    x = (x * mult).to(torch.bfloat16)
-    for swiglu in (False, True):
-        y, ref = _case(M, d, N, swiglu, seed=172, x=x)
-        assert rel_err(y, ref) <= BF16_TOL
-
-
-@pytest.mark.parametrize("M", [3, 40, 200])
-def test_mxfp8_zero_and_non_finite_rows(M):
-    d, N = 256, 256
-    x = WL.activations(M, d, 173).clone()
-    x[0] = 0
-    x[1, 7] = float("inf")
-    x[2, 200] = float("nan")
-    y, ref = _case(M, d, N, False, seed=173, x=x)
-    assert torch.all(y[0].float() == 0)
-    assert torch.all(torch.isnan(y[1:3].float()))
+@pytest.mark.parametrize("M,d,N,swiglu", [
+    (65, 128, 128, False),     # one k group, one ragged row block
+    (129, 1024, 640, False),   # odd number of 128-column blocks, ragged rows
+    (250, 2048, 896, True),    # several k groups and tiles
+    (700, 768, 2304, True),    # 6 x 9 tiles: a last partial wave split in k over CTA pairs
+    (1030, 512, 1280, False),  # several row blocks, ragged
+])
+def test_mxfp8_promotion_kernel(M, d, N, swiglu):
+    """MXFP8 at M > 64 with bf16 output: x split per 32-deep block into e4m3
+    hi/lo planes with ue8m0 scales, block-scaled MMAs on the stored codes."""
+    y, ref = _case(M, d, N, swiglu, seed=178 + M)
     assert rel_err(y, ref) <= BF16_TOL
 
 
-@pytest.mark.parametrize("M,swiglu", [(1, True), (40, False), (64, True)])
-def test_mxfp8_decode_repeated_calls_bit_identical(M, swiglu):
-    d, N = 1024, 1024
-    inp = WL.case(M, d, N, swiglu, seed=174)
-    if swiglu:
-        Wq, s = T.fold(gpu(inp["W_gate"]), gpu(inp["g"]), gpu(inp["W_up"]), wtype=MX)
-    else:
-        Wq, s = T.fold(gpu(inp["W"]), gpu(inp["g"]), wtype=MX)
+@pytest.mark.parametrize("M,swiglu", [(200, False), (300, True)])
+def test_mxfp8_dequant_once_route(M, swiglu):
+    """The tile path's other route (the weight converted to bf16 once per call),
+    which NVFP4, partial and AdaLN outputs take, forced for a bf16 output."""
+    fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 4)
+    try:
+        y, ref = _case(M, 512, 384, swiglu, seed=179)
+    finally:
+        fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 0)
+    assert rel_err(y, ref) <= BF16_TOL
+
+
+def test_mxfp8_promotion_repeated_calls_and_timeout():
+    """320 tiles on the SMs: whole waves, then a tail split in k over CTA pairs
+    whose halves are added in a fixed order, so repeated calls give the same
+    bits.  A withheld scaler arrival (each CTA has several tiles, so its MMA
+    issuer waits for the accumulator) times out cleanly: the status word
+    reports it and the next call is correct."""
+    M, d, N = 2048, 256, 2560
+    inp = WL.case(M, d, N, True, seed=180)
+    Wq, s = T.fold(gpu(inp["W_gate"]), gpu(inp["g"]), gpu(inp["W_up"]), wtype=MX)
     x = gpu(inp["x"])
     ws = T.Workspace()
-    first = run(x, Wq, N, 1e-6, swiglu=swiglu, scales=s, ws=ws).clone()
-    for _ in range(200):
-        assert torch.equal(run(x, Wq, N, 1e-6, swiglu=swiglu, scales=s, ws=ws), first)
+    first = run(x, Wq, N, 1e-6, swiglu=True, scales=s, ws=ws).clone()
+    Wg, Wu = O.deinterleave128(mx_ref(inp["W_gate"], inp["g"], inp["W_up"])[2])
+    ref = O.norm_proj_swiglu(inp["x"], np.ones(d), Wg, Wu, 1e-6)
+    assert rel_err(first, ref) <= BF16_TOL
+    for _ in range(50):
+        assert torch.equal(run(x, Wq, N, 1e-6, swiglu=True, scales=s, ws=ws), first)
     assert ws.status()[0] == fnb.FN_OK
-
-
-@pytest.mark.parametrize("M", [8, 40])
-def test_mxfp8_nvfp4_output(M):
-    d, N = 512, 512
-    inp = WL.case(M, d, N, True, seed=175)
-    g = inp["g"]
-    Wq, s = T.fold(gpu(inp["W_gate"]), gpu(g), gpu(inp["W_up"]), wtype=MX)
-    Wg, Wu = O.deinterleave128(mx_ref(inp["W_gate"], g, inp["W_up"])[2])
-    ref = O.norm_proj_swiglu(inp["x"], np.ones(d), Wg, Wu, inp["eps"])
-    gs = torch.tensor([448.0 * 6.0 / 4.0], dtype=torch.float32, device="cuda")
-    q, sf = T.norm_proj_swiglu_nvfp4(gpu(inp["x"]), Wq, N, inp["eps"], gs, scales=s)
-    torch.cuda.synchronize()
-    check_nvfp4(q.cpu().numpy(), sf.cpu().numpy(), ref, float(gs.item()), BF16_TOL)
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 20_000_000) == fnb.FN_OK
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_WITHHOLD_ARRIVE, 1) == fnb.FN_OK
+    try:
+        T.norm_proj(x, Wq, N, 1e-6, swiglu=True, scales=s, ws=ws)
+        st, word = ws.status()
+    finally:
+        fnb.fn_set_debug(fnb.FN_DEBUG_WITHHOLD_ARRIVE, 0)
+        fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 2_000_000_000)
+    assert st == fnb.FN_ERR_TIMEOUT and (word >> 8) != 0
+    ws.buf.zero_()
+    assert torch.equal(run(x, Wq, N, 1e-6, swiglu=True, scales=s, ws=ws), first)
+    assert ws.status()[0] == fnb.FN_OK
 
 
 @pytest.mark.parametrize("M", [8, 100])
@@ -221,7 +223,7 @@ def test_mxfp8_timeout_is_reported():
 @pytest.fixture(scope="module")
 def mx_workload():
     w = WL.WORKLOADS["fp8_swiglu"]
-    inp = WL.workload_case("fp8_swiglu", 64)
+    inp = WL.workload_case("fp8_swiglu", 256)
     g = inp["g"]
     Wq, s = T.fold(gpu(inp["W_gate"]), gpu(g), gpu(inp["W_up"]), wtype=MX)
     Wg, Wu = O.deinterleave128(mx_ref(inp["W_gate"], g, inp["W_up"])[2])
@@ -229,7 +231,7 @@ def mx_workload():
     return w, inp, Wq, s, Wg, Wu
 
 
-@pytest.mark.parametrize("M", [1, 64])
+@pytest.mark.parametrize("M", [1, 64, 256])
 def test_mxfp8_fp8_workload(mx_workload, M):
     """The fp8 SwiGLU workload's shape (d = 5120, 2 x 13824 columns) with the
     weight folded to MXFP8 instead of 128x128 fp32 block scales."""

@@ -60,7 +60,7 @@ WORKLOADS: Dict[str, Workload] = {
         Workload("fp8_swiglu", (1, 64, 256, 8192), 5120, 13824, True, "fp8_e4m3_b128", False, 4),
         # the fp8 workload's shapes and inputs with the weight folded to the
         # block-scaled MXFP8 format instead of 128x128 fp32 block scales
-        Workload("mxfp8_swiglu", (1, 64), 5120, 13824, True, "mxfp8_e4m3", False, 4),
+        Workload("mxfp8_swiglu", (1, 64, 256, 8192), 5120, 13824, True, "mxfp8_e4m3", False, 4),
     )
 }
 WORKLOAD_ORDER = ("tiny", "decode_qkv", "ffn_swiglu", "prefill_swiglu_large", "fp8_swiglu", "mxfp8_swiglu")
