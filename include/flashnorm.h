@@ -387,14 +387,22 @@ uint64_t fn_kernel_launches(void);
  *   FN_DEBUG_PREFETCH         decode path: weight prefetch into L2 before waiting on
  *                             the previous kernel; value = mode | (k_blocks << 8),
  *                             mode 0 off, 1 TMA prefetch, 2 per-thread prefetch
- *                             (default: mode 2, 8 k-blocks)
+ *                             (default: mode 2, 8 k-blocks; the cluster decode kernel
+ *                             prefetches at most its ring depth)
  *   FN_DEBUG_CLUSTER          decode path: 1 (default) split K inside thread-block
  *                             clusters when the column tiles fill at most half the SMs,
  *                             with the largest cluster size whose clusters all fit at
  *                             once; 2..8 start from that size; 0 always stream-K + fix-up
+ *   FN_DEBUG_DECODE_GROUPS    decode path, bf16 weights, plain projection, bf16 output:
+ *                             0 (default) column groups per thread-block cluster (k split
+ *                             across the cluster, partials reduced in distributed shared
+ *                             memory, no fix-up kernel) where that balances the SMs about
+ *                             as well as stream-K; 1 never; 2 whenever such a plan fits;
+ *                             2 | (T << 4) | (S << 8): T boxes of 64 columns per cluster
+ *                             of S CTAs when that plan fits (T 1..3, S 2..8)
  */
 enum { FN_DEBUG_WAIT_BUDGET_NS = 1, FN_DEBUG_WITHHOLD_ARRIVE = 2, FN_DEBUG_FORCE_PATH = 3, FN_DEBUG_PREFETCH = 4,
-       FN_DEBUG_CLUSTER = 5 };
+       FN_DEBUG_CLUSTER = 5, FN_DEBUG_DECODE_GROUPS = 6 };
 fn_status fn_set_debug(int key, int64_t value);
 
 #ifdef __cplusplus

@@ -35,6 +35,7 @@ FN_DEBUG_WITHHOLD_ARRIVE = 2
 FN_DEBUG_FORCE_PATH = 3
 FN_DEBUG_PREFETCH = 4
 FN_DEBUG_CLUSTER = 5
+FN_DEBUG_DECODE_GROUPS = 6
 
 _vp, _i64, _f32, _sz, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_int
 

@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libflashnorm.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-SOURCES = ["api.cu", "fold.cu", "decode.cu", "decode_fp8.cu", "decode_mx.cu", "tc.cu", "tc2.cu", "tc8.cu", "noalloc.cu",
+SOURCES = ["api.cu", "fold.cu", "decode.cu", "decode_cl.cu", "decode_fp8.cu", "decode_mx.cu", "tc.cu", "tc2.cu", "tc8.cu", "noalloc.cu",
            "post_scale.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -27,6 +27,7 @@ std::atomic<int> g_force_path{0};
 std::atomic<int> g_prefetch_iters{8};
 std::atomic<int> g_prefetch_mode{2};
 std::atomic<int> g_cluster_mode{1};
+std::atomic<int> g_group_mode{0};
 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
@@ -246,6 +247,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.prefetch_iters = g_prefetch_iters.load();
   a.prefetch_mode = g_prefetch_mode.load();
   a.cluster_mode = g_cluster_mode.load();
+  a.group_mode = g_group_mode.load();
   a.single_sm_tiles = force == 3 ? 1 : 0;
   a.ad_scale = ad.scale;
   a.ad_bias = ad.bias;
@@ -532,6 +534,11 @@ fn_status fn_set_debug(int key, int64_t value) {
     case FN_DEBUG_CLUSTER:
       if (value < 0 || value > 8) return FN_ERR_INVALID_ARG;
       g_cluster_mode.store(static_cast<int>(value));
+      return FN_OK;
+    case FN_DEBUG_DECODE_GROUPS:
+      if (value < 0 || (value & 0xF) > 2 || ((value >> 4) & 0xF) > 3 || ((value >> 8) & 0xF) > 8 || (value >> 12))
+        return FN_ERR_INVALID_ARG;
+      g_group_mode.store(static_cast<int>(value));
       return FN_OK;
     case FN_DEBUG_PREFETCH:
       if (value < 0 || (value & 0xFF) > 2) return FN_ERR_INVALID_ARG;

@@ -32,7 +32,6 @@
 //
 // This file holds the bf16-weight kernel; fp8 weights have their own kernel
 // (decode_fp8.cu) that feeds the e4m3 tiles to the tensor cores unconverted.
-#include <atomic>
 #include <cstddef>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -442,37 +441,6 @@ inline int cluster_split(int tiles, int kblocks, int num_sms) {
   return S;
 }
 
-// Whether `tiles` clusters of S CTAs can all be resident at once (cached per
-// device and cluster size).
-template <auto Kernel>
-bool clusters_fit(int S, int tiles, int threads, size_t smem) {
-  static std::atomic<int> cache[64][9];   // 0 unknown, else max active clusters + 1
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64 || S > 8) return false;
-  int v = cache[dev][S].load(std::memory_order_relaxed);
-  if (v == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles * S));
-    cfg.blockDim = dim3(static_cast<unsigned>(threads));
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, Kernel, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      n = 0;
-    }
-    v = n + 1;
-    cache[dev][S].store(v, std::memory_order_relaxed);
-  }
-  return v - 1 >= tiles;
-}
-
 template <int MPAD, int HALVES, int OUT = kOutBf16>
 cudaError_t launch_impl(const CallArgs& a) {
   if (a.ws_bytes < workspace_bytes<MPAD, HALVES>(a.d, a.ncols, a.num_sms)) return cudaErrorInvalidValue;
@@ -560,6 +528,8 @@ cudaError_t launch_decode(const CallArgs& a) {
   const int mp = decode_mpad(a.M);
   if (a.wtype == 1) return launch_decode_fp8(a, mp);
   if (a.wtype == 2) return launch_decode_mx(a, mp);
+  int T = 0, S = 0;
+  if (decode_cl_plan(a, T, S)) return launch_decode_cl(a, T, S);
   if (a.part_out) {   // partial output: a plain projection of the stored columns
     if (mp == 16) return dec::launch_impl<16, 1, kOutPartial>(a);
     if (mp == 32) return dec::launch_impl<32, 1, kOutPartial>(a);

@@ -9,6 +9,7 @@
 // so repeated calls are bit-identical), applies the deferred 1/rms (FlashNorm
 // talk summary, Proposal 2) and, for the gated projection, SwiGLU.
 #pragma once
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -267,6 +268,37 @@ cudaError_t launch_fixup(const Params& p, cudaStream_t stream) {
   const long long threads = static_cast<long long>(p.tiles) * 128 * ((p.M + 3) / 4);
   const unsigned fgrid = static_cast<unsigned>((threads + FIX_THREADS - 1) / FIX_THREADS);
   return launch_pdl(decode_fixup_kernel<MPAD, HALVES, OUT>, fgrid, FIX_THREADS, 0, stream, p);
+}
+
+// Whether `tiles` clusters of S CTAs can all be resident at once (cached per
+// device and cluster size).
+template <auto Kernel>
+bool clusters_fit(int S, int tiles, int threads, size_t smem) {
+  static std::atomic<int> cache[64][9];   // 0 unknown, else max active clusters + 1
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64 || S > 8) return false;
+  int v = cache[dev][S].load(std::memory_order_relaxed);
+  if (v == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles * S));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, Kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    v = n + 1;
+    cache[dev][S].store(v, std::memory_order_relaxed);
+  }
+  return v - 1 >= tiles;
 }
 
 // Workspace needed by a decode call: the header and two partial slots per CTA

@@ -48,6 +48,7 @@ struct CallArgs {
   int prefetch_iters;     // decode: weight k-blocks per CTA prefetched into L2 early
   int prefetch_mode;      // decode: 0 none, 1 TMA prefetch, 2 per-thread prefetch
   int cluster_mode;       // decode: 1 allow split-K inside clusters, 0 stream-K only
+  int group_mode;         // decode: column groups per cluster (decode_cl.cu): 0 auto, 1 never, 2 whenever they fit
   int single_sm_tiles;    // tile path: 1 keeps the one-SM kernel where the pair kernel would run
   const float* ad_scale;  // AdaLN (tile path only): scale rows fp32 [n_cond, d], or null
   const float* ad_bias;   //   shift bias rows fp32 [n_cond, ncols]
@@ -87,6 +88,14 @@ cudaError_t launch_tc(const CallArgs& a);
 cudaError_t launch_tc_pair(const CallArgs& a);
 // Rows from which the tile path runs on pairs of SMs.
 constexpr int64_t kPairTileMinM = 512;
+// Small-M path for bf16 weights, plain projection, bf16 output, when the
+// weight is too small to keep every SM busy without splitting most column
+// tiles: T 64-column boxes per cluster of S CTAs, k split across the cluster,
+// partials reduced through distributed shared memory (decode_cl.cu).  Returns
+// false (and launches nothing) when no cluster plan is chosen for the shape.
+bool decode_cl_plan(const CallArgs& a, int& T, int& S);
+cudaError_t launch_decode_cl(const CallArgs& a, int T, int S);
+
 // fp8 weights (128x128 block scales) at M > 64 with bf16 output: x split once
 // into exact e4m3 hi/lo planes, the stored codes multiplied as they are, the
 // block scales applied per 128-deep k block to fp32 sums (tc8.cu).  MXFP8
