@@ -478,7 +478,13 @@ def kernel_for(wl: WL.Workload, M: int, out: str, per_m: bool = True):
     """Name of the dominant kernel of a call, its sources and its ncu summary file."""
     # the library's promotion-kernel thresholds: fp8 from 48 rows, MXFP8 above 64
     promotion = out == "bf16" and ((wl.wtype == "fp8_e4m3_b128" and M >= 48) or (wl.wtype == "mxfp8_e4m3" and M > 64))
-    if M <= 64 and not promotion:
+    # bf16 plain projections with bf16 output at these workloads' sizes (the decode QKV
+    # shape) take the cluster decode kernel, which needs no fix-up kernel
+    grouped = wl.wtype == "bf16" and not wl.swiglu and out == "bf16"
+    if M <= 64 and grouped:
+        kname, sources = "decode_cl_kernel", ["decode_cl.cu", "decode_common.cuh", "ptx.cuh"]
+        label = "decode_cl_kernel (k split inside clusters, partials reduced in distributed shared memory)"
+    elif M <= 64 and not promotion:
         kname, src = {"bf16": ("decode_kernel", "decode.cu"), "fp8_e4m3_b128": ("decode_fp8_kernel", "decode_fp8.cu"),
                       "mxfp8_e4m3": ("decode_mx_kernel", "decode_mx.cu")}[wl.wtype]
         sources = [src, "decode_common.cuh", "ptx.cuh", "nvfp4.cuh"]
