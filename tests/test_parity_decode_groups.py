@@ -120,13 +120,14 @@ def test_zero_and_non_finite_rows(M):
     assert rel_err(y, ref) <= BF16_TOL
 
 
-def test_repeated_calls_bit_identical_and_timeout():
+@pytest.mark.parametrize("M", [8, 64])
+def test_repeated_calls_bit_identical_and_timeout(M):
     """Repeats of the decode QKV shape give the same bits; a withheld reducer
     arrival makes the epilogue's bounded wait give up with FN_ERR_TIMEOUT, the
     cluster still meets at its barriers and exits, and the next call (zeroed
     workspace) is correct."""
     w = WL.WORKLOADS["decode_qkv"]
-    inp = WL.workload_case("decode_qkv", 8)
+    inp = WL.workload_case("decode_qkv", M)
     Wp = _fold(inp)
     x = gpu(inp["x"])
     ws = T.Workspace()
