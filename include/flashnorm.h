@@ -400,9 +400,12 @@ uint64_t fn_kernel_launches(void);
  *                             as well as stream-K; 1 never; 2 whenever such a plan fits;
  *                             2 | (T << 4) | (S << 8): T boxes of 64 columns per cluster
  *                             of S CTAs when that plan fits (T 1..3, S 2..8)
+ *   FN_DEBUG_PAIR_TILE        tile path on pairs of SMs (bf16 weights, M >= 512): 0 automatic,
+ *                             1 256 x 256 output tiles (two accumulators, overlapped epilogue),
+ *                             2 256 x 512 output tiles (two pair MMAs per K step)
  */
 enum { FN_DEBUG_WAIT_BUDGET_NS = 1, FN_DEBUG_WITHHOLD_ARRIVE = 2, FN_DEBUG_FORCE_PATH = 3, FN_DEBUG_PREFETCH = 4,
-       FN_DEBUG_CLUSTER = 5, FN_DEBUG_DECODE_GROUPS = 6 };
+       FN_DEBUG_CLUSTER = 5, FN_DEBUG_DECODE_GROUPS = 6, FN_DEBUG_PAIR_TILE = 7 };
 fn_status fn_set_debug(int key, int64_t value);
 
 #ifdef __cplusplus

@@ -36,6 +36,7 @@ FN_DEBUG_FORCE_PATH = 3
 FN_DEBUG_PREFETCH = 4
 FN_DEBUG_CLUSTER = 5
 FN_DEBUG_DECODE_GROUPS = 6
+FN_DEBUG_PAIR_TILE = 7
 
 _vp, _i64, _f32, _sz, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_int
 

@@ -27,6 +27,7 @@ std::atomic<int> g_force_path{0};
 std::atomic<int> g_prefetch_iters{8};
 std::atomic<int> g_prefetch_mode{2};
 std::atomic<int> g_cluster_mode{1};
+std::atomic<int> g_pair_tile{0};
 std::atomic<int> g_group_mode{0};
 
 constexpr int kMaxDevices = 64;
@@ -247,6 +248,7 @@ fn_status norm_proj_common(const void* x, int64_t M, int64_t d, const void* Wp, 
   a.prefetch_iters = g_prefetch_iters.load();
   a.prefetch_mode = g_prefetch_mode.load();
   a.cluster_mode = g_cluster_mode.load();
+  a.pair_tile = g_pair_tile.load();
   a.group_mode = g_group_mode.load();
   a.single_sm_tiles = force == 3 ? 1 : 0;
   a.ad_scale = ad.scale;
@@ -539,6 +541,10 @@ fn_status fn_set_debug(int key, int64_t value) {
       if (value < 0 || (value & 0xF) > 2 || ((value >> 4) & 0xF) > 3 || ((value >> 8) & 0xF) > 8 || (value >> 12))
         return FN_ERR_INVALID_ARG;
       g_group_mode.store(static_cast<int>(value));
+      return FN_OK;
+    case FN_DEBUG_PAIR_TILE:
+      if (value < 0 || value > 2) return FN_ERR_INVALID_ARG;
+      g_pair_tile.store(static_cast<int>(value));
       return FN_OK;
     case FN_DEBUG_PREFETCH:
       if (value < 0 || (value & 0xFF) > 2) return FN_ERR_INVALID_ARG;

@@ -50,6 +50,7 @@ struct CallArgs {
   int cluster_mode;       // decode: 1 allow split-K inside clusters, 0 stream-K only
   int group_mode;         // decode: column groups per cluster (decode_cl.cu): 0 auto, 1 never, 2 whenever they fit
   int single_sm_tiles;    // tile path: 1 keeps the one-SM kernel where the pair kernel would run
+  int pair_tile;          // pair kernel tile: 0 automatic, 1 256 x 256, 2 256 x 512
   const float* ad_scale;  // AdaLN (tile path only): scale rows fp32 [n_cond, d], or null
   const float* ad_bias;   //   shift bias rows fp32 [n_cond, ncols]
   const int* ad_index;    //   condition index per row [M]; null: no AdaLN

@@ -9,7 +9,10 @@
 // pair, 128 rows per CTA.  Each CTA stages only its own 128 x 64 x tile and its
 // own 64 x 128 half of the weight tile, so an SM moves 32 KB from L2 per
 // 64-deep k step instead of 48 KB for the same flops; for SwiGLU the gate
-// columns of a tile sit in CTA 0 and the up columns in CTA 1.
+// columns of a tile sit in CTA 0 and the up columns in CTA 1.  The wide form
+// computes a 256 x 512 tile with two pair MMAs per K step (each CTA stages two
+// 128-column halves, 48 KB per k step for twice the flops) into one
+// 512-column accumulator.
 //
 // Joins (all bounded waits; a CTA that gives up raises its partner's abort
 // flag too):
@@ -33,7 +36,9 @@
 //
 // Layout per CTA: 10 warps, as tc.cu.
 //   warp 0      TMA producer (own x rows, own weight columns), 7 stages of 32 KB
-//   warp 1      TMEM owner; in CTA 0 the pair-MMA issuer (M=256 N=256 K=16)
+//               (wide: 4 stages of 48 KB)
+//   warp 1      TMEM owner; in CTA 0 the pair-MMA issuer (M=256 N=256 K=16; wide:
+//               two per K step)
 //   warps 2-5   sum-of-squares reducers, one thread per row of this CTA
 //   warps 6-9   epilogue: TMEM -> registers, post-scale (+SwiGLU), bf16 store
 #include <cuda_bf16.h>
@@ -46,16 +51,29 @@ namespace fn {
 namespace tc2 {
 
 constexpr int BM = 128;                  // rows per CTA (256 per pair)
-constexpr int BN = 256;                  // output tile columns
-constexpr int BNH = 128;                 // weight columns staged per CTA
 constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
 constexpr int B_BOX_BYTES = 64 * BK * 2; // 8 KB: 64 columns x 64 k rows
-constexpr int B_BYTES = BNH * BK * 2;    // 16 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int STAGES = 7;
+constexpr int HALF_B = 2 * B_BOX_BYTES;  // 16 KB: 128 weight columns per CTA and MMA
 constexpr int NUM_THREADS = 320;
-constexpr int TMEM_COLS = 2 * BN;
+constexpr int TMEM_COLS = 512;
+constexpr int MMA_N = 256;               // columns of one pair MMA (128 from each CTA)
+
+// Tile shapes.  Narrow: a 256 x 256 output tile per pair, one pair MMA per K
+// step, two TMEM accumulators (the epilogue of one tile overlaps the next).
+// Wide: 256 x 512, two pair MMAs per K step into one 512-column accumulator,
+// so each staged byte feeds a third more flops (the kernel is bound by the
+// operand delivery rate into the SMs) at the cost of an epilogue that the
+// next tile's MMAs wait for.
+template <bool WIDE>
+struct Shape {
+  static constexpr int H = WIDE ? 2 : 1;             // pair MMAs per K step
+  static constexpr int BN = H * MMA_N;               // output tile columns (stored weight columns)
+  static constexpr int B_BYTES = H * HALF_B;         // weight bytes staged per CTA and stage
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = WIDE ? 4 : 7;
+  static constexpr int NBUF = WIDE ? 1 : 2;          // TMEM accumulators
+};
 
 enum : unsigned { kSiteProdEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteRedFull, kSiteRedSsqEmpty,
                   kSiteEpiAccFull, kSiteEpiSsqFull, kSiteDrain, kSiteExit };
@@ -71,6 +89,7 @@ struct Params {
   int withhold;
 };
 
+template <int STAGES>
 struct alignas(8) Bars {
   uint64_t full[STAGES], empty[STAGES];
   uint64_t mdone[STAGES];                // the pair MMA of the stage completed (both CTAs)
@@ -84,8 +103,12 @@ struct alignas(8) Bars {
   int epi_ok[2];                         // the epilogue group's common wait outcome, per buffer
 };
 
-constexpr size_t smem_bytes() { return 1024 + STAGES * STAGE_BYTES + sizeof(Bars); }
-static_assert(smem_bytes() <= 232448, "shared memory budget");
+template <bool WIDE>
+constexpr size_t smem_bytes() {
+  using Sh = Shape<WIDE>;
+  return 1024 + Sh::STAGES * Sh::STAGE_BYTES + sizeof(Bars<Sh::STAGES>);
+}
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
   const int per_group = p.group_m * p.num_n;
@@ -120,13 +143,15 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
   }
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool WIDE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const Params p) {
+  using Sh = Shape<WIDE>;
+  constexpr int STAGES = Sh::STAGES, STAGE_BYTES = Sh::STAGE_BYTES, BN = Sh::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars& bars = *reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
+  Bars<STAGES>& bars = *reinterpret_cast<Bars<STAGES>*>(smem + STAGES * STAGE_BYTES);
   auto stage_a = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stage_b = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
 
@@ -182,14 +207,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         int mb, nb;
         tile_coords(t, p, mb, nb);
         const int row0 = mb * (2 * BM) + static_cast<int>(rank) * BM;
-        const int col0 = nb * BN + static_cast<int>(rank) * BNH;
+        // per pair MMA h, this CTA's 128 columns: [nb BN + h 256 + rank 128, +128)
+        // (for SwiGLU the gate block in CTA 0, the matching up block in CTA 1)
+        const int col0 = nb * BN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait_spin(&bars.empty[s], ph ^ 1, ctl, kSiteProdEmpty)) { ok = false; break; }
-          if (rank == 0) mbar_arrive_expect_tx(&bars.full[s], 2 * (A_BYTES + B_BYTES));
+          if (rank == 0) mbar_arrive_expect_tx(&bars.full[s], 2 * STAGE_BYTES);
           const uint32_t fb = full0 + s * 8;
           tma_load_2d_pair(stage_a(s), &tmap_x, fb, kb * BK, row0);
-          tma_load_2d_pair(stage_b(s), &tmap_w, fb, col0, kb * BK);
-          tma_load_2d_pair(stage_b(s) + B_BOX_BYTES, &tmap_w, fb, col0 + 64, kb * BK);
+#pragma unroll
+          for (int h = 0; h < Sh::H; ++h) {
+            tma_load_2d_pair(stage_b(s) + h * HALF_B, &tmap_w, fb, col0 + h * MMA_N, kb * BK);
+            tma_load_2d_pair(stage_b(s) + h * HALF_B + B_BOX_BYTES, &tmap_w, fb, col0 + h * MMA_N + 64, kb * BK);
+          }
           issued |= 1u << s;
           last_ph = (last_ph & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -207,14 +237,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       if (rank == 0) {
         // -------------------------------------------------------- pair-MMA issuer
-        constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, /*a MN-major*/ false, /*b MN-major*/ true);
+        constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, MMA_N, /*a MN-major*/ false, /*b MN-major*/ true);
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;
         int i = 0;
         for (int t = pair; t < p.num_tiles && ok; t += npairs, ++i) {
-          const int b = i & 1;
-          const uint32_t aph = (i >> 1) & 1;
+          const int b = Sh::NBUF == 2 ? (i & 1) : 0;
+          const uint32_t aph = Sh::NBUF == 2 ? (i >> 1) & 1 : i & 1;
           // CTA 1's epilogue arrives here after its TMEM loads completed (tcgen05.wait::ld),
           // so the buffer may be overwritten once the phase completes
           if (!mbar_wait_spin(&bars.acc_empty[b], aph ^ 1, ctl, kSiteMmaAccEmpty)) break;
@@ -229,9 +259,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             for (int kk = 0; kk < BK / 16; ++kk) {
               // A: this CTA's x rows, K-major (the partner's rows at the same offset)
               const uint64_t adesc = sdesc_sw128(a0 + kk * 32, 16, 1024);
-              // B: this CTA's 128 weight columns, N-major, two 64-column boxes 8 KB apart
-              const uint64_t bdesc = sdesc_sw128(b0 + kk * 2048, B_BOX_BYTES, 1024);
-              umma_bf16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0);
+#pragma unroll
+              for (int h = 0; h < Sh::H; ++h) {
+                // B: this CTA's 128 weight columns of MMA h, N-major, two 64-column boxes 8 KB apart
+                const uint64_t bdesc = sdesc_sw128(b0 + h * HALF_B + kk * 2048, B_BOX_BYTES, 1024);
+                umma_bf16_pair(d_tmem + h * MMA_N, adesc, bdesc, IDESC, (kb | kk) != 0);
+              }
             }
             umma_commit_pair(&bars.empty[s], 0x3);
             umma_commit_pair(&bars.mdone[s], 0x3);
@@ -282,30 +315,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     for (int t = pair; t < p.num_tiles; t += npairs, ++i) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
-      const int b = i & 1;
-      const uint32_t aph = (i >> 1) & 1;
+      const int b = Sh::NBUF == 2 ? (i & 1) : 0;
+      const uint32_t aph = Sh::NBUF == 2 ? (i >> 1) & 1 : i & 1;
+      const int sb = i & 1;                 // sums-of-squares buffer
+      const uint32_t sph = (i >> 1) & 1;
       // One thread waits and the whole epilogue group follows its decision, so
       // the group never splits at the named barrier or the .sync.aligned loads.
       if (et == 0) {
         bool ok = mbar_wait_spin(&bars.acc_full[b], aph, ctl, kSiteEpiAccFull);
-        ok = ok && mbar_wait(&bars.ssq_full[b], aph, ctl, kSiteEpiSsqFull);
-        bars.epi_ok[b] = ok ? 1 : 0;
+        ok = ok && mbar_wait(&bars.ssq_full[sb], sph, ctl, kSiteEpiSsqFull);
+        bars.epi_ok[sb] = ok ? 1 : 0;
       }
       named_bar_sync(1, 128);
-      if (!bars.epi_ok[b]) break;
+      if (!bars.epi_ok[sb]) break;
       tc_fence_after();
-      const float r = inv_rms(bars.ssq[b][row], p.inv_d, p.eps);
-      mbar_arrive(&bars.ssq_empty[b]);
+      const float r = inv_rms(bars.ssq[sb][row], p.inv_d, p.eps);
+      mbar_arrive(&bars.ssq_empty[sb]);
       const int grow = mb * (2 * BM) + static_cast<int>(rank) * BM + row;
       const bool row_ok = grow < p.M;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
       if constexpr (SWIGLU) {
-        __nv_bfloat16* yrow = p.y + static_cast<int64_t>(grow) * p.nout + nb * (BN / 2);
+        // accumulator columns of MMA h: [h 256, +128) gate, [h 256 + 128, +128) up,
+        // output columns [nb BN/2 + h 128, +128)
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
+          const int h = c / 128, cc = c % 128;
+          const int ocol = nb * (BN / 2) + c;
           uint32_t gv[32], uv[32];
-          tmem_ld32(taddr + c, gv);
-          tmem_ld32(taddr + BN / 2 + c, uv);
+          tmem_ld32(taddr + h * MMA_N + cc, gv);
+          tmem_ld32(taddr + h * MMA_N + 128 + cc, uv);
           tmem_ld_wait();
           uint32_t o[16];
 #pragma unroll
@@ -314,8 +352,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const float u0 = __uint_as_float(uv[2 * j]) * r, u1 = __uint_as_float(uv[2 * j + 1]) * r;
             o[j] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
           }
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(yrow + c);
+          if (row_ok && ocol < p.nout) {
+            uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(grow) * p.nout + ocol);
 #pragma unroll
             for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
           }
@@ -365,8 +403,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool WIDE>
 cudaError_t launch_impl(const CallArgs& a) {
+  constexpr int BN = Shape<WIDE>::BN;
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.d, BM, BK)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tw, a.Wp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d, a.ncols, BK, 64))
@@ -393,17 +432,25 @@ cudaError_t launch_impl(const CallArgs& a) {
   p.status = static_cast<unsigned int*>(a.ws);
   p.budget_ns = a.budget_ns;
   p.withhold = a.withhold;
-  constexpr size_t SMEM = smem_bytes();
-  cudaError_t e = ensure_smem_limit<tc2_kernel<SWIGLU>>(static_cast<int>(SMEM));
+  constexpr size_t SMEM = smem_bytes<WIDE>();
+  cudaError_t e = ensure_smem_limit<tc2_kernel<SWIGLU, WIDE>>(static_cast<int>(SMEM));
   if (e != cudaSuccess) return e;
   const int pairs = p.num_tiles < a.num_sms / 2 ? p.num_tiles : a.num_sms / 2;
-  return launch_pdl(tc2_kernel<SWIGLU>, static_cast<unsigned>(2 * pairs), NUM_THREADS, SMEM, a.stream, tx, tw, p);
+  return launch_pdl(tc2_kernel<SWIGLU, WIDE>, static_cast<unsigned>(2 * pairs), NUM_THREADS, SMEM, a.stream, tx, tw,
+                    p);
 }
 
 }  // namespace tc2
 
+// 256 x 512 tiles where the k range is long enough to hide their
+// non-overlapped epilogue: at d = 8192 (large prefill) they ran 16 % faster
+// than 256 x 256 tiles; at d = 4096 (FFN, 4096 rows) the two tied.
+constexpr int64_t kWidePairTileMinD = 6144;
+
 cudaError_t launch_tc_pair(const CallArgs& a) {
-  return a.swiglu ? tc2::launch_impl<true>(a) : tc2::launch_impl<false>(a);
+  const bool wide = a.pair_tile == 2 || (a.pair_tile == 0 && a.d >= kWidePairTileMinD);
+  if (a.swiglu) return wide ? tc2::launch_impl<true, true>(a) : tc2::launch_impl<true, false>(a);
+  return wide ? tc2::launch_impl<false, true>(a) : tc2::launch_impl<false, false>(a);
 }
 
 }  // namespace fn

@@ -1,6 +1,6 @@
-"""GPU parity of the tile kernel on pairs of SMs (2-CTA clusters, 256 x 256
-tiles, tcgen05.mma.cta_group::2), which the library runs for bf16 weights at
-M >= 512.
+"""GPU parity of the tile kernel on pairs of SMs (2-CTA clusters, 256 x 256 or
+256 x 512 tiles, tcgen05.mma.cta_group::2), which the library runs for bf16
+weights at M >= 512.
 
 Against the fp64 oracle on the stored folded weight within 1e-2 (1 + |y_ref|),
 against the single-SM tile kernel (FN_DEBUG_FORCE_PATH = 3) within the same
@@ -31,6 +31,16 @@ def _lib():
     fnb.fn_set_debug(fnb.FN_DEBUG_FORCE_PATH, 0)
 
 
+@pytest.fixture(autouse=True, params=[1, 2], ids=["tile256x256", "tile256x512"])
+def pair_tile(request):
+    """Every test runs with both pair tiles: 256 x 256 (one pair MMA per K step,
+    two accumulators) and 256 x 512 (two pair MMAs per K step into one
+    512-column accumulator)."""
+    assert fnb.fn_set_debug(fnb.FN_DEBUG_PAIR_TILE, request.param) == fnb.FN_OK
+    yield request.param
+    fnb.fn_set_debug(fnb.FN_DEBUG_PAIR_TILE, 0)
+
+
 def _case(M, d, N, swiglu, seed):
     inp = WL.case(M, d, N, swiglu, seed=seed)
     g = inp["g"]
@@ -47,6 +57,7 @@ def _case(M, d, N, swiglu, seed):
 @pytest.mark.parametrize("M,d,N,swiglu", [
     (512, 256, 512, False),
     (600, 512, 384, False),    # ragged rows; 3 column blocks: the last tile's second half is past N
+    (520, 640, 640, True),     # 5 output blocks of 128: the wide tile's last second MMA is past N
     (700, 384, 256, True),     # the last pair: CTA 0 partly, CTA 1 wholly past M
     (1024, 1024, 1280, True),
     (777, 4096, 256, False),   # long k range
