@@ -336,15 +336,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
       if constexpr (SWIGLU) {
         // accumulator columns of MMA h: [h 256, +128) gate, [h 256 + 128, +128) up,
-        // output columns [nb BN/2 + h 128, +128)
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
+        // output columns [nb BN/2 + h 128, +128).  Chunks of 32 columns; the next
+        // chunk's TMEM loads are issued before this chunk's math, so their latency
+        // hides under it (two register buffers).
+        auto load_chunk = [&](int c, uint32_t(&gv)[32], uint32_t(&uv)[32]) {
           const int h = c / 128, cc = c % 128;
-          const int ocol = nb * (BN / 2) + c;
-          uint32_t gv[32], uv[32];
           tmem_ld32(taddr + h * MMA_N + cc, gv);
           tmem_ld32(taddr + h * MMA_N + 128 + cc, uv);
-          tmem_ld_wait();
+        };
+        auto finish_chunk = [&](int c, const uint32_t(&gv)[32], const uint32_t(&uv)[32]) {
+          const int ocol = nb * (BN / 2) + c;
           uint32_t o[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -357,6 +358,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
           }
+        };
+        uint32_t ga[32], ua[32], gb[32], ub[32];
+        load_chunk(0, ga, ua);
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 64) {
+          tmem_ld_wait();                       // chunk c (buffer a) has landed
+          load_chunk(c + 32, gb, ub);           // BN / 2 is a multiple of 64
+          finish_chunk(c, ga, ua);
+          tmem_ld_wait();                       // chunk c + 32 (buffer b)
+          if (c + 64 < BN / 2) load_chunk(c + 64, ga, ua);
+          finish_chunk(c + 32, gb, ub);
         }
       } else {
         __nv_bfloat16* yrow = p.y + static_cast<int64_t>(grow) * p.nout;
@@ -443,9 +455,10 @@ cudaError_t launch_impl(const CallArgs& a) {
 }  // namespace tc2
 
 // 256 x 512 tiles where the k range is long enough to hide their
-// non-overlapped epilogue: at d = 8192 (large prefill) they ran 16 % faster
-// than 256 x 256 tiles; at d = 4096 (FFN, 4096 rows) the two tied.
-constexpr int64_t kWidePairTileMinD = 6144;
+// non-overlapped epilogue: at d = 8192 (large prefill) they ran 17 % faster
+// than 256 x 256 tiles; at d = 4096 (FFN, 4096 rows), with the epilogue's TMEM
+// loads pipelined, about 1.5 % faster.
+constexpr int64_t kWidePairTileMinD = 4096;
 
 cudaError_t launch_tc_pair(const CallArgs& a) {
   const bool wide = a.pair_tile == 2 || (a.pair_tile == 0 && a.d >= kWidePairTileMinD);
