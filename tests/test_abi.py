@@ -180,6 +180,22 @@ def test_set_debug_validates_keys(L):
     assert fnb.fn_set_debug(fnb.FN_DEBUG_WAIT_BUDGET_NS, 2_000_000_000) == fnb.FN_OK
 
 
+def test_set_debug_decode_groups_and_pair_tile(L):
+    """The cluster decode plan knob: mode 0..2, a forced plan's T (0..3) in bits
+    4..7 and S (0..8) in bits 8..11, nothing above; the pair-tile knob 0..2."""
+    G, P = fnb.FN_DEBUG_DECODE_GROUPS, fnb.FN_DEBUG_PAIR_TILE
+    for v in (0, 1, 2, 2 | (3 << 4) | (4 << 8), 2 | (1 << 4) | (8 << 8)):
+        assert fnb.fn_set_debug(G, v) == fnb.FN_OK
+    for v in (-1, 3, 2 | (4 << 4), 2 | (3 << 4) | (9 << 8), 1 << 12):
+        assert fnb.fn_set_debug(G, v) == fnb.FN_ERR_INVALID_ARG
+    assert fnb.fn_set_debug(G, 0) == fnb.FN_OK
+    for v in (0, 1, 2):
+        assert fnb.fn_set_debug(P, v) == fnb.FN_OK
+    for v in (-1, 3):
+        assert fnb.fn_set_debug(P, v) == fnb.FN_ERR_INVALID_ARG
+    assert fnb.fn_set_debug(P, 0) == fnb.FN_OK
+
+
 def test_no_device_means_no_launch(L):
     """Valid arguments without a GPU fail cleanly (no device), never crash."""
     import torch
