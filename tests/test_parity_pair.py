@@ -8,7 +8,8 @@ bound, bit-identical over repeated calls, and the bounded waits of both CTAs
 of a pair: a withheld arrival times out in both and the next call is correct.
 Shapes cover ragged rows (the second CTA of the last pair partly or wholly
 past M), an odd number of 128-column blocks (the second CTA's weight half past
-the last column) and a long k range.
+the last column), a long k range, and more tiles than pairs (a partial second
+wave).
 """
 import numpy as np
 import pytest
@@ -61,6 +62,10 @@ def _case(M, d, N, swiglu, seed):
     (700, 384, 256, True),     # the last pair: CTA 0 partly, CTA 1 wholly past M
     (1024, 1024, 1280, True),
     (777, 4096, 256, False),   # long k range
+    # 80 and 90 tiles of 256 x 512 on 74 pairs: a second, partial wave of
+    # tiles (plain; SwiGLU with ragged rows)
+    (512, 256, 20480, False),
+    (600, 256, 7680, True),
 ])
 def test_pair_kernel_against_oracle_and_single_sm(M, d, N, swiglu):
     inp, Wp, ref = _case(M, d, N, swiglu, seed=240 + M)
