@@ -26,12 +26,14 @@
 // order (= k order, so repeated calls give the same bits), applies 1/rms and
 // stores bf16.
 //
-// Layout: 8 warps, as the stream-K decode kernel.
+// Layout: 8 warps, as the stream-K decode kernel, during the k range:
 //   warp 0      TMA producer
 //   warp 1      TMEM owner and MMA issuer
 //   warps 2-3   sum-of-squares reducers (one thread per activation row)
-//   warps 4-7   epilogue: TMEM -> registers -> peers' shared memory, then the
-//               finish of this CTA's column share
+//   warps 4-7   (idle until the exchange)
+// and then all 8 for the exchange (warp w reads TMEM lane quarter w mod 4, half
+// of the rows each, and pushes 16-byte pieces) and the finish of this CTA's
+// column share (one thread per column and group of four rows).
 #include <cstddef>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
