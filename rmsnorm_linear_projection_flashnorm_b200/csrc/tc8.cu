@@ -1,5 +1,6 @@
 // Fused RMSNorm + projection, tile path (M > 64) for fp8 e4m3 weights with an
-// fp32 scale per 128 x 128 block, sm_100a.
+// fp32 scale per 128 x 128 block, and for MXFP8 weights (e4m3 with a ue8m0
+// scale per 32 k values and column), sm_100a.
 //
 // The arithmetic is FlashNorm's (FlashNorm talk summary, Proposal 2: matmul on
 // raw x, the sum of squares alongside, 1/rms applied after; the folded weight
@@ -22,6 +23,12 @@
 // Marlin explainer's section 4 (dequantisation hidden under the MMA stream),
 // applied to the sums instead of the weights: no weight tile is converted and
 // no bf16 copy of the weight is written.
+//
+// MXFP8 weights (the MX instance): the split runs per 32-deep block and its
+// powers of two become the activations' ue8m0 scale bytes, so block-scaled
+// MMAs (kind::mxf8f6f4.block_scale) apply both operands' scales in hardware
+// and one TMEM accumulator holds a work item's whole k range; the scalers only
+// read it once per item.
 //
 // Compared with converting the staged weight tiles to bf16 on chip, the weight
 // bytes per flop in shared memory are the same (B is read once per half of the
