@@ -121,9 +121,11 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
  * M >= 1024 at least one bf16 copy of the weight (2 d ncols
  * bytes), which the NVFP4 and partial-output calls convert once per call with
  * the rounding of the on-chip conversion (bf16(fp32(q) * s)); with MXFP8
- * weights the same bf16 copy at every M > 64, and at M <= 64 the activations
- * split once per call (2 x 64 x d bytes at most, their scale chunks and
- * per-group sums of squares).  Zero it once
+ * weights at M > 64 the larger of the same bf16 copy (NVFP4, partial and
+ * AdaLN outputs) and the promotion kernel's split activations (2 M d bytes,
+ * their scale chunks over whole 128-row blocks and per-block sums of squares),
+ * and at M <= 64 the activations split once per call (2 x 64 x d bytes at
+ * most, their scale chunks and per-group sums of squares).  Zero it once
  * before its first use (the status word must start at zero); the calls keep
  * the status word at zero unless a device-side wait times out.  Depends on
  * the SM count of the current device (148 is assumed when no device is
@@ -151,8 +153,15 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
  *   block scale and added to fp32 sums in k order.  MXFP8 weights: at M <= 64 the e4m3
  *   codes and their scales go to block-scaled MMAs as stored (the bf16
  *   activations split exactly into two e4m3 parts sharing one power-of-two
- *   scale per 32 k values); at M > 64 the weight is converted to bf16 once per
- *   call into the workspace (an exact conversion) for the tile kernel.
+ *   scale per 32 k values); at M > 64 the promotion tile kernel does the same
+ *   per 128 x 256 tile (the split per 32-deep block, its powers of two as the
+ *   activations' scale bytes, block-scaled MMAs over the whole k range).  The
+ *   NVFP4 and partial outputs and AdaLN at M > 64 convert the weight to bf16
+ *   once per call into the workspace (an exact conversion) for the tile kernel.
+ *   bf16 weights at M <= 64 with a plain projection and bf16 output may run
+ *   a decode kernel that splits k inside thread-block clusters over groups of
+ *   columns and adds the partials over distributed shared memory (no fix-up
+ *   kernel); its results are deterministic too.
  */
 fn_status fn_norm_proj(const void* x, int64_t M, int64_t d, const void* Wp, const float* scales, fn_wtype wt,
                        int64_t N, float eps, void* y, void* workspace, size_t ws_bytes, fn_stream_t stream);
