@@ -476,8 +476,8 @@ def roofline_entry(units_per_call: float, us_per_call: float, hbm_bound: bool, p
 
 def kernel_for(wl: WL.Workload, M: int, out: str, per_m: bool = True):
     """Name of the dominant kernel of a call, its sources and its ncu summary file."""
-    # the library's promotion-kernel thresholds: fp8 from 48 rows, MXFP8 above 64
-    promotion = out == "bf16" and ((wl.wtype == "fp8_e4m3_b128" and M >= 48) or (wl.wtype == "mxfp8_e4m3" and M > 64))
+    # the library's promotion-kernel thresholds: fp8 from 33 rows, MXFP8 above 64
+    promotion = out == "bf16" and ((wl.wtype == "fp8_e4m3_b128" and M >= 33) or (wl.wtype == "mxfp8_e4m3" and M > 64))
     # bf16 plain projections with bf16 output at these workloads' sizes (the decode QKV
     # shape) take the cluster decode kernel, which needs no fix-up kernel
     grouped = wl.wtype == "bf16" and not wl.swiglu and out == "bf16"

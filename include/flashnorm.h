@@ -115,7 +115,7 @@ fn_status fn_fold_weights(const void* W0, const void* W1, const float* g, int64_
  * M <= 64, the per-CTA partial sums of the split-K decode path; with fp8
  * weights and 17 <= M <= 64 also the activations split once per call into
  * the two e4m3 operand parts (2 x 64 x d bytes at most) with their scale
- * factors and per-block sums of squares; with fp8 weights and M >= 48 the
+ * factors and per-block sums of squares; with fp8 weights and M >= 33 the
  * activations split once per call for the block-scale promotion kernel
  * (2 M d bytes of e4m3 codes, 8 bytes per row and 128-deep k block), and at
  * M >= 1024 at least one bf16 copy of the weight (2 d ncols
@@ -145,7 +145,7 @@ size_t fn_workspace_size(int64_t M, int64_t d, int64_t N, fn_wtype wt, int swigl
  *   M == 0 is a no-op.  M <= 64 runs the split-K decode kernel (plus a small
  *   fix-up kernel for the column tiles whose k range it split), larger M the
  *   tensor-core tile kernel; both are deterministic (repeated calls with the
- *   same inputs give the same bits).  fp8 weights from M = 48 (bf16
+ *   same inputs give the same bits).  fp8 weights from M = 33 (bf16
  *   output; NVFP4 and partial outputs from M = 65): the stored
  *   e4m3 codes go to the tensor cores as they are, against the activations
  *   split exactly into two e4m3 parts per row and 128-deep k block (one

@@ -105,9 +105,10 @@ cudaError_t launch_decode_cl(const CallArgs& a, int T, int S);
 size_t tc8_workspace_bytes(int64_t M, int64_t d, bool mx = false);
 cudaError_t launch_tc8(const CallArgs& a);
 // fp8 weights with bf16 output take the promotion kernel from this many rows:
-// at 48 and 64 rows of the fp8 SwiGLU workload (d=5120, N=13824) it ran 5-10 %
-// faster than the split-K decode kernel, at 32 rows 14 % slower.
-constexpr int64_t kFp8PromotionMinM = 48;
+// on the fp8 SwiGLU workload's shape (d=5120, N=13824) it ran 5-10 % faster
+// than the split-K decode kernel at 33, 48 and 64 rows (where the decode
+// kernel pads to 64 rows), 14 % slower at 32.
+constexpr int64_t kFp8PromotionMinM = 33;
 
 // Offline fold and the unfused-chain helper kernels.
 cudaError_t launch_fold_bf16(const void* W0, const void* W1, const float* g, int64_t d, int64_t N, void* Wp,

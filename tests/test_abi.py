@@ -163,12 +163,12 @@ def test_workspace_size_fp8_tile_path(L):
     assert fnb.fn_workspace_size(8192, d, N, fp8, 1) >= 256 + d * 2 * N * 2
     assert fnb.fn_workspace_size(8192, d, N, fp8, 0) > 8 << 20
     assert fnb.fn_workspace_size(65, 1024, 1024, fp8, 0) <= 8 << 20
-    # from 48 rows bf16 output takes the promotion kernel, NVFP4 and partial
+    # from 33 rows bf16 output takes the promotion kernel, NVFP4 and partial
     # outputs still the decode kernel: the size covers both
-    for m in (48, 64):
+    for m in (33, 48, 64):
         need = 256 + 2 * r256(m * d) + 2 * r256((d // 128) * m * 4)
         assert fnb.fn_workspace_size(m, d, N, fp8, 1) >= need
-        assert fnb.fn_workspace_size(m, d, N, fp8, 1) >= fnb.fn_workspace_size(47, d, N, fp8, 1)
+        assert fnb.fn_workspace_size(m, d, N, fp8, 1) >= fnb.fn_workspace_size(32, d, N, fp8, 1)
 
 
 def test_set_debug_validates_keys(L):

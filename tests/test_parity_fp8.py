@@ -101,7 +101,7 @@ def _check(y, ref_stored, ref_exact):
 @pytest.mark.parametrize("M,d,N,swiglu", [
     (5, 256, 384, False),      # decode, odd number of 128-column blocks
     (200, 256, 384, False),    # tile path: the last 256-column tile is half past the weight
-    (40, 384, 256, True),      # decode SwiGLU
+    (40, 384, 256, True),      # SwiGLU at 40 rows: the promotion kernel (33..64 rows)
     (300, 512, 384, True),     # tile SwiGLU, ragged M
     (64, 128, 128, False),     # single k block, single tile
     (129, 640, 640, True),
