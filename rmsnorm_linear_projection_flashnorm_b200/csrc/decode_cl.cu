@@ -433,10 +433,12 @@ bool fits_t(int T, int S, int groups) {
 // The cluster plan: among T in 1..3 boxes per cluster and S in 2..8 CTAs per
 // cluster (T * 64 divisible by S, at most one CTA per 64-deep k block), the
 // one whose busiest CTA streams the fewest weight bytes, with all clusters
-// resident at once.  It is taken when that CTA streams at most 5/4 of what a
-// stream-K CTA does (1x if stream-K would split no tile, so that it needs no
-// fix-up kernel either): the fix-up kernel and the two kernel boundaries it
-// adds cost a fifth to a third of a call at these sizes.
+// resident at once.  It is taken when the extra bytes its busiest CTA streams
+// beyond a stream-K CTA's share cost less than the fix-up kernel and the
+// kernel boundary it saves (about 2 us net of the cluster exchange, i.e. about
+// 13 MB of weight at the HBM rate): best * W <= sk * (W + 13 MB), W the weight
+// bytes; or, if stream-K would split no tile (no fix-up kernel), only when its
+// busiest CTA streams no more.
 bool decode_cl_plan(const CallArgs& a, int& T, int& S) {
   const int mode = a.group_mode & 0xF, want_t = (a.group_mode >> 4) & 0xF, want_s = (a.group_mode >> 8) & 0xF;
   if (mode == 1 || a.wtype != 0 || a.swiglu || a.yq || a.part_out || a.M > 64) return false;
@@ -467,7 +469,9 @@ bool decode_cl_plan(const CallArgs& a, int& T, int& S) {
   const long long grid = total < a.num_sms ? total : a.num_sms;
   const long long sk_load = 2 * ((total + grid - 1) / grid);   // 64-column boxes x k blocks per CTA
   const bool split = dec::any_split_tile(static_cast<int>(grid), total, static_cast<int>(kblocks));
-  return split ? 4 * best <= 5 * sk_load : best <= sk_load;
+  if (!split) return best <= sk_load;
+  const double wbytes = static_cast<double>(a.d) * static_cast<double>(a.ncols) * 2.0;
+  return static_cast<double>(best) * wbytes <= static_cast<double>(sk_load) * (wbytes + 13.0e6);
 }
 
 cudaError_t launch_decode_cl(const CallArgs& a, int T, int S) {
